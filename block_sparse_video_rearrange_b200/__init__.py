@@ -1,0 +1,15 @@
+"""RainFusion v2 block-sparse video attention for B200 (sm_100a).
+
+The compute path lives in the CUDA library `librf.so` (built from `csrc/`),
+reached through `block_sparse_video_rearrange_b200.rf` (ctypes binding).
+`synth` holds the seeded synthetic input generator.
+"""
+import importlib
+
+__all__ = ["rf", "synth"]
+
+
+def __getattr__(name):
+    if name in __all__:
+        return importlib.import_module(f"{__name__}.{name}")
+    raise AttributeError(name)

@@ -1,0 +1,414 @@
+"""CPU ORACLE for the RainFusion v2 block-sparse attention path.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg import this module.  It shares no code with the CUDA path:
+geometry, permutation, pooling, ranking and attention are written out here from
+the pages, in float64, plainly and slowly.
+
+Sources (the web pages this path is described on):
+  [UG]  "RainFusion Attention" user guide (vllm-omni docs): the opening
+        paragraphs, the "Configuration" table and "Geometry handling".
+  [PR]  xllm pull request "feat: add RainFusion sparse attention for wan2.2"
+        (#1867): the change summary.
+  [API] CANN "aclnnRainFusionAttention" API page: "Formula" and the list of
+        constraints.
+  [ABS] "RainFusion2.0: Temporal-Spatial Awareness and Hardware-Efficient
+        Block-wise Sparse Attention", abstract.
+
+Where the pages leave a step open, the reading taken is stated beside the code
+(R1..R14 below are the same readings listed in the design notes).
+
+Pins (what ties this oracle to something other than itself) live in
+tests/test_oracle_*.py: the worked MiniMax geometry from [UG] "Geometry
+handling", a nested-loop construction of the tile order, round trips,
+brute-force top-k by subset enumeration, a library dense attention for
+sparsity 0, element-by-element softmax loops on tiny inputs, and invariants.
+Parity of the *selection* with the pages' own (unpublished) kernel is
+unpinned beyond these invariants: the pages print no worked selection.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Dict, List, Sequence, Tuple
+
+import numpy as np
+
+BLOCK = 128          # [UG] opening paragraph: 128-token key blocks; [PR] pool size 128
+TILE = 8             # [UG] "Geometry handling": grids aligned to 8x8
+DENSE_MIN_BLOCKS = 32  # [UG] opening paragraphs: video segments below 32 blocks run dense
+K_EPS = 1e-6         # R4: guards (1 - 0.8) * 465 = 92.99999... against float noise
+
+
+@dataclasses.dataclass(frozen=True)
+class SeqGeometry:
+    """Derived sizes of one sequence (all counts in tokens unless named *blocks*)."""
+    prefix_len: int   # P: text / condition rows, kept dense
+    t: int
+    h: int
+    w: int
+    h8: int           # 8 * floor(h / 8)
+    w8: int
+    aligned: int      # A = t * h8 * w8 tokens inside whole 8x8 tiles
+    sparse: int       # S = 128 * floor(A / 128) rows in the sparse region
+    promoted: int     # R = t*h*w - S video rows promoted to the dense prefix
+    lp: int           # Lp = P + R, the dense prefix length after promotion
+    length: int       # L = Lp + S
+    n_pb: int         # prefix blocks = ceil(Lp / 128); the last may be partial
+    nb: int           # video (sparse-region) blocks = S / 128
+    ns: int           # first-frame sink blocks
+    k: int            # ranked key blocks kept per sparse query block
+    dense: bool       # the whole sequence runs dense (nb < 32)
+
+    @property
+    def n_blocks(self) -> int:
+        return self.n_pb + self.nb
+
+
+def keep_count(nb: int, sparsity: float) -> int:
+    """Number of ranked video key blocks each sparse query block keeps.
+
+    [UG] "Configuration": sparsity is the nominal fraction of key blocks
+    dropped, in [0, 1], and 0 disables sparsity.  Reading R4: keep
+    ceil((1 - s) * nb) blocks, computed in double with a 1e-6 guard.
+    """
+    if not (0.0 <= sparsity <= 1.0) or not math.isfinite(sparsity):
+        raise ValueError("sparsity must be finite and in [0, 1]")
+    k = math.ceil((1.0 - sparsity) * nb - K_EPS)
+    return max(0, min(nb, k))
+
+
+def geometry(prefix_len: int, t: int, h: int, w: int, sparsity: float) -> SeqGeometry:
+    """Sizes of one sequence under suffix promotion ([UG] "Geometry handling").
+
+    Video tokens inside whole 8x8 tiles are "aligned".  The sparse region is the
+    largest whole number of 128-row blocks of aligned tokens (taken in tile
+    order); every other video token (the ragged edge, plus the aligned tokens
+    past that last whole block, reading R2) is promoted to the dense prefix.
+    Nothing is padded.
+    """
+    h8, w8 = TILE * (h // TILE), TILE * (w // TILE)
+    aligned = t * h8 * w8
+    sparse = BLOCK * (aligned // BLOCK)
+    promoted = t * h * w - sparse
+    lp = prefix_len + promoted
+    nb = sparse // BLOCK
+    n_pb = -(-lp // BLOCK)
+    ns = min(nb, -(-(h8 * w8) // BLOCK))      # blocks holding first-frame tokens (sinks)
+    dense = nb < DENSE_MIN_BLOCKS
+    k = nb if dense else keep_count(nb, sparsity)
+    return SeqGeometry(prefix_len, t, h, w, h8, w8, aligned, sparse, promoted, lp,
+                       lp + sparse, n_pb, nb, ns, k, dense)
+
+
+# --------------------------------------------------------------------------------------
+# Step 1: the token permutation ([UG] opening paragraph and "Geometry handling";
+#         [ABS] insight 2, spatiotemporal-aware token permutation).
+# --------------------------------------------------------------------------------------
+
+def video_order(t: int, h: int, w: int) -> List[int]:
+    """V': video raster indices in rearranged order.
+
+    Reading R1: aligned tokens are ordered by (frame, tile row, tile column,
+    row in tile, column in tile), so every 128-row block is two 8x8 tiles of
+    one frame; ragged tokens follow in raster order.  Built by sorting keys.
+    """
+    h8, w8 = TILE * (h // TILE), TILE * (w // TILE)
+
+    def key(v: int):
+        tau, rem = divmod(v, h * w)
+        y, x = divmod(rem, w)
+        if y < h8 and x < w8:
+            return (0, tau, y // TILE, x // TILE, y % TILE, x % TILE)
+        return (1, v, 0, 0, 0, 0)
+
+    return sorted(range(t * h * w), key=key)
+
+
+def permutation(g: SeqGeometry) -> np.ndarray:
+    """src[r] = original row of rearranged row r, for one sequence.
+
+    Original rows are [text 0..P-1 | video raster].  Rearranged rows are
+    [text (original order) | promoted | sparse], reading R3: promoted rows sit
+    right after the text and join the always-kept prefix.
+    """
+    vp = video_order(g.t, g.h, g.w)
+    sparse, promoted = vp[:g.sparse], vp[g.sparse:]
+    P = g.prefix_len
+    src = list(range(P)) + [P + v for v in promoted] + [P + v for v in sparse]
+    return np.asarray(src, dtype=np.int64)
+
+
+def rearrange_rows(x: np.ndarray, src: np.ndarray) -> np.ndarray:
+    """Rearranged sequence: row r takes original row src[r] (rows on axis -2)."""
+    return x[..., src, :]
+
+
+def inverse_rows(y: np.ndarray, src: np.ndarray) -> np.ndarray:
+    """Inverse permutation ([PR] inverse rearrange): O[src[r]] = O'[r]."""
+    out = np.empty_like(y)
+    out[..., src, :] = y
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# Step 2: block-mean pooling ([UG] opening paragraph; [ABS] insight 1).
+# --------------------------------------------------------------------------------------
+
+def block_rows(g: SeqGeometry, b: int) -> range:
+    """Rows of block b of one rearranged sequence.
+
+    Blocks 0..n_pb-1 tile the dense prefix from row 0 (the last may be
+    partial, [API] constraints: ceiling division); blocks n_pb.. tile the
+    sparse region from row Lp.
+    """
+    if b < g.n_pb:
+        return range(BLOCK * b, min(BLOCK * (b + 1), g.lp))
+    i = b - g.n_pb
+    return range(g.lp + BLOCK * i, g.lp + BLOCK * (i + 1))
+
+
+def block_means(x_r: np.ndarray, g: SeqGeometry) -> np.ndarray:
+    """[nb, D] float64 means of each sparse-region block of one head's rows x_r [L, D]."""
+    out = np.zeros((g.nb, x_r.shape[-1]), dtype=np.float64)
+    for i in range(g.nb):
+        rows = block_rows(g, g.n_pb + i)
+        out[i] = np.asarray(x_r[rows.start:rows.stop], dtype=np.float64).mean(axis=0)
+    return out
+
+
+# --------------------------------------------------------------------------------------
+# Step 3: per-query-block ranking and selection ([UG] opening paragraphs and
+#         "Configuration"; [API] selectIdx / selectNum constraints).
+# --------------------------------------------------------------------------------------
+
+def topk_blocks(scores: np.ndarray, k: int) -> List[int]:
+    """Indices of the k best scores: higher score first, lower index on ties (R9)."""
+    order = sorted(range(len(scores)), key=lambda j: (-float(scores[j]), j))
+    return order[:k]
+
+
+def select_sequence(qbar: np.ndarray, kbar: np.ndarray, g: SeqGeometry) -> Tuple[np.ndarray, np.ndarray]:
+    """selectIdx [n_blocks, N1, n_blocks] (-1 padded) and selectNum [n_blocks, N1] for one sequence.
+
+    qbar: [N1, nb, D], kbar: [N2, nb, D] float64 block means.
+    * Prefix query blocks and first-frame query blocks are dense ([UG]: prefix
+      rows and first-frame blocks remain dense; reading R6).
+    * Every other video query block i on head n ranks video key blocks j by
+      the plain dot product of block means, qbar[n, i] . kbar[n // G, j]
+      (reading R7; GQA head grouping R8), keeps the top k, adds the
+      first-frame sinks (reading R5: sinks do not count toward k), and always
+      keeps every prefix block ([UG]: prefix rows are dense).
+    * A row lists kept blocks in ascending order, prefix blocks first, padded
+      with -1 ([API]: invalid slots are -1).
+    """
+    n1, n2 = qbar.shape[0], kbar.shape[0]
+    G = n1 // n2
+    nblk = g.n_blocks
+    idx = np.full((nblk, n1, nblk), -1, dtype=np.int32)
+    num = np.zeros((nblk, n1), dtype=np.int32)
+    everything = list(range(nblk))
+    for n in range(n1):
+        scores = qbar[n] @ kbar[n // G].T          # [nb, nb]: scores[i, j] = qbar_i . kbar_j
+        for qb in range(nblk):
+            i = qb - g.n_pb
+            if g.dense or qb < g.n_pb or i < g.ns:
+                row = everything
+            else:
+                keep = set(topk_blocks(scores[i], g.k)) | set(range(g.ns))
+                row = list(range(g.n_pb)) + [g.n_pb + j for j in sorted(keep)]
+            idx[qb, n, :len(row)] = row
+            num[qb, n] = len(row)
+    return idx, num
+
+
+# --------------------------------------------------------------------------------------
+# Step 4: block-sparse attention ([API] "Formula": Softmax(scale * Q K^T + mask) V,
+#         restricted to the key blocks each query block selected).
+# --------------------------------------------------------------------------------------
+
+def attend_query_block(q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray, g: SeqGeometry,
+                       qb: int, key_blocks: Sequence[int], scale: float) -> np.ndarray:
+    """float64 output rows of query block qb of one head.
+
+    The keys are the union of the rows of the listed blocks (-1 entries are
+    ignored); the only mask is that rows past the dense prefix end do not
+    belong to the last prefix block (reading R10: no user mask).  Logits are
+    formed in float64 from the exact input values, then a max-subtracted
+    softmax, then the weighted sum of values.
+    """
+    qrows = block_rows(g, qb)
+    krows: List[int] = []
+    for b in key_blocks:
+        if b < 0:
+            continue
+        krows.extend(block_rows(g, int(b)))
+    q = np.asarray(q_r[qrows.start:qrows.stop], dtype=np.float64)
+    k = np.asarray(k_r[krows], dtype=np.float64)
+    v = np.asarray(v_r[krows], dtype=np.float64)
+    logits = scale * (q @ k.T)
+    logits -= logits.max(axis=1, keepdims=True)
+    p = np.exp(logits)
+    p /= p.sum(axis=1, keepdims=True)
+    return p @ v
+
+
+# --------------------------------------------------------------------------------------
+# Whole-path helpers over a batch in BNSD or TND layout.
+# --------------------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Problem:
+    """Shapes of one call: per-sequence geometry plus heads and layout."""
+    layout: str                       # "BNSD" or "TND"
+    batch: int                        # BNSD batch size (1 for TND)
+    geoms: List[SeqGeometry]          # one per sequence (BNSD: one, shared by the batch)
+    n1: int
+    n2: int
+    d: int
+
+    def sequences(self) -> List[Tuple[int, SeqGeometry]]:
+        """(sequence id, geometry) in q-block order: BNSD batch elements, or TND sequences."""
+        if self.layout == "BNSD":
+            return [(b, self.geoms[0]) for b in range(self.batch)]
+        return list(enumerate(self.geoms))
+
+    def row_offsets(self) -> List[int]:
+        offs, acc = [], 0
+        for g in self.geoms:
+            offs.append(acc)
+            acc += g.length
+        return offs
+
+    def head_rows(self, x: np.ndarray, seq: int, head: int) -> np.ndarray:
+        """View [L, D] of one sequence and head."""
+        if self.layout == "BNSD":
+            return x[seq, head]
+        off = self.row_offsets()[seq]
+        return x[off:off + self.geoms[seq].length, head, :]
+
+    @property
+    def max_kv_blocks(self) -> int:
+        return max(g.n_blocks for g in self.geoms)
+
+    @property
+    def t_qblk(self) -> int:
+        return sum(g.n_blocks for _, g in self.sequences())
+
+
+def make_problem(layout: str, batch: int, seqs: Sequence[Tuple[int, int, int, int]],
+                 n1: int, n2: int, d: int, sparsity: float) -> Problem:
+    if n1 % n2:
+        raise ValueError("N1 must be a multiple of N2 ([API] constraints)")
+    geoms = [geometry(p, t, h, w, sparsity) for (p, t, h, w) in seqs]
+    return Problem(layout, batch, geoms, n1, n2, d)
+
+
+def rearrange(p: Problem, x: np.ndarray) -> np.ndarray:
+    """Apply the per-sequence permutation to a BNSD [B,N,L,D] or TND [T,N,D] array."""
+    y = np.empty_like(x)
+    if p.layout == "BNSD":
+        src = permutation(p.geoms[0])
+        y[...] = x[:, :, src, :]
+        return y
+    for s, (off, g) in enumerate(zip(p.row_offsets(), p.geoms)):
+        src = permutation(g)
+        y[off:off + g.length] = x[off + src]
+    return y
+
+
+def inverse_rearrange(p: Problem, y: np.ndarray) -> np.ndarray:
+    x = np.empty_like(y)
+    if p.layout == "BNSD":
+        src = permutation(p.geoms[0])
+        x[:, :, src, :] = y
+        return x
+    for off, g in zip(p.row_offsets(), p.geoms):
+        src = permutation(g)
+        x[off + src] = y[off:off + g.length]
+    return x
+
+
+def pooled_means(p: Problem, x_r: np.ndarray, heads: int) -> List[np.ndarray]:
+    """Per sequence, [heads, nb, D] float64 block means of the rearranged x_r."""
+    out = []
+    for s, g in p.sequences():
+        out.append(np.stack([block_means(p.head_rows(x_r, s, n), g) for n in range(heads)])
+                   if g.nb else np.zeros((heads, 0, p.d)))
+    return out
+
+
+def select(p: Problem, qbars: List[np.ndarray], kbars: List[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:
+    """selectIdx [T_qblk, N1, maxKv] and selectNum [T_qblk, N1] over all sequences ([API])."""
+    maxkv = p.max_kv_blocks
+    idx = np.full((p.t_qblk, p.n1, maxkv), -1, dtype=np.int32)
+    num = np.zeros((p.t_qblk, p.n1), dtype=np.int32)
+    t0 = 0
+    for (s, g), qb, kb in zip(p.sequences(), qbars, kbars):
+        i_s, n_s = select_sequence(qb, kb, g)
+        idx[t0:t0 + g.n_blocks, :, :g.n_blocks] = i_s
+        num[t0:t0 + g.n_blocks] = n_s
+        t0 += g.n_blocks
+    return idx, num
+
+
+def qblock_table(p: Problem) -> List[Tuple[int, SeqGeometry, int]]:
+    """For each global query block t: (sequence id, geometry, local block index)."""
+    out = []
+    for s, g in p.sequences():
+        out.extend((s, g, b) for b in range(g.n_blocks))
+    return out
+
+
+def attention(p: Problem, q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray,
+              idx: np.ndarray, num: np.ndarray, scale: float,
+              items: Sequence[Tuple[int, int]] | None = None) -> Dict[Tuple[int, int], np.ndarray]:
+    """float64 output rows for (global q-block, q-head) items (default: all).
+
+    Inputs are float64 arrays in the rearranged layout.  Head n reads key/value
+    head n // G ([API] constraints: N1 = G * N2).
+    """
+    G = p.n1 // p.n2
+    table = qblock_table(p)
+    if items is None:
+        items = [(t, n) for t in range(len(table)) for n in range(p.n1)]
+    out = {}
+    for (t, n) in items:
+        s, g, b = table[t]
+        row = idx[t, n, :num[t, n]]
+        out[(t, n)] = attend_query_block(p.head_rows(q_r, s, n), p.head_rows(k_r, s, n // G),
+                                         p.head_rows(v_r, s, n // G), g, b, row, scale)
+    return out
+
+
+def assemble_output(p: Problem, parts: Dict[Tuple[int, int], np.ndarray], like: np.ndarray) -> np.ndarray:
+    """Scatter per-(q-block, head) rows into a rearranged-layout float64 array shaped like `like`."""
+    o = np.full(like.shape, np.nan, dtype=np.float64)
+    table = qblock_table(p)
+    for (t, n), rows in parts.items():
+        s, g, b = table[t]
+        r = block_rows(g, b)
+        p.head_rows(o, s, n)[r.start:r.stop] = rows
+    return o
+
+
+def run_path(p: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> Dict[str, object]:
+    """Whole path on float64 inputs in original order: permute, pool, select, attend, un-permute."""
+    q_r, k_r, v_r = rearrange(p, q), rearrange(p, k), rearrange(p, v)
+    qbars, kbars = pooled_means(p, q_r, p.n1), pooled_means(p, k_r, p.n2)
+    idx, num = select(p, qbars, kbars)
+    o_r = assemble_output(p, attention(p, q_r, k_r, v_r, idx, num, scale), q_r)
+    return dict(q_r=q_r, k_r=k_r, v_r=v_r, qbar=qbars, kbar=kbars, idx=idx, num=num,
+                o_r=o_r, o=inverse_rearrange(p, o_r))
+
+
+def kept_flops(p: Problem, idx: np.ndarray, num: np.ndarray) -> int:
+    """4 * D * (query rows) * (valid key rows) summed over selected (q-block, head, key block)."""
+    table = qblock_table(p)
+    total = 0
+    for t, (s, g, b) in enumerate(table):
+        mq = len(block_rows(g, b))
+        for n in range(p.n1):
+            kv = sum(len(block_rows(g, int(j))) for j in idx[t, n, :num[t, n]])
+            total += 4 * p.d * mq * kv
+    return total

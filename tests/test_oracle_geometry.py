@@ -1,0 +1,146 @@
+"""Pins for the oracle's geometry and permutation (CPU only).
+
+The worked MiniMax example comes from the "RainFusion Attention" user guide,
+section "Geometry handling"; everything else is brute force or a closed form.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+from oracle import rainfusion as rf
+from tests.conftest import read_golden
+
+
+def test_minimax_geometry_matches_worked_example():
+    gold = read_golden("minimax_geometry.txt")
+    g = rf.geometry(256, gold["grid_t"], gold["grid_h"], gold["grid_w"], 0.8)
+    assert g.t * g.h * g.w == gold["video_rows"]
+    assert g.promoted == gold["promoted_rows"]
+    assert g.sparse == gold["sparse_rows"]
+    assert g.nb == gold["sparse_blocks"]
+    src = rf.permutation(g)
+    # The promoted rows are real video rows placed in the prefix, right after the text.
+    promoted_src = src[256:256 + g.promoted]
+    assert np.all(promoted_src >= 256)
+    assert len(promoted_src) == gold["promoted_rows"]
+
+
+def _nested_loop_video_order(t, h, w):
+    """Tile order written as explicit loops: frame, tile row, tile column, row, column."""
+    h8, w8 = 8 * (h // 8), 8 * (w // 8)
+    order = []
+    for tau in range(t):
+        for hb in range(h8 // 8):
+            for wb in range(w8 // 8):
+                for hi in range(8):
+                    for wi in range(8):
+                        order.append(tau * h * w + (8 * hb + hi) * w + 8 * wb + wi)
+    for tau in range(t):
+        for y in range(h):
+            for x in range(w):
+                if y >= h8 or x >= w8:
+                    order.append(tau * h * w + y * w + x)
+    return order
+
+
+@pytest.mark.parametrize("t,h,w", [(1, 8, 8), (2, 16, 24), (3, 13, 21), (2, 30, 52), (1, 7, 9), (4, 5, 40)])
+def test_video_order_equals_nested_loops(t, h, w):
+    assert rf.video_order(t, h, w) == _nested_loop_video_order(t, h, w)
+
+
+@pytest.mark.parametrize("p,t,h,w", [(128, 9, 16, 32), (512, 3, 30, 52), (0, 2, 24, 42), (7, 1, 5, 5),
+                                     (384, 2, 24, 40), (1, 3, 17, 9)])
+def test_permutation_is_bijection_and_round_trips(p, t, h, w):
+    g = rf.geometry(p, t, h, w, 0.8)
+    src = rf.permutation(g)
+    assert g.length == p + t * h * w
+    assert sorted(src.tolist()) == list(range(g.length))
+    x = np.random.default_rng(0).standard_normal((2, g.length, 3))
+    y = rf.rearrange_rows(x, src)
+    assert np.array_equal(rf.inverse_rows(y, src), x)
+    # text stays first, in its original order
+    assert np.array_equal(src[:p], np.arange(p))
+
+
+def test_aligned_blocks_are_two_adjacent_tiles_of_one_frame():
+    # grid with an even number of tile columns: each 128-row block = 2 whole 8x8 tiles
+    p, t, h, w = 64, 3, 16, 32
+    g = rf.geometry(p, t, h, w, 0.5)
+    src = rf.permutation(g)
+    assert g.promoted == 0 and g.nb == t * h * w // 128
+    for i in range(g.nb):
+        rows = src[g.lp + 128 * i: g.lp + 128 * (i + 1)] - p
+        tau = rows // (h * w)
+        y = (rows % (h * w)) // w
+        x = rows % w
+        assert len(set(tau.tolist())) == 1
+        cells = sorted(set(zip((y // 8).tolist(), (x // 8).tolist())))
+        assert len(cells) == 2 and cells[0][0] == cells[1][0] and cells[1][1] == cells[0][1] + 1
+        assert cells[0][1] % 2 == 0
+
+
+def test_promoted_rows_are_ragged_edge_plus_aligned_leftover():
+    # (21, 24, 40): A = 20,160 = 157.5 blocks, so 64 aligned rows are promoted (reading R2).
+    p, t, h, w = 384, 21, 24, 40
+    g = rf.geometry(p, t, h, w, 0.8)
+    assert (g.aligned, g.sparse, g.promoted, g.nb, g.n_pb, g.lp) == (20160, 20096, 64, 157, 4, 448)
+    src = rf.permutation(g)
+    promoted = (src[p:g.lp] - p).tolist()
+    assert len(promoted) == 64
+    # the leftover is the last whole 8x8 tile of the last frame, in tile order
+    ys = [(v % (h * w)) // w for v in promoted]
+    xs = [v % w for v in promoted]
+    assert all(v // (h * w) == t - 1 for v in promoted)
+    assert set(ys) == set(range(16, 24)) and set(xs) == set(range(32, 40))
+    # ragged grid: promoted = every token outside the 8x8-aligned area, in raster order
+    p, t, h, w = 512, 21, 30, 52
+    g = rf.geometry(p, t, h, w, 0.8)
+    assert (g.h8, g.w8, g.aligned, g.sparse, g.promoted) == (24, 48, 24192, 24192, 8568)
+    assert (g.lp, g.n_pb, g.nb, g.ns) == (9080, 71, 189, 9)
+    src = rf.permutation(g)
+    promoted = (src[p:g.lp] - p).tolist()
+    raster_ragged = [v for v in range(t * h * w) if (v % (h * w)) // w >= 24 or v % w >= 48]
+    assert promoted == raster_ragged
+
+
+def test_tiny_and_config_counts():
+    g = rf.geometry(128, 9, 16, 32, 0.8)
+    assert (g.sparse, g.nb, g.ns, g.promoted, g.n_pb, g.length) == (4608, 36, 4, 0, 1, 4736)
+    g = rf.geometry(512, 21, 48, 80, 0.8)
+    assert (g.nb, g.ns, g.n_pb, g.length, g.k) == (630, 30, 4, 81152, 126)
+    g = rf.geometry(256, 13, 32, 48, 0.8)
+    assert (g.nb, g.ns, g.n_pb, g.promoted) == (156, 12, 2, 0)
+
+
+def test_sink_blocks_cover_exactly_the_first_frame():
+    for (p, t, h, w) in [(128, 9, 16, 32), (256, 62, 24, 42), (512, 21, 30, 52), (0, 3, 8, 8)]:
+        g = rf.geometry(p, t, h, w, 0.8)
+        src = rf.permutation(g)
+        frame = (src[g.lp:] - p) // (h * w)          # frame of every sparse row
+        first_frame_blocks = {i // 128 for i in np.nonzero(frame == 0)[0].tolist()}
+        assert first_frame_blocks == set(range(g.ns))
+
+
+@pytest.mark.parametrize("nb", [32, 36, 189, 465, 630])
+def test_keep_count_closed_forms(nb):
+    assert rf.keep_count(nb, 0.0) == nb          # sparsity 0 disables sparsity
+    assert rf.keep_count(nb, 1.0) == 0
+    prev = nb
+    for s in np.linspace(0, 1, 21):
+        k = rf.keep_count(nb, float(s))
+        assert k <= prev
+        prev = k
+        # nominal: the dropped fraction is s up to one block
+        assert abs((nb - k) / nb - s) <= 1.0 / nb + 1e-12
+    with pytest.raises(ValueError):
+        rf.keep_count(nb, 1.5)
+    with pytest.raises(ValueError):
+        rf.keep_count(nb, float("nan"))
+
+
+def test_short_video_runs_dense():
+    g = rf.geometry(64, 2, 16, 16, 0.9)             # 512 video tokens = 4 blocks < 32
+    assert g.dense and g.k == g.nb
+    g = rf.geometry(64, 8, 16, 32, 0.9)             # 32 blocks: not dense
+    assert not g.dense and g.nb == 32
