@@ -1,0 +1,282 @@
+// Device-side helpers: token permutation index math and sm_100a PTX wrappers
+// (mbarrier, TMA, tcgen05).  Included by the .cu files only.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rf_internal.h"
+
+// ---------------------------------------------------------------------------
+// Geometry on the device
+// ---------------------------------------------------------------------------
+
+// Sequence instance holding global query block `tb` (instances are few; a
+// linear scan is cheaper than a table lookup through memory).
+__device__ __forceinline__ int rf_seq_of_qblk(const RfGeomDev& g, int tb) {
+  int s = 0;
+#pragma unroll 1
+  for (int i = 1; i < g.n_seqs; ++i)
+    if (tb >= g.seq[i].qblk_off) s = i;
+  return s;
+}
+
+// Element offset of (instance s, head n, row r) in a tensor with `heads` heads.
+__device__ __forceinline__ size_t rf_row_offset(const RfGeomDev& g, const RfSeqDev& s, int heads,
+                                                int n, int r) {
+  if (g.layout == RF_LAYOUT_BNSD)
+    return (((size_t)s.batch_idx * heads + n) * (size_t)s.L + (size_t)r) * (size_t)g.d;
+  return (((size_t)s.row_off + (size_t)r) * heads + n) * (size_t)g.d;
+}
+
+// First row and row count of local block b (prefix blocks tile [0, Lp) with a
+// possibly partial last block; sparse blocks tile [Lp, L) exactly).
+__host__ __device__ __forceinline__ void rf_block_span(const RfSeqDev& s, int b, int& r0, int& nrows) {
+  if (b < s.n_pb) {
+    r0 = b * RF_BLOCK;
+    nrows = (s.Lp - r0) < RF_BLOCK ? (s.Lp - r0) : RF_BLOCK;
+  } else {
+    r0 = s.Lp + (b - s.n_pb) * RF_BLOCK;
+    nrows = RF_BLOCK;
+  }
+}
+
+// Original (input-order) row of rearranged row r of one sequence.
+//   rearranged = [text | promoted | sparse]; the video part follows V', the
+//   video tokens in tile order: aligned tokens by (frame, tile row, tile col,
+//   row in tile, col in tile), then the ragged tokens in raster order.
+//   Sparse rows are V'[0, S); promoted rows are V'[S, t*h*w).
+__host__ __device__ __forceinline__ int rf_orig_row(const RfSeqDev& s, int r) {
+  if (r < s.P) return r;
+  int v = (r < s.Lp) ? (s.S + (r - s.P)) : (r - s.Lp);
+  int y, x, f;
+  if (v < s.A) {
+    const int frame = s.h8 * s.w8;
+    f = v / frame;
+    const int rem = v - f * frame;
+    const int tile = rem >> 6, within = rem & 63;
+    const int tiles_per_row = s.w8 >> 3;
+    const int hb = tile / tiles_per_row, wb = tile - hb * tiles_per_row;
+    y = (hb << 3) + (within >> 3);
+    x = (wb << 3) + (within & 7);
+  } else {
+    const int q = v - s.A;
+    const int per = s.h * s.w - s.h8 * s.w8;  // ragged tokens per frame (> 0 here)
+    f = q / per;
+    const int q2 = q - f * per;
+    const int rw = s.w - s.w8;                 // ragged columns in the top h8 rows
+    const int top = s.h8 * rw;
+    if (q2 < top) {
+      y = q2 / rw;
+      x = s.w8 + (q2 - y * rw);
+    } else {
+      const int q3 = q2 - top;
+      y = s.h8 + q3 / s.w;
+      x = q3 - (y - s.h8) * s.w;
+    }
+  }
+  return s.P + (f * s.h + y) * s.w + x;
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers (sm_100a)
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t rf_smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t rf_globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of barrier `bar` to complete, for at most
+// RF_WAIT_LIMIT_NS; gives up early once *abort is set.  Returns false when it
+// gave up (the caller records it and unwinds).
+#define RF_WAIT_LIMIT_NS 1000000000ull
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = rf_globaltimer();
+#pragma unroll 1
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (rf_globaltimer() - t0 > RF_WAIT_LIMIT_NS) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const void* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
+}
+
+// 3-D tiled TMA load into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, uint32_t bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation issued so far by this thread completes.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f16, fp32 accumulate.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16, fp32 accumulate.
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float rf_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two floats to packed 16-bit (lo = a, hi = b), round to nearest even.
+template <bool kBf16>
+__device__ __forceinline__ uint32_t rf_pack2(float a, float b) {
+  uint32_t r;
+  if (kBf16)
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  else
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// UMMA (tcgen05) descriptors
+// ---------------------------------------------------------------------------
+
+// Shared-memory matrix descriptor for a 128-byte-swizzled tile (1024-byte
+// aligned atoms of 8 rows x 128 bytes).  lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;  // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::f16 with fp32 accumulation.
+//   fmt: 0 = f16, 1 = bf16; b_mn_major: B operand stored N-contiguous.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(uint32_t fmt, uint32_t m, uint32_t n,
+                                                      uint32_t b_mn_major) {
+  return (1u << 4)             // D format: f32
+         | (fmt << 7)          // A format
+         | (fmt << 10)         // B format
+         | (0u << 15)          // A K-major
+         | (b_mn_major << 16)  // B major
+         | ((n >> 3) << 17) | ((m >> 4) << 24);
+}

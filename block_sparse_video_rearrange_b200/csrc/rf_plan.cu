@@ -1,0 +1,382 @@
+// librf host side: plan creation and validation (the first phase of the
+// two-phase call on the "aclnnRainFusionAttention" API page), workspace
+// layout, status reporting and the whole-path entry point.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+
+#include "rf_device.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Number of ranked key blocks a sparse query block keeps: ceil((1 - s) * nb),
+// with a 1e-6 guard so that (1 - 0.8) * 465 = 92.999... rounds to 93
+// ("RainFusion Attention" user guide, "Configuration": nominal dropped fraction).
+int keep_count(int nb, double sparsity) {
+  double k = std::ceil((1.0 - sparsity) * (double)nb - 1e-6);
+  if (k < 0) k = 0;
+  if (k > nb) k = nb;
+  return (int)k;
+}
+
+// Sizes of one sequence under suffix promotion ("RainFusion Attention" user
+// guide, "Geometry handling"): the sparse region is the largest whole number of
+// 128-row blocks of tokens inside whole 8x8 tiles; every other video token is
+// promoted into the always-dense prefix.
+RfSeqDev seq_geometry(const rf_seq_geom_t& s, double sparsity) {
+  RfSeqDev d;
+  std::memset(&d, 0, sizeof(d));
+  d.P = s.prefix_len;
+  d.t = s.t;
+  d.h = s.h;
+  d.w = s.w;
+  d.h8 = 8 * (s.h / 8);
+  d.w8 = 8 * (s.w / 8);
+  d.A = s.t * d.h8 * d.w8;
+  d.nb = d.A / RF_BLOCK;
+  d.S = d.nb * RF_BLOCK;
+  d.L = s.prefix_len + s.t * s.h * s.w;
+  d.Lp = d.L - d.S;
+  d.n_pb = (d.Lp + RF_BLOCK - 1) / RF_BLOCK;
+  int first_frame = d.h8 * d.w8;
+  d.ns = (first_frame + RF_BLOCK - 1) / RF_BLOCK;
+  if (d.ns > d.nb) d.ns = d.nb;
+  d.dense = d.nb < RF_DENSE_MIN_BLOCKS ? 1 : 0;
+  d.k = d.dense ? d.nb : keep_count(d.nb, sparsity);
+  return d;
+}
+
+}  // namespace
+
+rf_status_t rf_fail(rf_status_t st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+rf_status_t rf_check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return rf_fail(RF_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  return RF_OK;
+}
+
+rf_status_t rf_require_device() {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return rf_fail(RF_ERR_UNSUPPORTED_DEVICE, std::string("no CUDA device: ") + cudaGetErrorString(e));
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return rf_fail(RF_ERR_UNSUPPORTED_DEVICE, "cannot query the device's compute capability");
+  }
+  if (major != 10 || minor != 0)
+    return rf_fail(RF_ERR_UNSUPPORTED_DEVICE,
+                   "librf is built for sm_100a (B200); device is sm_" + std::to_string(major) +
+                       std::to_string(minor));
+  return RF_OK;
+}
+
+extern "C" {
+
+const char* rf_status_string(rf_status_t s) {
+  switch (s) {
+    case RF_OK: return "ok";
+    case RF_ERR_INVALID_ARG: return "invalid argument";
+    case RF_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs sm_100)";
+    case RF_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case RF_ERR_CUDA: return "CUDA error";
+    case RF_ERR_DEVICE_FAULT: return "device-side fault recorded (bad selectIdx entry or expired wait)";
+    case RF_ERR_UNSUPPORTED: return "supported by the method but not built";
+  }
+  return "unknown status";
+}
+
+const char* rf_last_error(void) { return g_last_error.c_str(); }
+
+rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch, int32_t n1,
+                           int32_t n2, int32_t d, rf_layout_t layout, rf_dtype_t dtype,
+                           double sparsity, int32_t block_q, int32_t block_kv, rf_plan_t** out) {
+  g_last_error.clear();
+  if (!out || !seqs) return rf_fail(RF_ERR_INVALID_ARG, "null seqs or out");
+  if (layout != RF_LAYOUT_BNSD && layout != RF_LAYOUT_TND)
+    return rf_fail(RF_ERR_INVALID_ARG, "layout must be BNSD or TND");
+  if (dtype != RF_BF16 && dtype != RF_FP16)
+    return rf_fail(RF_ERR_INVALID_ARG, "dtype must be bf16 or fp16");
+  if (!(sparsity >= 0.0 && sparsity <= 1.0) || !std::isfinite(sparsity))
+    return rf_fail(RF_ERR_INVALID_ARG, "sparsity must be finite and in [0, 1]");
+  if (block_q <= 0 || block_kv <= 0)
+    return rf_fail(RF_ERR_INVALID_ARG, "blockShape entries must be > 0");
+  if (block_q != RF_BLOCK || block_kv != RF_BLOCK)
+    return rf_fail(RF_ERR_UNSUPPORTED, "only 128 x 128 blocks are built");
+  if (n1 <= 0 || n2 <= 0 || n1 % n2 != 0)
+    return rf_fail(RF_ERR_INVALID_ARG, "heads: need n1 > 0, n2 > 0 and n1 % n2 == 0");
+  if (d <= 0) return rf_fail(RF_ERR_INVALID_ARG, "head dim must be > 0");
+  if (d != 64 && d != 128) return rf_fail(RF_ERR_UNSUPPORTED, "head dim must be 64 or 128");
+  if (layout == RF_LAYOUT_BNSD) {
+    if (n_seqs != 1) return rf_fail(RF_ERR_INVALID_ARG, "BNSD takes exactly one geometry");
+    if (batch < 1 || batch > RF_MAX_SEQS)
+      return rf_fail(RF_ERR_INVALID_ARG, "BNSD batch must be in [1, 32]");
+  } else {
+    if (batch != 1) return rf_fail(RF_ERR_INVALID_ARG, "TND requires batch == 1");
+    if (n_seqs < 1 || n_seqs > RF_MAX_SEQS)
+      return rf_fail(RF_ERR_INVALID_ARG, "TND takes 1..32 sequences");
+  }
+  for (int i = 0; i < n_seqs; ++i) {
+    const rf_seq_geom_t& s = seqs[i];
+    if (s.prefix_len < 0 || s.t < 0 || s.h < 0 || s.w < 0)
+      return rf_fail(RF_ERR_INVALID_ARG, "negative geometry");
+    int64_t len = (int64_t)s.prefix_len + (int64_t)s.t * s.h * s.w;
+    if (len <= 0) return rf_fail(RF_ERR_INVALID_ARG, "empty sequence");
+    if (len > (1ll << 30)) return rf_fail(RF_ERR_INVALID_ARG, "sequence too long");
+  }
+
+  rf_plan* p = new (std::nothrow) rf_plan();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "out of host memory");
+  std::memset(&p->g, 0, sizeof(p->g));
+  p->layout = layout;
+  p->dtype = dtype;
+  p->sparsity = sparsity;
+  p->batch = batch;
+  p->n_user_seqs = n_seqs;
+  RfGeomDev& g = p->g;
+  g.layout = layout;
+  g.n1 = n1;
+  g.n2 = n2;
+  g.d = d;
+  g.n_seqs = layout == RF_LAYOUT_BNSD ? batch : n_seqs;
+
+  int64_t rows = 0, qblk = 0, pooled = 0, scores = 0, flops = 0;
+  int max_kv = 0, max_nb = 0;
+  for (int i = 0; i < g.n_seqs; ++i) {
+    const rf_seq_geom_t& src = seqs[layout == RF_LAYOUT_BNSD ? 0 : i];
+    RfSeqDev s = seq_geometry(src, sparsity);
+    s.batch_idx = layout == RF_LAYOUT_BNSD ? i : 0;
+    s.row_off = layout == RF_LAYOUT_BNSD ? 0 : rows;
+    s.qblk_off = (int)qblk;
+    s.pool_off = (int)pooled;
+    s.score_off = scores;
+    g.seq[i] = s;
+    int nblk = s.n_pb + s.nb;
+    if (nblk > max_kv) max_kv = nblk;
+    if (s.nb > max_nb) max_nb = s.nb;
+    rows += s.L;
+    qblk += nblk;
+    pooled += s.nb;
+    if (!s.dense) scores += (int64_t)n1 * s.nb * s.nb;
+    flops += 4ll * d * (int64_t)s.L * s.L * n1;
+    if (layout == RF_LAYOUT_TND || i == 0) {
+      rf_seq_info_t inf;
+      inf.row_offset = s.row_off;
+      inf.length = s.L;
+      inf.lp = s.Lp;
+      inf.sparse = s.S;
+      inf.promoted = (int64_t)s.L - s.P - s.S;
+      inf.n_pb = s.n_pb;
+      inf.nb = s.nb;
+      inf.ns = s.ns;
+      inf.k = s.k;
+      inf.qblk_offset = s.qblk_off;
+      inf.dense = s.dense;
+      p->info.push_back(inf);
+    }
+  }
+  if (max_kv > RF_MAX_KV_LIST || max_nb > RF_MAX_NB) {
+    delete p;
+    return rf_fail(RF_ERR_UNSUPPORTED, "a sequence has more than 2048 blocks");
+  }
+  if (qblk * n1 > (1ll << 31) - 1) {
+    delete p;
+    return rf_fail(RF_ERR_INVALID_ARG, "too many query blocks");
+  }
+  g.t_qblk = (int)qblk;
+  g.max_kv = max_kv;
+  g.pooled_total = (int)pooled;
+  g.max_nb = max_nb;
+  p->rows_total = layout == RF_LAYOUT_BNSD ? (int64_t)batch * g.seq[0].L : rows;
+  p->kept_flops_upper = flops;
+
+  // Workspace: [status words | pooled Q fp32 [N1][pooled][D] | pooled K fp32
+  // [N2][pooled][D] | block scores fp32, per non-dense sequence [N1][nb][nb]].
+  int64_t off = 0;
+  p->off_status = off;
+  off += 256;
+  p->off_pq = off;
+  off = align_up(off + (int64_t)n1 * pooled * d * 4, 256);
+  p->off_pk = off;
+  off = align_up(off + (int64_t)n2 * pooled * d * 4, 256);
+  p->off_scores = off;
+  off = align_up(off + scores * 4, 256);
+  p->ws_bytes = off;
+  *out = p;
+  return RF_OK;
+}
+
+rf_status_t rf_plan_info(const rf_plan_t* p, rf_plan_info_t* out) {
+  if (!p || !out) return rf_fail(RF_ERR_INVALID_ARG, "null plan or out");
+  out->rows_total = p->rows_total;
+  out->t_qblk = p->g.t_qblk;
+  out->max_kv_blocks = p->g.max_kv;
+  out->workspace_bytes = p->ws_bytes;
+  out->pooled_blocks = p->g.pooled_total;
+  out->kept_flops_upper = p->kept_flops_upper;
+  out->ws_pooled_q = p->off_pq;
+  out->ws_pooled_k = p->off_pk;
+  out->n_seqs = p->g.n_seqs;
+  out->n1 = p->g.n1;
+  out->n2 = p->g.n2;
+  out->d = p->g.d;
+  return RF_OK;
+}
+
+rf_status_t rf_plan_seq_info(const rf_plan_t* p, int32_t seq, rf_seq_info_t* out) {
+  if (!p || !out) return rf_fail(RF_ERR_INVALID_ARG, "null plan or out");
+  if (seq < 0 || seq >= (int)p->info.size()) return rf_fail(RF_ERR_INVALID_ARG, "seq out of range");
+  *out = p->info[seq];
+  return RF_OK;
+}
+
+void rf_plan_destroy(rf_plan_t* p) { delete p; }
+
+rf_status_t rf_plan_permutation(const rf_plan_t* p, int32_t seq, int64_t* src_rows, int64_t n) {
+  if (!p || !src_rows) return rf_fail(RF_ERR_INVALID_ARG, "null plan or output");
+  if (seq < 0 || seq >= (int)p->info.size()) return rf_fail(RF_ERR_INVALID_ARG, "seq out of range");
+  const RfSeqDev& s = p->g.seq[seq];
+  if (n != s.L) return rf_fail(RF_ERR_INVALID_ARG, "n must equal the sequence length");
+  for (int r = 0; r < s.L; ++r) src_rows[r] = rf_orig_row(s, r);
+  return RF_OK;
+}
+
+static rf_status_t check_ws(const rf_plan_t* p, const void* ws, size_t ws_bytes) {
+  if (!ws) return rf_fail(RF_ERR_INVALID_ARG, "null workspace");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255) != 0)
+    return rf_fail(RF_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((int64_t)ws_bytes < p->ws_bytes)
+    return rf_fail(RF_ERR_WORKSPACE_TOO_SMALL,
+                   "workspace needs " + std::to_string(p->ws_bytes) + " bytes");
+  return RF_OK;
+}
+
+static bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; }
+
+rf_status_t rf_rearrange(const rf_plan_t* p, const void* q, const void* k, const void* v,
+                         void* q_r, void* k_r, void* v_r, void* ws, size_t ws_bytes,
+                         rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (!q || !k || !v || !q_r || !k_r || !v_r) return rf_fail(RF_ERR_INVALID_ARG, "null tensor");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_r) || !aligned16(k_r) ||
+      !aligned16(v_r))
+    return rf_fail(RF_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (q == q_r || k == k_r || v == v_r) return rf_fail(RF_ERR_INVALID_ARG, "in-place rearrange");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  return rf_launch_rearrange(p, q, k, v, q_r, k_r, v_r, ws, (cudaStream_t)stream);
+}
+
+rf_status_t rf_pool_select(const rf_plan_t* p, const void* q_r, const void* k_r,
+                           int32_t* select_idx, int32_t* select_num, void* ws, size_t ws_bytes,
+                           rf_pool_mode_t pool_mode, rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (!select_idx || !select_num) return rf_fail(RF_ERR_INVALID_ARG, "null selectIdx/selectNum");
+  if (pool_mode != RF_POOL_FROM_WS && pool_mode != RF_POOL_RECOMPUTE)
+    return rf_fail(RF_ERR_INVALID_ARG, "bad pool mode");
+  if (pool_mode == RF_POOL_RECOMPUTE &&
+      (!q_r || !k_r || !aligned16(q_r) || !aligned16(k_r)))
+    return rf_fail(RF_ERR_INVALID_ARG, "recompute needs 16-byte aligned q_r and k_r");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  if (pool_mode == RF_POOL_RECOMPUTE) {
+    st = rf_launch_pool(p, q_r, k_r, ws, (cudaStream_t)stream);
+    if (st != RF_OK) return st;
+  }
+  return rf_launch_select(p, select_idx, select_num, ws, (cudaStream_t)stream);
+}
+
+rf_status_t rf_block_sparse_attn(const rf_plan_t* p, const void* q_r, const void* k_r,
+                                 const void* v_r, const int32_t* select_idx,
+                                 const int32_t* select_num, float scale, int32_t inner_precise,
+                                 void* o_r, void* ws, size_t ws_bytes, rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (!q_r || !k_r || !v_r || !o_r || !select_idx || !select_num)
+    return rf_fail(RF_ERR_INVALID_ARG, "null tensor");
+  if (!aligned16(q_r) || !aligned16(k_r) || !aligned16(v_r) || !aligned16(o_r))
+    return rf_fail(RF_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (o_r == q_r || o_r == k_r || o_r == v_r) return rf_fail(RF_ERR_INVALID_ARG, "o_r aliases an input");
+  if (inner_precise != 0 && inner_precise != 1)
+    return rf_fail(RF_ERR_INVALID_ARG, "inner_precise must be 0 or 1");
+  if (inner_precise == 1 && p->dtype == RF_BF16)
+    return rf_fail(RF_ERR_INVALID_ARG, "bf16 inputs allow only inner_precise 0 (fp32 softmax)");
+  if (inner_precise == 1) return rf_fail(RF_ERR_UNSUPPORTED, "fp16 softmax is not built");
+  if (!(scale > 0.0f) || !std::isfinite(scale))
+    return rf_fail(RF_ERR_INVALID_ARG, "scale must be finite and > 0");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  return rf_launch_attn(p, q_r, k_r, v_r, select_idx, select_num, scale, o_r, ws,
+                        (cudaStream_t)stream);
+}
+
+rf_status_t rf_inverse_rearrange(const rf_plan_t* p, const void* o_r, void* o, rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (!o_r || !o) return rf_fail(RF_ERR_INVALID_ARG, "null tensor");
+  if (!aligned16(o_r) || !aligned16(o)) return rf_fail(RF_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (o_r == o) return rf_fail(RF_ERR_INVALID_ARG, "in-place inverse rearrange");
+  rf_status_t st = rf_require_device();
+  if (st != RF_OK) return st;
+  return rf_launch_inverse(p, o_r, o, (cudaStream_t)stream);
+}
+
+rf_status_t rf_forward(const rf_plan_t* p, const void* q, const void* k, const void* v, void* q_r,
+                       void* k_r, void* v_r, int32_t* select_idx, int32_t* select_num, float scale,
+                       void* o_r, void* o, void* ws, size_t ws_bytes, rf_stream_t stream) {
+  rf_status_t st = rf_rearrange(p, q, k, v, q_r, k_r, v_r, ws, ws_bytes, stream);
+  if (st != RF_OK) return st;
+  st = rf_pool_select(p, nullptr, nullptr, select_idx, select_num, ws, ws_bytes, RF_POOL_FROM_WS,
+                      stream);
+  if (st != RF_OK) return st;
+  st = rf_block_sparse_attn(p, q_r, k_r, v_r, select_idx, select_num, scale, 0, o_r, ws, ws_bytes,
+                            stream);
+  if (st != RF_OK) return st;
+  return rf_inverse_rearrange(p, o_r, o, stream);
+}
+
+rf_status_t rf_check_device_status(const rf_plan_t* p, void* ws, uint32_t* flags_out,
+                                   rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p || !ws) return rf_fail(RF_ERR_INVALID_ARG, "null plan or workspace");
+  rf_status_t st = rf_require_device();
+  if (st != RF_OK) return st;
+  uint32_t words[2] = {0, 0};
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t* dev = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p->off_status);
+  if (cudaMemcpyAsync(words, dev, sizeof(words), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess ||
+      cudaMemsetAsync(dev, 0, sizeof(words), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return rf_fail(RF_ERR_CUDA, std::string("status read: ") + cudaGetErrorString(cudaGetLastError()));
+  if (flags_out) {
+    flags_out[0] = words[0];
+    flags_out[1] = words[1];
+  }
+  if (words[0] || words[1])
+    return rf_fail(RF_ERR_DEVICE_FAULT, "bad selectIdx entries: " + std::to_string(words[0]) +
+                                            ", expired waits: " + std::to_string(words[1]));
+  return RF_OK;
+}
+
+}  // extern "C"

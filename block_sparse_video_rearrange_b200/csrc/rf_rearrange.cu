@@ -1,0 +1,168 @@
+// Token permutation kernels (HBM-bound): rf_rearrange for Q, K and V in one
+// launch with the block means of Q and K fused in, the inverse permutation of
+// the output, and a stand-alone block-mean pass over already-rearranged
+// tensors.
+//
+// "RainFusion Attention" user guide, opening paragraph and "Geometry
+// handling": video tokens are arranged in (t, h, w) order with a misaligned
+// suffix promoted to the dense prefix; xllm PR #1867 summary: Q, K and V are
+// permuted in one call and an inverse restores the original order;
+// RainFusion2.0 abstract, insight 1: block means serve as the representative
+// token of each 128-token block.
+//
+// One CTA moves one 128-row block of one head of one tensor: 16-byte vector
+// loads and stores, whole rows per group of D/8 threads, every load of a
+// thread issued before its first store.  The source of a rearranged row is
+// computed from the geometry (no index table in memory).
+#include <cuda_fp16.h>
+
+#include "rf_device.cuh"
+
+namespace {
+
+enum Mode { kRearrange = 0, kInverse = 1, kPoolOnly = 2 };
+
+constexpr int kThreads = 256;
+
+// How the fused pooling reads the two 16-bit values packed in a 32-bit word.
+struct DecodeBf16 {
+  __device__ static float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  __device__ static float hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+};
+struct DecodeF16 {
+  __device__ static float lo(uint32_t w) {
+    return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+  }
+  __device__ static float hi(uint32_t w) {
+    return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+  }
+};
+
+template <int D, int MODE, class Dec>
+__global__ void __launch_bounds__(kThreads)
+    rf_permute_kernel(const RfGeomDev g, const uint4* __restrict__ q, const uint4* __restrict__ k,
+                      const uint4* __restrict__ v, uint4* __restrict__ q_out,
+                      uint4* __restrict__ k_out, uint4* __restrict__ v_out,
+                      float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
+  constexpr int kChunks = D / 8;                  // 16-byte chunks per row
+  constexpr int kRowLanes = kThreads / kChunks;   // rows handled in parallel
+  constexpr int kRowsPerThread = RF_BLOCK / kRowLanes;
+  __shared__ float red[kRowLanes][D + 4];
+
+  const int tb = blockIdx.x % g.t_qblk;           // global block
+  const int th = blockIdx.x / g.t_qblk;           // tensor-major head index
+  int tensor, head, heads;
+  if (MODE == kInverse || th < g.n1) {
+    tensor = 0; head = th; heads = g.n1;
+  } else if (th < g.n1 + g.n2) {
+    tensor = 1; head = th - g.n1; heads = g.n2;
+  } else {
+    tensor = 2; head = th - g.n1 - g.n2; heads = g.n2;
+  }
+  const RfSeqDev& s = g.seq[rf_seq_of_qblk(g, tb)];
+  const int b = tb - s.qblk_off;
+  int r0, nrows;
+  rf_block_span(s, b, r0, nrows);
+  const bool pool = (MODE != kInverse) && tensor < 2 && b >= s.n_pb;
+  if (MODE == kPoolOnly && !pool) return;
+
+  const uint4* src = tensor == 0 ? q : (tensor == 1 ? k : v);
+  uint4* dst = tensor == 0 ? q_out : (tensor == 1 ? k_out : v_out);
+  const int ch = threadIdx.x % kChunks;
+  const int rl = threadIdx.x / kChunks;
+
+  uint4 val[kRowsPerThread];
+#pragma unroll
+  for (int i = 0; i < kRowsPerThread; ++i) {
+    const int rr = rl + i * kRowLanes;
+    val[i] = make_uint4(0, 0, 0, 0);
+    if (rr < nrows) {
+      const int r = r0 + rr;
+      const int from = (MODE == kRearrange) ? rf_orig_row(s, r) : r;
+      val[i] = __ldg(src + rf_row_offset(g, s, heads, head, from) / 8 + ch);
+    }
+  }
+  if (MODE != kPoolOnly) {
+#pragma unroll
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const int rr = rl + i * kRowLanes;
+      if (rr < nrows) {
+        const int r = r0 + rr;
+        const int to = (MODE == kInverse) ? rf_orig_row(s, r) : r;
+        dst[rf_row_offset(g, s, heads, head, to) / 8 + ch] = val[i];
+      }
+    }
+  }
+  if (!pool) return;  // uniform over the CTA
+
+  // Column sums of the block in fp32 and a fixed order (a lane's rows in
+  // order, then the lanes in order), then the mean.
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRowsPerThread; ++i) {
+    const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      acc[2 * c] += Dec::lo(w[c]);
+      acc[2 * c + 1] += Dec::hi(w[c]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float sum = 0.f;
+#pragma unroll 4
+    for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
+    float* out = tensor == 0 ? pooled_q : pooled_k;
+    const size_t idx =
+        ((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x;
+    out[idx] = sum * (1.0f / RF_BLOCK);
+  }
+}
+
+template <int MODE>
+rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v, void* qo,
+                   void* ko, void* vo, void* ws, cudaStream_t st, int tensor_heads) {
+  const RfGeomDev& g = p->g;
+  const long long grid = (long long)g.t_qblk * tensor_heads;
+  if (grid == 0) return RF_OK;
+  if (grid > 0x7FFFFFFFll) return rf_fail(RF_ERR_INVALID_ARG, "grid too large");
+  float* pq = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + p->off_pq) : nullptr;
+  float* pk = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + p->off_pk) : nullptr;
+  const uint4* a = static_cast<const uint4*>(q);
+  const uint4* b = static_cast<const uint4*>(k);
+  const uint4* c = static_cast<const uint4*>(v);
+  uint4* x = static_cast<uint4*>(qo);
+  uint4* y = static_cast<uint4*>(ko);
+  uint4* z = static_cast<uint4*>(vo);
+  const bool bf = p->dtype == RF_BF16;
+  dim3 grd((unsigned)grid), blk(kThreads);
+  if (g.d == 128) {
+    if (bf) rf_permute_kernel<128, MODE, DecodeBf16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
+    else    rf_permute_kernel<128, MODE, DecodeF16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
+  } else {
+    if (bf) rf_permute_kernel<64, MODE, DecodeBf16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
+    else    rf_permute_kernel<64, MODE, DecodeF16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
+  }
+  return rf_check_launch("rf_permute_kernel");
+}
+
+}  // namespace
+
+rf_status_t rf_launch_rearrange(const rf_plan* p, const void* q, const void* k, const void* v,
+                                void* q_r, void* k_r, void* v_r, void* ws, cudaStream_t st) {
+  return launch<kRearrange>(p, q, k, v, q_r, k_r, v_r, ws, st, p->g.n1 + 2 * p->g.n2);
+}
+
+rf_status_t rf_launch_pool(const rf_plan* p, const void* q_r, const void* k_r, void* ws,
+                           cudaStream_t st) {
+  return launch<kPoolOnly>(p, q_r, k_r, nullptr, nullptr, nullptr, nullptr, ws, st,
+                           p->g.n1 + p->g.n2);
+}
+
+rf_status_t rf_launch_inverse(const rf_plan* p, const void* o_r, void* o, cudaStream_t st) {
+  return launch<kInverse>(p, o_r, nullptr, nullptr, o, nullptr, nullptr, nullptr, st, p->g.n1);
+}

@@ -1,0 +1,213 @@
+// Block ranking and selection: selectIdx / selectNum for every (query block,
+// query head).
+//
+// "RainFusion Attention" user guide, opening paragraphs: key blocks are
+// pooled, ranked per query block, and the highest-scoring ones are attended;
+// prefix rows and first-frame blocks stay dense; segments under 32 blocks run
+// dense.  "Configuration": sparsity is the nominal dropped fraction.
+// "aclnnRainFusionAttention" API page, constraints: selectIdx is
+// [T, headNum, maxKvBlockNum] with -1 in unused slots; selectNum is [T, headNum].
+// RainFusion2.0 abstract: block means are the representative tokens; the
+// first frame is a sink.
+//
+// Two kernels:
+//  1. rf_scores_kernel: per sparse sequence and query head n, the fp32 matrix
+//     scores[i][j] = qbar[n][i] . kbar[n / G][j] (64 x 64 tiles, 4 x 4 per
+//     thread, D chunks staged through shared memory).
+//  2. rf_topk_kernel: one warp per selectIdx row.  Keys are the scores mapped
+//     to order-preserving 32-bit integers, held in registers (32 lanes x M).
+//     A 32-step radix select finds the k-th largest key; ties at the
+//     threshold go to the lowest block index; sinks are added; the row is
+//     written in ascending order with a ballot prefix sum.  No sorting, no
+//     shared memory, no atomics.
+#include "rf_device.cuh"
+
+namespace {
+
+constexpr int kTile = 64;
+constexpr int kKc = 32;
+
+__global__ void __launch_bounds__(256)
+    rf_scores_kernel(const RfGeomDev g, const float* __restrict__ pq, const float* __restrict__ pk,
+                     float* __restrict__ scores) {
+  __shared__ float As[kKc][kTile + 4];
+  __shared__ float Bs[kKc][kTile + 4];
+  // Decode blockIdx.x into (instance, head, tile row, tile col) over the
+  // non-dense instances in order.
+  int rem = blockIdx.x;
+  int si = -1, tiles = 0;
+  for (int i = 0; i < g.n_seqs; ++i) {
+    const RfSeqDev& s = g.seq[i];
+    if (s.dense) continue;
+    const int tn = (s.nb + kTile - 1) / kTile;
+    const int cnt = g.n1 * tn * tn;
+    if (rem < cnt) { si = i; tiles = tn; break; }
+    rem -= cnt;
+  }
+  if (si < 0) return;
+  const RfSeqDev& s = g.seq[si];
+  const int n = rem / (tiles * tiles);
+  const int tr = (rem / tiles) % tiles;
+  const int tc = rem % tiles;
+  const int gk = n / (g.n1 / g.n2);
+  const float* A = pq + ((size_t)n * g.pooled_total + s.pool_off) * g.d;
+  const float* B = pk + ((size_t)gk * g.pooled_total + s.pool_off) * g.d;
+  const int i0 = tr * kTile, j0 = tc * kTile;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+
+  for (int k0 = 0; k0 < g.d; k0 += kKc) {
+    // 64 rows x 32 k of A and of B: 512 float4 each, 2 per thread.
+#pragma unroll
+    for (int rep = 0; rep < 2; ++rep) {
+      const int e = threadIdx.x + rep * 256;
+      const int row = e / (kKc / 4), c4 = e % (kKc / 4);
+      float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
+      if (i0 + row < s.nb) va = *reinterpret_cast<const float4*>(A + (size_t)(i0 + row) * g.d + k0 + 4 * c4);
+      if (j0 + row < s.nb) vb = *reinterpret_cast<const float4*>(B + (size_t)(j0 + row) * g.d + k0 + 4 * c4);
+      As[4 * c4 + 0][row] = va.x; As[4 * c4 + 1][row] = va.y;
+      As[4 * c4 + 2][row] = va.z; As[4 * c4 + 3][row] = va.w;
+      Bs[4 * c4 + 0][row] = vb.x; Bs[4 * c4 + 1][row] = vb.y;
+      Bs[4 * c4 + 2][row] = vb.z; Bs[4 * c4 + 3][row] = vb.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < kKc; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+    }
+    __syncthreads();
+  }
+  float* C = scores + s.score_off + (size_t)n * s.nb * s.nb;
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    const int i = i0 + ty * 4 + x;
+    if (i >= s.nb) continue;
+#pragma unroll
+    for (int y = 0; y < 4; ++y) {
+      const int j = j0 + tx * 4 + y;
+      if (j < s.nb) C[(size_t)i * s.nb + j] = acc[x][y];
+    }
+  }
+}
+
+// Order-preserving map of a float to uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t rf_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int M>  // keys per lane: nb <= 32 * M
+__global__ void __launch_bounds__(256)
+    rf_topk_kernel(const RfGeomDev g, const float* __restrict__ scores, int32_t* __restrict__ sel_idx,
+                   int32_t* __restrict__ sel_num) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long rows = (long long)g.t_qblk * g.n1;
+  if (warp >= rows) return;
+  const int tb = warp / g.n1, n = warp % g.n1;
+  const RfSeqDev& s = g.seq[rf_seq_of_qblk(g, tb)];
+  const int b = tb - s.qblk_off;
+  const int nblk = s.n_pb + s.nb;
+  int32_t* row = sel_idx + (size_t)warp * g.max_kv;
+  const int i = b - s.n_pb;
+
+  if (s.dense || b < s.n_pb || i < s.ns || s.k >= s.nb) {
+    for (int c = lane; c < g.max_kv; c += 32) row[c] = c < nblk ? c : -1;
+    if (lane == 0) sel_num[warp] = nblk;
+    return;
+  }
+
+  // Keys of this row; absent slots hold 0, below every real key.
+  const float* sc = scores + s.score_off + ((size_t)n * s.nb + i) * s.nb;
+  uint32_t key[M];
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const int j = lane + 32 * m;
+    key[m] = j < s.nb ? rf_key(sc[j]) : 0u;
+  }
+  const int k = s.k;
+  unsigned long long sel = 0;  // bit m: block lane + 32m is kept
+  if (k > 0) {
+    // Largest T with #{key >= T} >= k, one bit at a time from the top.
+    uint32_t T = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int cnt = 0;
+#pragma unroll
+      for (int m = 0; m < M; ++m) cnt += key[m] >= cand ? 1 : 0;
+      cnt = __reduce_add_sync(0xffffffffu, cnt);
+      if (cnt >= k) T = cand;
+    }
+    int gt = 0;
+#pragma unroll
+    for (int m = 0; m < M; ++m) gt += key[m] > T ? 1 : 0;
+    gt = __reduce_add_sync(0xffffffffu, gt);
+    int need = k - gt;  // keys equal to T to take, lowest block index first
+    const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+      const bool eq = key[m] == T && key[m] != 0u;
+      const uint32_t ball = __ballot_sync(0xffffffffu, eq);
+      const bool take_eq = eq && (int)__popc(ball & lt_mask) < need;
+      need -= min(need, (int)__popc(ball));
+      if (key[m] > T || take_eq) sel |= 1ull << m;
+    }
+  }
+  // First-frame sinks.
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+    if (lane + 32 * m < s.ns) sel |= 1ull << m;
+
+  for (int c = lane; c < s.n_pb; c += 32) row[c] = c;
+  int pos = s.n_pb;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+#pragma unroll
+  for (int m = 0; m < M; ++m) {
+    const bool on = (sel >> m) & 1ull;
+    const uint32_t ball = __ballot_sync(0xffffffffu, on);
+    if (on) row[pos + __popc(ball & lt_mask)] = s.n_pb + lane + 32 * m;
+    pos += __popc(ball);
+  }
+  for (int c = pos + lane; c < g.max_kv; c += 32) row[c] = -1;
+  if (lane == 0) sel_num[warp] = pos;
+}
+
+}  // namespace
+
+rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_num, void* ws,
+                             cudaStream_t st) {
+  const RfGeomDev& g = p->g;
+  const float* pq = reinterpret_cast<const float*>(static_cast<char*>(ws) + p->off_pq);
+  const float* pk = reinterpret_cast<const float*>(static_cast<char*>(ws) + p->off_pk);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + p->off_scores);
+  long long tiles = 0;
+  for (int i = 0; i < g.n_seqs; ++i) {
+    if (g.seq[i].dense) continue;
+    const long long tn = (g.seq[i].nb + kTile - 1) / kTile;
+    tiles += (long long)g.n1 * tn * tn;
+  }
+  if (tiles > 0) {
+    rf_scores_kernel<<<(unsigned)tiles, 256, 0, st>>>(g, pq, pk, scores);
+    rf_status_t s = rf_check_launch("rf_scores_kernel");
+    if (s != RF_OK) return s;
+  }
+  const long long rows = (long long)g.t_qblk * g.n1;
+  if (rows == 0) return RF_OK;
+  const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
+  if (g.max_nb <= 256)       rf_topk_kernel<8><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nb <= 512)  rf_topk_kernel<16><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nb <= 1024) rf_topk_kernel<32><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else                       rf_topk_kernel<64><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  return rf_check_launch("rf_topk_kernel");
+}

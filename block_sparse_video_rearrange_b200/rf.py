@@ -1,0 +1,315 @@
+"""ctypes binding of librf (include/rf.h): argument marshalling only.
+
+Every step of the path runs in librf's CUDA kernels; this module only turns
+torch tensors into device pointers and the current stream into a
+cudaStream_t.  Importing it fails loudly when librf.so has not been built.
+
+Pages the method is described on: the "RainFusion Attention" user guide
+(vllm-omni docs), the xllm pull request "feat: add RainFusion sparse
+attention for wan2.2" (#1867), the CANN "aclnnRainFusionAttention" API page
+and the RainFusion2.0 abstract.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librf.so")
+
+RF_OK = 0
+STATUS_NAMES = {0: "RF_OK", 1: "RF_ERR_INVALID_ARG", 2: "RF_ERR_UNSUPPORTED_DEVICE",
+                3: "RF_ERR_WORKSPACE_TOO_SMALL", 4: "RF_ERR_CUDA", 5: "RF_ERR_DEVICE_FAULT",
+                6: "RF_ERR_UNSUPPORTED"}
+LAYOUTS = {"BNSD": 0, "TND": 1}
+DTYPES = {"bf16": 0, "fp16": 1}
+TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
+POOL_MODES = {"from_ws": 0, "recompute": 1}
+
+EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange", "rf_pool_select",
+            "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
+            "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation")
+
+
+class RfError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
+        self.status = status
+
+
+class SeqGeom(ctypes.Structure):
+    _fields_ = [("prefix_len", ctypes.c_int32), ("t", ctypes.c_int32), ("h", ctypes.c_int32),
+                ("w", ctypes.c_int32)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("rows_total", ctypes.c_int64), ("t_qblk", ctypes.c_int64),
+                ("max_kv_blocks", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64),
+                ("pooled_blocks", ctypes.c_int64), ("kept_flops_upper", ctypes.c_int64),
+                ("ws_pooled_q", ctypes.c_int64), ("ws_pooled_k", ctypes.c_int64),
+                ("n_seqs", ctypes.c_int32), ("n1", ctypes.c_int32), ("n2", ctypes.c_int32),
+                ("d", ctypes.c_int32)]
+
+
+class SeqInfo(ctypes.Structure):
+    _fields_ = [("row_offset", ctypes.c_int64), ("length", ctypes.c_int64), ("lp", ctypes.c_int64),
+                ("sparse", ctypes.c_int64), ("promoted", ctypes.c_int64), ("n_pb", ctypes.c_int32),
+                ("nb", ctypes.c_int32), ("ns", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("qblk_offset", ctypes.c_int32), ("dense", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m block_sparse_video_rearrange_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "rf_plan_create": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
+                           i32, i32, ctypes.POINTER(vp)],
+        "rf_plan_info": [vp, ctypes.POINTER(PlanInfo)],
+        "rf_plan_seq_info": [vp, i32, ctypes.POINTER(SeqInfo)],
+        "rf_rearrange": [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "rf_pool_select": [vp, vp, vp, vp, vp, vp, sz, i32, vp],
+        "rf_block_sparse_attn": [vp, vp, vp, vp, vp, vp, ctypes.c_float, i32, vp, vp, sz, vp],
+        "rf_inverse_rearrange": [vp, vp, vp, vp],
+        "rf_forward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp],
+        "rf_check_device_status": [vp, vp, ctypes.POINTER(ctypes.c_uint32), vp],
+        "rf_plan_destroy": [vp],
+        "rf_plan_permutation": [vp, i32, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64],
+        "rf_status_string": [i32],
+        "rf_last_error": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int32
+    lib.rf_plan_destroy.restype = None
+    lib.rf_status_string.restype = ctypes.c_char_p
+    lib.rf_last_error.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != RF_OK:
+        raise RfError(status, where, _lib.rf_last_error().decode())
+
+
+class Plan:
+    """Host-side plan: validated geometry and sizes (no device memory)."""
+
+    def __init__(self, seqs: Sequence[Tuple[int, int, int, int]], n1: int, n2: int, d: int,
+                 layout: str = "BNSD", dtype: str = "bf16", sparsity: float = 0.8, batch: int = 1,
+                 block_q: int = 128, block_kv: int = 128):
+        arr = (SeqGeom * max(1, len(seqs)))(*[SeqGeom(*map(int, s)) for s in seqs])
+        handle = ctypes.c_void_p()
+        _check(_lib.rf_plan_create(arr, len(seqs), batch, n1, n2, d, LAYOUTS[layout], DTYPES[dtype],
+                                   float(sparsity), block_q, block_kv, ctypes.byref(handle)),
+               "rf_plan_create")
+        self._h = handle
+        self._lib = _lib  # kept so that destruction at interpreter exit still finds it
+        self.layout, self.dtype, self.sparsity, self.batch = layout, dtype, float(sparsity), batch
+        self.seqs = [tuple(map(int, s)) for s in seqs]
+        info = PlanInfo()
+        _check(_lib.rf_plan_info(self._h, ctypes.byref(info)), "rf_plan_info")
+        self.info = info
+        self.seq_info: List[SeqInfo] = []
+        for i in range(len(seqs)):
+            si = SeqInfo()
+            _check(_lib.rf_plan_seq_info(self._h, i, ctypes.byref(si)), "rf_plan_seq_info")
+            self.seq_info.append(si)
+
+    def __del__(self):
+        h, lib_ = getattr(self, "_h", None), getattr(self, "_lib", None)
+        if h is not None and h.value and lib_ is not None:
+            lib_.rf_plan_destroy(h)
+            self._h = None
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._h
+
+    @property
+    def n1(self) -> int:
+        return self.info.n1
+
+    @property
+    def n2(self) -> int:
+        return self.info.n2
+
+    @property
+    def d(self) -> int:
+        return self.info.d
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return TORCH_DTYPES[self.dtype]
+
+    def tensor_shape(self, heads: int) -> Tuple[int, ...]:
+        if self.layout == "BNSD":
+            return (self.batch, heads, int(self.seq_info[0].length), self.d)
+        return (int(self.info.rows_total), heads, self.d)
+
+    def select_shapes(self) -> Tuple[Tuple[int, int, int], Tuple[int, int]]:
+        t, n, m = int(self.info.t_qblk), self.n1, int(self.info.max_kv_blocks)
+        return (t, n, m), (t, n)
+
+    @property
+    def workspace_bytes(self) -> int:
+        return int(self.info.workspace_bytes)
+
+    def permutation(self, seq: int = 0):
+        """src[r] = original row of rearranged row r of sequence `seq` (host-side arithmetic)."""
+        import numpy as np
+        n = int(self.seq_info[seq].length)
+        out = np.empty(n, dtype=np.int64)
+        _check(_lib.rf_plan_permutation(self._h, seq, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n),
+               "rf_plan_permutation")
+        return out
+
+    def seq_info_all(self) -> List[SeqInfo]:
+        """Geometry of every sequence instance in q-block order (BNSD: one per batch element)."""
+        if self.layout == "TND":
+            return list(self.seq_info)
+        out = []
+        base = self.seq_info[0]
+        nblk = base.n_pb + base.nb
+        for bi in range(self.batch):
+            si = SeqInfo()
+            ctypes.pointer(si)[0] = base
+            si.qblk_offset = bi * nblk
+            out.append(si)
+        return out
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("librf takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _expect(t: torch.Tensor, shape, dtype, name: str) -> None:
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype:
+        raise ValueError(f"{name}: expected {tuple(shape)} {dtype}, got {tuple(t.shape)} {t.dtype}")
+
+
+def rearrange(plan: Plan, q, k, v, q_r, k_r, v_r, ws, stream=None) -> None:
+    """Permute Q, K, V (one launch) and write the block means of Q and K into ws."""
+    for t, h, nm in ((q, plan.n1, "q"), (k, plan.n2, "k"), (v, plan.n2, "v"), (q_r, plan.n1, "q_r"),
+                     (k_r, plan.n2, "k_r"), (v_r, plan.n2, "v_r")):
+        _expect(t, plan.tensor_shape(h), plan.torch_dtype, nm)
+    _check(_lib.rf_rearrange(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(q_r), _ptr(k_r), _ptr(v_r),
+                             _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "rf_rearrange")
+
+
+def pool_select(plan: Plan, q_r, k_r, select_idx, select_num, ws, pool_mode: str = "from_ws",
+                stream=None) -> None:
+    """Rank key blocks per query block; write selectIdx / selectNum."""
+    si, sn = plan.select_shapes()
+    _expect(select_idx, si, torch.int32, "select_idx")
+    _expect(select_num, sn, torch.int32, "select_num")
+    _check(_lib.rf_pool_select(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(select_idx), _ptr(select_num),
+                               _ptr(ws), ws.numel() * ws.element_size(), POOL_MODES[pool_mode],
+                               _stream(stream)), "rf_pool_select")
+
+
+def block_sparse_attn(plan: Plan, q_r, k_r, v_r, select_idx, select_num, scale: float, o_r, ws,
+                      inner_precise: int = 0, stream=None) -> None:
+    """Softmax(scale Q K^T) V over the selected blocks (rearranged order)."""
+    _expect(o_r, plan.tensor_shape(plan.n1), plan.torch_dtype, "o_r")
+    _check(_lib.rf_block_sparse_attn(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(v_r), _ptr(select_idx),
+                                     _ptr(select_num), float(scale), int(inner_precise), _ptr(o_r),
+                                     _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "rf_block_sparse_attn")
+
+
+def inverse_rearrange(plan: Plan, o_r, o, stream=None) -> None:
+    """Scatter the output back to the original token order."""
+    _expect(o, plan.tensor_shape(plan.n1), plan.torch_dtype, "o")
+    _check(_lib.rf_inverse_rearrange(plan.handle, _ptr(o_r), _ptr(o), _stream(stream)),
+           "rf_inverse_rearrange")
+
+
+def check_device_status(plan: Plan, ws, stream=None) -> Tuple[int, Tuple[int, int]]:
+    """Synchronise, read and clear the kernels' status words: (status, (bad_index, timeouts))."""
+    flags = (ctypes.c_uint32 * 2)()
+    st = _lib.rf_check_device_status(plan.handle, _ptr(ws), flags, _stream(stream))
+    return st, (int(flags[0]), int(flags[1]))
+
+
+class Buffers:
+    """Device intermediates and outputs of one path invocation (owned by torch)."""
+
+    def __init__(self, plan: Plan, device="cuda"):
+        shp_q, shp_kv = plan.tensor_shape(plan.n1), plan.tensor_shape(plan.n2)
+        dt = plan.torch_dtype
+        self.q_r = torch.empty(shp_q, dtype=dt, device=device)
+        self.k_r = torch.empty(shp_kv, dtype=dt, device=device)
+        self.v_r = torch.empty(shp_kv, dtype=dt, device=device)
+        self.o_r = torch.empty(shp_q, dtype=dt, device=device)
+        self.o = torch.empty(shp_q, dtype=dt, device=device)
+        si, sn = plan.select_shapes()
+        self.select_idx = torch.empty(si, dtype=torch.int32, device=device)
+        self.select_num = torch.empty(sn, dtype=torch.int32, device=device)
+        self.ws = torch.zeros(max(256, plan.workspace_bytes) // 4 + 64, dtype=torch.int32, device=device)
+
+
+def forward(plan: Plan, q, k, v, bufs: Buffers, scale: Optional[float] = None, stream=None) -> torch.Tensor:
+    """The whole path in one librf call; returns bufs.o (original token order)."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(plan.d)
+    for t, h, nm in ((q, plan.n1, "q"), (k, plan.n2, "k"), (v, plan.n2, "v")):
+        _expect(t, plan.tensor_shape(h), plan.torch_dtype, nm)
+    b = bufs
+    _check(_lib.rf_forward(plan.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(b.q_r), _ptr(b.k_r), _ptr(b.v_r),
+                           _ptr(b.select_idx), _ptr(b.select_num), float(scale), _ptr(b.o_r), _ptr(b.o),
+                           _ptr(b.ws), b.ws.numel() * b.ws.element_size(), _stream(stream)), "rf_forward")
+    return b.o
+
+
+def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         seqs: Sequence[Tuple[int, int, int, int]], sparsity: float = 0.8,
+                         layout: str = "BNSD", scale: Optional[float] = None,
+                         plan: Optional[Plan] = None, bufs: Optional[Buffers] = None) -> torch.Tensor:
+    """User-level call: RainFusion v2 block-sparse attention of q, k, v (original token order).
+
+    q, k, v may live on the host (pinned or not) or on the GPU; the result is
+    returned on the device the inputs came from.  BNSD: q [B, N1, L, D],
+    k/v [B, N2, L, D]; TND: q [T, N1, D], k/v [T, N2, D].  `seqs` holds one
+    (prefix_len, t, h, w) per sequence (BNSD: one for the whole batch).
+    """
+    dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[q.dtype]
+    if plan is None:
+        if layout == "BNSD":
+            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[3], "BNSD", dtype, sparsity, batch=q.shape[0])
+        else:
+            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[2], "TND", dtype, sparsity)
+    host = not q.is_cuda
+    dev = torch.device("cuda", torch.cuda.current_device()) if host else q.device
+    if bufs is None:
+        bufs = Buffers(plan, dev)
+    qd, kd, vd = (x.to(dev, non_blocking=True) for x in (q, k, v))
+    out = forward(plan, qd.contiguous(), kd.contiguous(), vd.contiguous(), bufs, scale)
+    if host:
+        res = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        res.copy_(out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        return res
+    return out

@@ -1,0 +1,241 @@
+/*
+ * rf.h -- C ABI of librf, the B200 (sm_100a) RainFusion v2 block-sparse
+ * video attention path.
+ *
+ * The path (one call each, all asynchronous on the caller's stream):
+ *   rf_rearrange          (t,h,w) token permutation with suffix promotion, for
+ *                         Q, K and V in one launch; also writes the 128-row
+ *                         block means of Q and K into the workspace.
+ *   rf_pool_select        per-query-block ranking of key blocks by block-mean
+ *                         scores; writes selectIdx / selectNum.
+ *   rf_block_sparse_attn  Softmax(scale * Q K^T) V over the selected blocks,
+ *                         fp32 softmax, tcgen05 tensor cores.
+ *   rf_inverse_rearrange  scatter of the output back to the original order.
+ *   rf_forward            the four steps above in one call.
+ *
+ * Sources (the web pages the method is described on):
+ *   [UG]  "RainFusion Attention" user guide (vllm-omni docs): opening
+ *         paragraphs, "Configuration", "Geometry handling".
+ *   [PR]  xllm pull request "feat: add RainFusion sparse attention for
+ *         wan2.2" (#1867): change summary (rearrange, inverse, QKV in one
+ *         call, round-trip check).
+ *   [API] CANN "aclnnRainFusionAttention" API page: "Formula", the two-phase
+ *         call (workspace size, then execute), and the constraints list.
+ *   [ABS] RainFusion2.0 abstract: block means as representative tokens,
+ *         spatiotemporal token permutation, first-frame sink.
+ *
+ * Conventions (all entry points):
+ *   - Every pointer named q, k, v, *_r, o, select_idx, select_num or ws is a
+ *     DEVICE pointer owned by the caller; the library never frees or keeps it
+ *     beyond the call.  The library owns only the host-side plan.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     enqueue work and return; they do not synchronise (except
+ *     rf_check_device_status).
+ *   - The return value reports host-side validation and launch errors.  A
+ *     call that returns an error enqueued nothing.
+ *   - Device-side problems (an out-of-range selectIdx entry, an expired
+ *     bounded wait) never trap: the kernel records them in the workspace
+ *     status words and skips the offending work; rf_check_device_status
+ *     reports them as RF_ERR_DEVICE_FAULT.
+ *   - Only sm_100 devices are accepted (RF_ERR_UNSUPPORTED_DEVICE
+ *     otherwise), as [UG] "Requirements" has the NPU backend raise on any
+ *     other platform.
+ *
+ * Tensor layouts ([API] "Formula": TND and BNSD):
+ *   BNSD: Q [B, N1, L, D], K/V [B, N2, L, D], every batch element has the
+ *         same geometry (one rf_seq_geom_t).
+ *   TND:  Q [T, N1, D], K/V [T, N2, D]; sequences are packed back to back
+ *         along T in the order given to rf_plan_create.
+ *   All tensors are contiguous, dtype bf16 or fp16 (Q, K and V share it,
+ *   [API] constraints), D in {64, 128}.  Original row order of a sequence:
+ *   [text/condition prefix (prefix_len rows) | video in raster (t, y, x)].
+ *   Rearranged order: [prefix | promoted video rows | sparse video rows in
+ *   8x8-tile order], i.e. Lp = prefix_len + promoted dense rows, then
+ *   nb = S / 128 sparse blocks.
+ */
+#ifndef RF_H_
+#define RF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RF_API __attribute__((visibility("default")))
+#else
+#define RF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* rf_stream_t; /* == cudaStream_t */
+
+typedef enum {
+  RF_OK = 0,
+  RF_ERR_INVALID_ARG = 1,         /* an argument breaks a documented constraint */
+  RF_ERR_UNSUPPORTED_DEVICE = 2,  /* no CUDA device, or not sm_100 */
+  RF_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes < rf_plan_info().workspace_bytes */
+  RF_ERR_CUDA = 4,                /* a CUDA runtime / driver call failed */
+  RF_ERR_DEVICE_FAULT = 5,        /* a kernel recorded a bad index or an expired wait */
+  RF_ERR_UNSUPPORTED = 6          /* allowed by the pages but not built here */
+} rf_status_t;
+
+typedef enum { RF_LAYOUT_BNSD = 0, RF_LAYOUT_TND = 1 } rf_layout_t;
+typedef enum { RF_BF16 = 0, RF_FP16 = 1 } rf_dtype_t;
+
+/* How rf_pool_select obtains the block means of Q and K. */
+typedef enum {
+  RF_POOL_FROM_WS = 0,   /* use the means rf_rearrange wrote into this same workspace */
+  RF_POOL_RECOMPUTE = 1  /* recompute them from q_r / k_r first */
+} rf_pool_mode_t;
+
+/* One sequence: text/condition prefix length and video latent grid
+ * ([UG] "Geometry handling").  t, h, w >= 0; prefix_len >= 0; length > 0. */
+typedef struct {
+  int32_t prefix_len;
+  int32_t t, h, w;
+} rf_seq_geom_t;
+
+/* Sizes derived by rf_plan_create (phase one of the two-phase call, [API]). */
+typedef struct {
+  int64_t rows_total;      /* rows per head: BNSD B*L, TND T */
+  int64_t t_qblk;          /* total query blocks over all sequences ([API] selectIdx dim 0) */
+  int64_t max_kv_blocks;   /* selectIdx dim 2 = max over sequences of n_pb + nb */
+  int64_t workspace_bytes; /* device workspace every call below needs */
+  int64_t pooled_blocks;   /* total sparse blocks over sequences (block means per head) */
+  int64_t kept_flops_upper;/* 4*D*rows_q*rows_kv over the maximal selection (for reporting) */
+  int64_t ws_pooled_q;     /* byte offset in ws of the Q block means, fp32 [n1][pooled_blocks][d] */
+  int64_t ws_pooled_k;     /* byte offset in ws of the K block means, fp32 [n2][pooled_blocks][d] */
+  int32_t n_seqs;          /* sequences (BNSD: batch elements) */
+  int32_t n1, n2, d;
+} rf_plan_info_t;
+
+/* Per-sequence geometry under suffix promotion ([UG] "Geometry handling"). */
+typedef struct {
+  int64_t row_offset;  /* first row of the sequence along the row axis (TND T; BNSD 0) */
+  int64_t length;      /* L = prefix_len + t*h*w */
+  int64_t lp;          /* dense prefix rows after promotion */
+  int64_t sparse;      /* S = 128 * nb */
+  int64_t promoted;    /* video rows moved into the dense prefix */
+  int32_t n_pb;        /* prefix blocks = ceil(lp / 128); the last may be partial */
+  int32_t nb;          /* sparse video blocks */
+  int32_t ns;          /* first-frame sink blocks */
+  int32_t k;           /* ranked key blocks kept per sparse query block */
+  int32_t qblk_offset; /* first global query block of this sequence */
+  int32_t dense;       /* 1: the sequence runs dense (nb < 32, [UG]) */
+} rf_seq_info_t;
+
+typedef struct rf_plan rf_plan_t;
+
+/* Phase one: validate the problem and derive every size.  Host only; no
+ * device is touched, so it also works on a machine without a GPU.
+ *   seqs/n_seqs : sequences.  BNSD requires n_seqs == 1 (batch gives the count);
+ *                 TND requires batch == 1 and 1 <= n_seqs <= 32.
+ *   batch       : BNSD batch size B (1..32).
+ *   n1, n2      : query and key/value heads, n1 % n2 == 0 ([API] GQA constraint).
+ *   d           : head dim, 64 or 128 (others: RF_ERR_UNSUPPORTED).
+ *   sparsity    : finite, in [0, 1] ([UG] "Configuration"); 0 keeps every block.
+ *   block_q, block_kv : [API] blockShape; must be > 0; only 128 x 128 is built
+ *                 (others: RF_ERR_UNSUPPORTED).
+ *   out         : receives the plan; free with rf_plan_destroy.
+ * Errors: RF_ERR_INVALID_ARG for a broken constraint (out untouched). */
+RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
+                           int32_t n1, int32_t n2, int32_t d, rf_layout_t layout,
+                           rf_dtype_t dtype, double sparsity, int32_t block_q,
+                           int32_t block_kv, rf_plan_t** out);
+
+/* Sizes of a plan (host only). */
+RF_API rf_status_t rf_plan_info(const rf_plan_t* plan, rf_plan_info_t* out);
+
+/* Geometry of sequence `seq` (0 <= seq < n_seqs; host only). */
+RF_API rf_status_t rf_plan_seq_info(const rf_plan_t* plan, int32_t seq, rf_seq_info_t* out);
+
+/* Step 1 ([UG] opening paragraph and "Geometry handling"; [PR] rearrange with
+ * QKV in one call; [ABS] spatiotemporal token permutation).
+ * q, k, v     : inputs in original order (layout above).
+ * q_r,k_r,v_r : outputs, same shapes, rows permuted within each sequence.
+ *               Must not alias the inputs.
+ * ws          : workspace of at least workspace_bytes; receives the fp32
+ *               block means of the sparse blocks of Q and K (the fused
+ *               pooling of [UG] opening paragraph / [ABS] insight 1).
+ * Bit-exact copy; deterministic. */
+RF_API rf_status_t rf_rearrange(const rf_plan_t* plan, const void* q, const void* k, const void* v,
+                         void* q_r, void* k_r, void* v_r, void* ws, size_t ws_bytes,
+                         rf_stream_t stream);
+
+/* Steps 2-3 ([UG] opening paragraphs and "Configuration"; [API] selectIdx and
+ * selectNum constraints).
+ * q_r, k_r    : rearranged Q and K (read only when pool_mode == RF_POOL_RECOMPUTE;
+ *               may be NULL otherwise).
+ * select_idx  : int32 [t_qblk, n1, max_kv_blocks]; per row the kept key blocks of
+ *               the query block's own sequence, ascending, prefix blocks first,
+ *               padded with -1 ([API]).
+ * select_num  : int32 [t_qblk, n1], the number of valid entries per row.
+ * Selection: prefix and first-frame query blocks keep everything; other
+ * video query blocks keep every prefix block, the first-frame sink blocks,
+ * and the k key blocks with the highest block-mean dot product (ties: lower
+ * block index), k = ceil((1 - sparsity) * nb).  Sequences with nb < 32 are
+ * dense.  Deterministic (fp32 scores, no atomics). */
+RF_API rf_status_t rf_pool_select(const rf_plan_t* plan, const void* q_r, const void* k_r,
+                           int32_t* select_idx, int32_t* select_num, void* ws,
+                           size_t ws_bytes, rf_pool_mode_t pool_mode, rf_stream_t stream);
+
+/* Step 4 ([API] "Formula": Softmax(scale * Q K^T + atten_mask) V, restricted to
+ * the key blocks of selectIdx; no user mask is consumed, the only masked keys
+ * are rows past the dense prefix in its last, partial block).
+ * q_r,k_r,v_r : rearranged inputs; o_r : output, same shape as q_r (may not alias).
+ * select_idx, select_num : as written by rf_pool_select (any valid selection is
+ *               accepted: entries in [0, n_pb + nb) of the row's sequence; the
+ *               first select_num entries are used; out-of-range entries are
+ *               skipped and flagged in ws).
+ * scale       : > 0 and finite (typically 1/sqrt(D)).
+ * inner_precise : 0 = fp32 softmax ([API]: 1 = fp16 softmax is not allowed with
+ *               bf16 and is not built here: RF_ERR_UNSUPPORTED).
+ * Deterministic: no split-K, no atomics. */
+RF_API rf_status_t rf_block_sparse_attn(const rf_plan_t* plan, const void* q_r, const void* k_r,
+                                 const void* v_r, const int32_t* select_idx,
+                                 const int32_t* select_num, float scale,
+                                 int32_t inner_precise, void* o_r, void* ws, size_t ws_bytes,
+                                 rf_stream_t stream);
+
+/* Step 5 ([PR] inverse rearrange): o[orig(r)] = o_r[r] for every row r.
+ * o_r : [.., N1 heads ..] in rearranged order; o : same shape, original order. */
+RF_API rf_status_t rf_inverse_rearrange(const rf_plan_t* plan, const void* o_r, void* o,
+                                 rf_stream_t stream);
+
+/* The whole path: rf_rearrange, rf_pool_select (RF_POOL_FROM_WS),
+ * rf_block_sparse_attn (inner_precise 0) and rf_inverse_rearrange.
+ * q_r, k_r, v_r, o_r, select_idx, select_num are caller-provided intermediates. */
+RF_API rf_status_t rf_forward(const rf_plan_t* plan, const void* q, const void* k, const void* v,
+                       void* q_r, void* k_r, void* v_r, int32_t* select_idx,
+                       int32_t* select_num, float scale, void* o_r, void* o, void* ws,
+                       size_t ws_bytes, rf_stream_t stream);
+
+/* The token permutation of sequence `seq` (host only, no device needed):
+ * src_rows[r] = original row (within the sequence) of rearranged row r, for
+ * r < length.  n must equal rf_seq_info_t.length.  This is the same index
+ * arithmetic the kernels run ([UG] "Geometry handling"). */
+RF_API rf_status_t rf_plan_permutation(const rf_plan_t* plan, int32_t seq, int64_t* src_rows, int64_t n);
+
+/* Reads and clears the device status words in ws.  Synchronises `stream`.
+ * flags_out (may be NULL) receives the raw words: [0] out-of-range selectIdx
+ * entries seen, [1] expired bounded waits.  Returns RF_ERR_DEVICE_FAULT if
+ * either is non-zero. */
+RF_API rf_status_t rf_check_device_status(const rf_plan_t* plan, void* ws, uint32_t* flags_out,
+                                   rf_stream_t stream);
+
+/* Frees a plan (NULL is a no-op). */
+RF_API void rf_plan_destroy(rf_plan_t* plan);
+
+/* Static description of a status code. */
+RF_API const char* rf_status_string(rf_status_t status);
+
+/* Detail of the last error returned on the calling thread ("" if none). */
+RF_API const char* rf_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RF_H_ */

@@ -183,9 +183,14 @@ def block_means(x_r: np.ndarray, g: SeqGeometry) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 
 def topk_blocks(scores: np.ndarray, k: int) -> List[int]:
-    """Indices of the k best scores: higher score first, lower index on ties (R9)."""
-    order = sorted(range(len(scores)), key=lambda j: (-float(scores[j]), j))
-    return order[:k]
+    """Indices of the k best scores: higher score first, lower index on ties (R9).
+
+    A stable library sort: np.lexsort orders by the last key (descending
+    score), then by the first (ascending block index).
+    """
+    scores = np.asarray(scores, dtype=np.float64)
+    order = np.lexsort((np.arange(len(scores)), -scores))
+    return order[:k].tolist()
 
 
 def select_sequence(qbar: np.ndarray, kbar: np.ndarray, g: SeqGeometry) -> Tuple[np.ndarray, np.ndarray]:

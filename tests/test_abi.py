@@ -1,0 +1,124 @@
+"""C-ABI checks that need no GPU: the library loads, exports what include/rf.h
+declares, validates arguments on the host, and derives the oracle's geometry."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from block_sparse_video_rearrange_b200 import rf, synth
+from oracle import rainfusion as orc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "rf.h")).read()
+    return sorted(set(re.findall(r"RF_API\s+[\w\s\*]+?\b(rf_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(rf.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(rf.EXPORTED)
+
+
+def test_status_strings():
+    for code in range(7):
+        assert rf.lib().rf_status_string(code)
+    assert rf.lib().rf_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("kwargs,status", [
+    (dict(n1=6, n2=4), 1),                     # N1 = G * N2 violated
+    (dict(block_q=0), 1),                      # blockShape entries must be > 0
+    (dict(block_kv=-3), 1),
+    (dict(block_q=64), 6),                     # valid per the pages, not built here
+    (dict(sparsity=1.5), 1),
+    (dict(sparsity=float("nan")), 1),
+    (dict(sparsity=-0.1), 1),
+    (dict(d=96), 6),
+    (dict(d=0), 1),
+    (dict(batch=0), 1),
+    (dict(batch=33), 1),
+    (dict(seqs=[(0, 0, 0, 0)]), 1),            # empty sequence
+    (dict(seqs=[(-1, 2, 8, 8)]), 1),
+    (dict(seqs=[(0, 2, 8, 8), (0, 2, 8, 8)]), 1),  # BNSD takes one geometry
+    (dict(layout="TND", batch=2), 1),
+])
+def test_plan_validation(kwargs, status):
+    args = dict(seqs=[(128, 9, 16, 32)], n1=2, n2=2, d=64, layout="BNSD", dtype="bf16", sparsity=0.8,
+                batch=1, block_q=128, block_kv=128)
+    args.update(kwargs)
+    with pytest.raises(rf.RfError) as e:
+        rf.Plan(**args)
+    assert e.value.status == status
+
+
+@pytest.mark.parametrize("name", sorted(synth.WORKLOADS))
+def test_plan_geometry_matches_oracle(name):
+    w = synth.WORKLOADS[name]
+    seqs = [(s.prefix_len, s.t, s.h, s.w) for s in w.seqs]
+    plan = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch)
+    prob = orc.make_problem(w.layout, w.batch, seqs, w.n1, w.n2, w.d, w.sparsity)
+    assert plan.info.t_qblk == prob.t_qblk
+    assert plan.info.max_kv_blocks == prob.max_kv_blocks
+    row = 0
+    for si, g in zip(plan.seq_info, prob.geoms):
+        assert (si.length, si.lp, si.sparse, si.promoted) == (g.length, g.lp, g.sparse, g.promoted)
+        assert (si.n_pb, si.nb, si.ns, si.k, si.dense) == (g.n_pb, g.nb, g.ns, g.k, int(g.dense))
+        if w.layout == "TND":
+            assert si.row_offset == row
+        row += g.length
+    assert plan.info.rows_total == (prob.geoms[0].length if w.layout == "BNSD" else row)
+
+
+@pytest.mark.parametrize("s", [0.0, 0.5, 0.8, 0.9, 1.0, 0.37])
+def test_keep_count_matches_oracle(s):
+    for nb in (32, 36, 157, 189, 465, 630, 2048):
+        t, h, w = 1, 8, nb * 16   # nb blocks of two 8x8 tiles
+        plan = rf.Plan([(0, t, h, w)], 1, 1, 64, sparsity=s)
+        assert plan.seq_info[0].nb == nb
+        assert plan.seq_info[0].k == orc.keep_count(nb, s)
+
+
+def test_host_validation_runs_before_any_device_call():
+    plan = rf.Plan([(128, 9, 16, 32)], 2, 2, 64)
+    fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: validation fails first
+    # bf16 allows only the fp32 softmax (inner_precise 0)
+    st = rf.lib().rf_block_sparse_attn(plan.handle, fake, fake, fake, fake, fake, ctypes.c_float(0.125), 1,
+                                       ctypes.c_void_p(2 << 20), fake, plan.workspace_bytes, None)
+    assert st == 1
+    st = rf.lib().rf_block_sparse_attn(plan.handle, fake, fake, fake, fake, fake, ctypes.c_float(-1.0), 0,
+                                       ctypes.c_void_p(2 << 20), fake, plan.workspace_bytes, None)
+    assert st == 1
+    # an undersized workspace is rejected before the device is touched
+    st = rf.lib().rf_rearrange(plan.handle, fake, fake, fake, ctypes.c_void_p(2 << 20), ctypes.c_void_p(3 << 20),
+                               ctypes.c_void_p(4 << 20), fake, 16, None)
+    assert st == 3
+    # misaligned tensors
+    st = rf.lib().rf_inverse_rearrange(plan.handle, ctypes.c_void_p((1 << 20) + 2), fake, None)
+    assert st == 1
+
+
+@pytest.mark.parametrize("name", sorted(synth.WORKLOADS))
+def test_kernel_index_math_equals_oracle_permutation(name):
+    """The row mapping the CUDA kernels execute (run here on the host) against the
+    oracle's permutation, which is built by sorting keys."""
+    w = synth.WORKLOADS[name]
+    seqs = [(s.prefix_len, s.t, s.h, s.w) for s in w.seqs]
+    plan = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch)
+    for i, s in enumerate(seqs):
+        g = orc.geometry(*s, w.sparsity)
+        assert np.array_equal(plan.permutation(i), orc.permutation(g))
+
+
+@pytest.mark.parametrize("s", [(77, 9, 17, 33), (0, 6, 24, 40), (200, 10, 19, 21), (5, 3, 7, 9), (1, 2, 8, 8),
+                               (0, 1, 3, 3), (64, 4, 31, 9), (384, 21, 24, 40)])
+def test_kernel_index_math_ragged_cases(s):
+    plan = rf.Plan([s], 1, 1, 64)
+    assert np.array_equal(plan.permutation(0), orc.permutation(orc.geometry(*s, 0.8)))

@@ -1,0 +1,185 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_video_rearrange_b200 import rf, synth
+from oracle import rainfusion as orc
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+W = synth.Workload
+S = synth.SeqSpec
+
+# Small cases the oracle finishes in seconds; each spans several tiles and a ragged tail.
+SMALL = {
+    # the Tiny workload itself (D = 64, aligned grid, 4 sink blocks)
+    "tiny": synth.WORKLOADS["tiny"],
+    # ragged h and w, partial last prefix block (Lp = 518), D = 128
+    "ragged_d128": W("ragged_d128", "BNSD", "bf16", 1, (S(77, 9, 17, 33),), 2, 2, 128, 0.8, 11),
+    # batch of two, D = 64, higher sparsity
+    "batch2_d64": W("batch2_d64", "BNSD", "bf16", 2, (S(128, 9, 16, 32),), 2, 2, 64, 0.9, 12),
+    # varlen TND, fp16, GQA G = 2; the second sequence is short (20 blocks) and runs dense
+    "tnd_gqa_small": W("tnd_gqa_small", "TND", "fp16", 1, (S(64, 9, 16, 32), S(200, 10, 19, 21)),
+                       4, 2, 128, 0.8, 13),
+    # sparsity 0 must equal dense attention
+    "dense": W("dense", "BNSD", "bf16", 1, (S(100, 8, 16, 32),), 2, 1, 128, 0.0, 14),
+    # sparsity 1: prefix + sinks only
+    "s_one": W("s_one", "BNSD", "bf16", 1, (S(40, 9, 16, 32),), 2, 2, 128, 1.0, 15),
+    # no text prefix at all, odd tile column count
+    "no_prefix": W("no_prefix", "BNSD", "fp16", 1, (S(0, 6, 24, 40),), 2, 2, 64, 0.5, 16),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_full_parity(name):
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits)
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 100)
+    err = parity.check_attention(p, w, rbits, gpu)
+    if name == "dense":
+        assert np.all(gpu["num"] == p.geoms[0].n_blocks)
+        # against a library dense attention on the original order, per head
+        q, k, v = (synth.bits_to_float64(x, w.dtype) for x in bits)
+        o = synth.bits_to_float64(gpu["o"], w.dtype)
+        for n in range(w.n1):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(q[0, n]), torch.from_numpy(k[0, n // 2]), torch.from_numpy(v[0, n // 2]),
+                scale=gpu["scale"]).numpy()
+            assert np.max(np.abs(o[0, n] - ref)) <= parity.MAX_ABS
+
+
+def test_pool_recompute_mode_matches_fused_pool():
+    w = SMALL["ragged_d128"]
+    bits = synth.generate_qkv(w)
+    a = parity.run_gpu(w, bits, pool_mode="from_ws")
+    b = parity.run_gpu(w, bits, pool_mode="recompute")
+    assert np.array_equal(a["pooled_q"], b["pooled_q"]) and np.array_equal(a["pooled_k"], b["pooled_k"])
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["num"], b["num"])
+    assert np.array_equal(a["o"], b["o"])
+
+
+def test_deterministic_repeat():
+    w = SMALL["tnd_gqa_small"]
+    bits = synth.generate_qkv(w)
+    a = parity.run_gpu(w, bits)
+    b = parity.run_gpu(w, bits)
+    for key in ("q_r", "idx", "num", "o_r", "o"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_handmade_selection_with_padding_and_bad_entries():
+    """Any valid selectIdx is accepted; -1 slots are skipped; out-of-range entries are
+    skipped and counted in the status words; selectNum 0 gives zeros."""
+    w = SMALL["ragged_d128"]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    g = p.geoms[0]
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity)
+    q, k, v = (parity.to_device(x, w.dtype) for x in bits)
+    b = rf.Buffers(plan)
+    rf.rearrange(plan, q, k, v, b.q_r, b.k_r, b.v_r, b.ws)
+    rng = np.random.default_rng(0)
+    T, N, M = b.select_idx.shape
+    idx = np.full((T, N, M), -1, dtype=np.int32)
+    num = np.zeros((T, N), dtype=np.int32)
+    clean = np.full((T, N, M), -1, dtype=np.int32)
+    clean_num = np.zeros((T, N), dtype=np.int32)
+    bad = 0
+    for t in range(T):
+        for n in range(N):
+            if (t + n) % 7 == 3:
+                continue  # selectNum 0 -> zero output rows
+            chosen = sorted(rng.choice(g.n_blocks, size=int(rng.integers(1, g.n_blocks - 2)), replace=False).tolist())
+            row = list(chosen)
+            if t % 3 == 0:
+                row.insert(1, -1)
+            if t % 5 == 0:
+                row.append(g.n_blocks + 3)   # out of range
+                bad += 1
+            idx[t, n, :len(row)] = row
+            num[t, n] = len(row)
+            clean[t, n, :len(chosen)] = chosen
+            clean_num[t, n] = len(chosen)
+    b.select_idx.copy_(torch.from_numpy(idx))
+    b.select_num.copy_(torch.from_numpy(num))
+    scale = 0.09
+    rf.block_sparse_attn(plan, b.q_r, b.k_r, b.v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
+    st, flags = rf.check_device_status(plan, b.ws)
+    assert st == 5                                      # RF_ERR_DEVICE_FAULT
+    assert flags[0] == bad * 1 and flags[1] == 0
+    st, flags = rf.check_device_status(plan, b.ws)
+    assert st == 0 and flags == (0, 0)                  # cleared
+    gpu = dict(idx=clean, num=clean_num, scale=scale, o_r=parity.to_bits(b.o_r))
+    rbits = [orc.rearrange(p, x) for x in bits]
+    items = [(t, n) for t in range(T) for n in range(N) if clean_num[t, n] > 0]
+    parity.check_attention(p, w, rbits, gpu, items)
+    o_r = synth.bits_to_float64(gpu["o_r"], w.dtype)
+    for t in range(T):
+        for n in range(N):
+            if clean_num[t, n] == 0:
+                r = orc.block_rows(g, t)
+                assert np.all(o_r[0, n, r.start:r.stop] == 0)
+
+
+def test_forward_entry_point_equals_step_calls():
+    w = SMALL["tnd_gqa_small"]
+    bits = synth.generate_qkv(w)
+    steps = parity.run_gpu(w, bits)
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity)
+    b = rf.Buffers(plan)
+    q, k, v = (parity.to_device(x, w.dtype) for x in bits)
+    out = rf.forward(plan, q, k, v, b)
+    torch.cuda.synchronize()
+    assert np.array_equal(parity.to_bits(out), steps["o"])
+
+
+def test_user_call_with_host_tensors():
+    w = SMALL["batch2_d64"]
+    bits = synth.generate_qkv(w)
+    steps = parity.run_gpu(w, bits)
+    q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in bits)
+    out = rf.rainfusion_attention(q, k, v, parity.seqs_of(w), sparsity=w.sparsity)
+    assert not out.is_cuda
+    assert np.array_equal(out.view(torch.int16).numpy().view(np.uint16), steps["o"])
+
+
+# ------------------------------------------------------------------------------------------
+# Full-size workloads in the bench's launch configuration: permutation bit-exact over
+# everything, pooling and selection over every row, attention on sampled items.
+# ------------------------------------------------------------------------------------------
+
+FULL = [("wan", None), ("minimax", 0.8), ("minimax", 0.5), ("minimax", 0.9), ("tnd_gqa", None),
+        ("aligned", 0.8), ("aligned", 0.0)]
+
+
+@pytest.mark.parametrize("name,s", FULL)
+def test_full_size_parity(name, s):
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits)
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 1000), stats
+    items = parity.sample_items(p, np.random.default_rng(7), per_kind=3)
+    parity.check_attention(p, w, rbits, gpu, items)
