@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="profiling only: shrink the layer to this many query heads (G kept)")
     return ap.parse_args()
 
 
@@ -219,6 +221,18 @@ def oracle_step_sample(w, bits, budget_items=24, seed=0):
     return step_s, flops_total, desc, t_front + t_attn
 
 
+def reduce_over_ranks(maxima, sums, device):
+    """Times: the max over ranks (the job ends when the slowest rank does);
+    work: the sum over ranks.  Every rank calls this with the same layout."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(maxima), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor(list(sums), dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()], [float(x) for x in u.tolist()]
+
+
 def oracle_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -239,6 +253,10 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from block_sparse_video_rearrange_b200 import synth
     w = synth.workload(args.workload, args.sparsity)
+    if args.heads:
+        g = w.n1 // w.n2
+        w = synth.Workload(w.name, w.layout, w.dtype, w.batch, w.seqs, args.heads, max(1, args.heads // g), w.d,
+                           w.sparsity, w.seed)
     sparsity = w.sparsity
 
     if args.impl == "reference":
@@ -346,14 +364,10 @@ def main():
     ms_step = total_ms / args.steps
     attn_ms = float(np.mean(per[:, 2]))
     if world > 1:
-        t = torch.tensor([ms_step, attn_ms, e2e[0] if e2e else 0.0], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, attn_ms, e2e_max = (float(x) for x in t.tolist())
+        (ms_step, attn_ms, e2e_max), (flops_all,) = reduce_over_ranks(
+            [ms_step, attn_ms, e2e[0] if e2e else 0.0], [float(flops)], dev)
         if e2e:
             e2e = (e2e_max, e2e[1], e2e[2])
-        ft = torch.tensor([float(flops)], device=dev, dtype=torch.float64)
-        dist.all_reduce(ft, op=dist.ReduceOp.SUM)
-        flops_all = float(ft.item())
     else:
         flops_all = float(flops)
 
@@ -379,7 +393,8 @@ def main():
             "vs_baseline": None,
             "dtype": "bf16" if w.dtype == "bf16" else "fp16",
             "data": "synthetic (seeded smooth-field + noise per 8x8 cell; no real activations available)",
-            "config": {"workload": WORKLOAD_DESC[w.name.split("@")[0]], "sparsity": sparsity,
+            "config": {"workload": WORKLOAD_DESC[w.name.split("@")[0]] + (f" [reduced to {w.n1} heads]" if args.heads else ""),
+                       "sparsity": sparsity,
                        "global_batch": w.batch * world, "seq_len": int(plan.info.rows_total),
                        "parallelism": f"independent layer per GPU x{world}",
                        "l2": "inputs larger than L2 (Q+K+V %.2f GB vs 126 MB)" % (
