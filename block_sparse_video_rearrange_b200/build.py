@@ -21,12 +21,13 @@ def nvcc_path():
     raise RuntimeError("nvcc not found")
 
 
-def command(ptxas_verbose=False, out=LIB):
+def command(ptxas_verbose=False, out=LIB, defines=()):
     cmd = [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo",
            "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
            "-shared", "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-o", out]
     if ptxas_verbose:
         cmd += ["-Xptxas", "-v"]
+    cmd += [f"-D{d}" for d in defines]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
     return cmd
 

@@ -14,19 +14,33 @@
 // its query blocks run, and within a head the dense query blocks (prefix,
 // first frame) come first.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax + epilogue; thread = query row = TMEM lane
-//   warp 4     TMA producer: Q once, then K_j / V_j of each selected block
-//              through a kStages-deep ring of shared-memory stages
-//   warp 5     TMEM allocation and the single-thread tcgen05.mma issue
-// TMEM columns: S double buffer [0,128) and [128,256) (fp32 128 x 128), O at
-// [256, 256 + D) (fp32 128 x D).  P is written back over its own S buffer as
-// packed 16-bit pairs and is the A operand (from TMEM) of O += P V.
-// Pipeline per selected block j:
-//   MMA:     S_{j+1} = Q K_{j+1}^T   (overlaps softmax of block j)
-//   softmax: m, p = exp2(s * scale * log2e - m), l += sum p, P_j -> TMEM;
-//            O is rescaled only when the row max grows by more than 2^8
-//   MMA:     O += P_j V_j
+// Warp roles (384 threads = three warpgroups):
+//   warps 0-3  softmax warpgroup 0: the even-numbered selected blocks
+//   warps 4-7  softmax warpgroup 1: the odd-numbered selected blocks
+//              (thread = query row = TMEM lane in both groups)
+//   warp 8     TMA producer: Q once, then K_j / V_j of each selected block;
+//              block j always uses shared-memory stage j % 2
+//   warp 9     TMEM allocation and the single-thread tcgen05.mma issue
+//   warps 10-11 idle (they complete the third warpgroup)
+// The kernel launches with 168 registers per thread; the third warpgroup
+// gives registers back (72 each) and the softmax groups take them (216 each),
+// so that a thread holds its whole 128-column score row: 2*128*216 + 128*72
+// = 384*168.
+// TMEM columns: S_w at [128 w, 128 w + 128) and O_w at [256 + 128 w, +D) for
+// warpgroup w.  P is written back over its own S buffer as packed 16-bit pairs
+// and is the A operand (from TMEM) of O_w += P V.
+// Each warpgroup keeps its own running max / sum and accumulator over its
+// half of the blocks; the epilogue merges the two halves (a fixed split, so
+// the result is deterministic).  MMA issue order: S_0, S_1, then for every j:
+// O_{j%2} += P_j V_j followed by S_{j+2}, so one group's softmax overlaps the
+// other group's matrix products.
+// The softmax works in the exp2 domain; O_w is rescaled only when a row max
+// grows by more than 2^8 (a warp-uniform decision).  Column pairs selected by
+// RF_EMU_PAIR_MASK take their exponentials from a polynomial on the FMA pipe
+// (rf_exp2_poly) instead of the MUFU unit.  Measured on the Wan2.2-shaped
+// layer, offloading 12.5% or 25% of them was slower than none (the extra
+// instructions cost more than the MUFU time they save at this schedule), so
+// the default mask is 0.
 // Every wait is bounded: on expiry the CTA records it in the status words and
 // unwinds (waiting, again bounded, for its own copies and MMAs in flight).
 #include <cuda.h>
@@ -37,7 +51,18 @@
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
+constexpr uint32_t kSoftmaxRegs = 216;
+constexpr uint32_t kOtherRegs = 72;
+static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+#ifndef RF_EMU_PAIR_MASK
+#define RF_EMU_PAIR_MASK 0x0u
+#endif
+constexpr uint32_t kEmuPairMask = RF_EMU_PAIR_MASK;  // bit i: pair i of every 16 column pairs uses rf_exp2_poly
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -52,12 +77,14 @@ struct __align__(1024) AttnSmem {
   uint64_t bar_q;
   uint64_t bar_k_full[kStages], bar_k_empty[kStages];
   uint64_t bar_v_full[kStages], bar_v_empty[kStages];
-  uint64_t bar_s_full[2], bar_p_full[2];
-  uint64_t bar_o_done;
+  uint64_t bar_s_full[2], bar_p_full[2], bar_o_done[2];
+  uint64_t bar_final;
   uint64_t bar_drain;
   uint32_t tmem_base;
   int abort;
   int n_valid;
+  float row_m[2][RF_BLOCK];
+  float row_l[2][RF_BLOCK];
   int list[RF_MAX_KV_LIST];
 };
 
@@ -81,6 +108,45 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ void record_timeout(volatile int* abort, uint32_t* status, int where) {
   *abort = 1;
   atomicOr(status + RF_STATUS_TIMEOUT, 1u << where);
+}
+
+__device__ __forceinline__ void softmax_bar_sync() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight softmax warps
+}
+
+// Row max of 128 raw scores (the first vr valid), eight independent chains.
+template <bool kFull>
+__device__ __forceinline__ float row_max(const uint32_t* sr, int vr) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if (kFull || c < vr) m[c & 7] = fmaxf(m[c & 7], __uint_as_float(sr[c]));
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// p = 2^(s * sl2 - m) for 128 scores (the first vr valid), packed pairwise to
+// 16-bit into pk[64]; returns the fp32 sum.  Pairs selected by kEmuPairMask
+// use the FMA-pipe polynomial, the others ex2.approx.
+template <bool kBf16, bool kFull>
+__device__ __forceinline__ float row_exp(const uint32_t* sr, int vr, float sl2, float neg_m, uint32_t* pk) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int c = 0; c < 128; c += 2) {
+    const bool emu = (kEmuPairMask >> ((c >> 1) & 15)) & 1u;
+    const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg_m);
+    const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg_m);
+    float p0 = emu ? rf_exp2_poly(x0) : rf_ex2(x0);
+    float p1 = emu ? rf_exp2_poly(x1) : rf_ex2(x1);
+    if (!kFull) {
+      p0 = c < vr ? p0 : 0.f;
+      p1 = c + 1 < vr ? p1 : 0.f;
+    }
+    acc[(c >> 1) & 3] += p0 + p1;
+    pk[c >> 1] = rf_pack2<kBf16>(p0, p1);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 template <int D, bool kBf16>
@@ -117,18 +183,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(rf_smem_u32(&sm.bar_s_full[i]), 1);
       mbar_init(rf_smem_u32(&sm.bar_p_full[i]), 128);
+      mbar_init(rf_smem_u32(&sm.bar_o_done[i]), 1);
     }
-    mbar_init(rf_smem_u32(&sm.bar_o_done), 1);
+    mbar_init(rf_smem_u32(&sm.bar_final), 1);
     mbar_init(rf_smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(rf_smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
   }
@@ -169,8 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const int nv = sm.n_valid;
   const int vr_last = s.Lp - (s.n_pb - 1) * RF_BLOCK;  // valid rows of the last prefix block
-
-  if (warp == 4) {
+  if (warp >= 8) {
+  reg_dealloc<kOtherRegs>();
+  if (warp == kProducerWarp) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && nv > 0) {
       const bool bnsd = g.layout == RF_LAYOUT_BNSD;
@@ -224,138 +292,152 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(rf_smem_u32(&sm.bar_v_full[j % kStages]), (j / kStages) & 1, &no_abort);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------- tcgen05.mma issue (one thread) ----------------
     if (lane == 0 && nv > 0) {
       const uint32_t fmt = kBf16 ? 1u : 0u;
       const uint32_t idesc_qk = umma_idesc_f16(fmt, 128, 128, 0);
       const uint32_t idesc_pv = umma_idesc_f16(fmt, 128, D, 1);
       const uint32_t q_addr = rf_smem_u32(sm.q);
-      auto issue_qk = [&](int j) {
-        const int st = j % kStages, buf = j & 1;
+      // S_j = Q K_j^T into the S buffer of warpgroup j % 2 (stage j % 2).
+      auto issue_qk = [&](int j) -> bool {
+        const int st = j % kStages;
+        if (!mbar_wait(rf_smem_u32(&sm.bar_k_full[st]), (j / kStages) & 1, abort)) return false;
+        tc_fence_after();
         const uint32_t k_addr = rf_smem_u32(sm.k[st]);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + buf * 128, umma_desc_sw128(q_addr + off, 16, 1024),
+          mma_ss(tmem + (j & 1) * 128, umma_desc_sw128(q_addr + off, 16, 1024),
                  umma_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
-        tc_commit(rf_smem_u32(&sm.bar_s_full[buf]));
+        tc_commit(rf_smem_u32(&sm.bar_s_full[j & 1]));
         tc_commit(rf_smem_u32(&sm.bar_k_empty[st]));
+        return true;
       };
       bool ok = mbar_wait(rf_smem_u32(&sm.bar_q), 0, abort);
-      if (ok) ok = mbar_wait(rf_smem_u32(&sm.bar_k_full[0]), 0, abort);
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0);
-      }
+      if (ok) ok = issue_qk(0);
+      if (ok && nv > 1) ok = issue_qk(1);
       for (int j = 0; ok && j < nv; ++j) {
-        if (j + 1 < nv) {
-          const int st = (j + 1) % kStages;
-          if (!mbar_wait(rf_smem_u32(&sm.bar_k_full[st]), ((j + 1) / kStages) & 1, abort)) { ok = false; break; }
-          tc_fence_after();
-          issue_qk(j + 1);
-        }
-        const int buf = j & 1, st = j % kStages;
-        if (!mbar_wait(rf_smem_u32(&sm.bar_p_full[buf]), (j >> 1) & 1, abort)) { ok = false; break; }
+        const int w = j & 1, i = j >> 1, st = j % kStages;
+        if (!mbar_wait(rf_smem_u32(&sm.bar_p_full[w]), i & 1, abort)) { ok = false; break; }
         if (!mbar_wait(rf_smem_u32(&sm.bar_v_full[st]), (j / kStages) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t v_addr = rf_smem_u32(sm.v[st]);
 #pragma unroll
         for (int kk = 0; kk < RF_BLOCK / 16; ++kk)
-          mma_ts(tmem + 256, tmem + buf * 128 + kk * 8,
+          mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8,
                  umma_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(rf_smem_u32(&sm.bar_o_done));
+                 (i > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(rf_smem_u32(&sm.bar_o_done[w]));
         tc_commit(rf_smem_u32(&sm.bar_v_empty[st]));
+        if (j + 2 < nv && !issue_qk(j + 2)) { ok = false; break; }
       }
       if (!ok) record_timeout(abort, a.status, 2);
-      // Drain: every MMA this thread issued has completed before TMEM is freed.
+      // Every MMA issued so far (all of them, on the normal path) completes
+      // before bar_final, which gates the epilogue, and before bar_drain,
+      // which gates freeing TMEM.
+      tc_commit(rf_smem_u32(&sm.bar_final));
       tc_commit(rf_smem_u32(&sm.bar_drain));
       volatile int no_abort = 0;
       mbar_wait(rf_smem_u32(&sm.bar_drain), 0, &no_abort);
     }
+  }
   } else {
-    // ---------------- softmax + epilogue (warps 0-3) ----------------
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    reg_alloc<kSoftmaxRegs>();
+    // ---------------- softmax + epilogue (warps 0-7) ----------------
+    const int wg = warp >> 2;                 // this warpgroup's block parity
+    const int row = (warp & 3) * 32 + lane;   // query row = TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    const uint32_t s_col = wg * 128, o_col = 256 + wg * 128;
     const float sl2 = a.sl2;
+    const int my_blocks = (nv + 1 - wg) >> 1;  // blocks j < nv with j % 2 == wg
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < nv; ++j) {
-      const int buf = j & 1;
-      if (!warp_wait(rf_smem_u32(&sm.bar_s_full[buf]), (j >> 1) & 1, abort)) { ok = false; break; }
+    for (int i = 0; i < my_blocks; ++i) {
+      const int j = 2 * i + wg;
+      if (!warp_wait(rf_smem_u32(&sm.bar_s_full[wg]), i & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(lane_base + buf * 128 + 0, sr + 0);
-      tmem_ld32(lane_base + buf * 128 + 32, sr + 32);
-      tmem_ld32(lane_base + buf * 128 + 64, sr + 64);
-      tmem_ld32(lane_base + buf * 128 + 96, sr + 96);
-      tmem_wait_ld();
       const int vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;  // uniform over the CTA
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c < vr) mx = fmaxf(mx, __uint_as_float(sr[c]));
-      const float mx_t = mx * sl2;
-      if (__any_sync(0xffffffffu, mx_t > m_run + kRescaleThreshold)) {
+      const uint32_t scol = lane_base + s_col;
+      uint32_t sr[128];
+      tmem_ld32(scol, sr);
+      tmem_ld32(scol + 32, sr + 32);
+      tmem_ld32(scol + 64, sr + 64);
+      tmem_ld32(scol + 96, sr + 96);
+      tmem_wait_ld();
+      const float mx_t = (vr == RF_BLOCK ? row_max<true>(sr, vr) : row_max<false>(sr, vr)) * sl2;
+      const bool rescale = __any_sync(0xffffffffu, mx_t > m_run + kRescaleThreshold);
+      float alpha = 1.f;
+      if (rescale) {
         const float m_new = fmaxf(m_run, mx_t);
-        const float alpha = rf_ex2(m_run - m_new);
+        alpha = rf_ex2(m_run - m_new);
         l_run *= alpha;
-        if (j > 0) {
-          // O holds P_0..P_{j-1} V: wait for the last of those MMAs, then rescale.
-          if (!warp_wait(rf_smem_u32(&sm.bar_o_done), (j - 1) & 1, abort)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll 1
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + 256 + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(lane_base + 256 + c0, o);
-          }
-          tmem_wait_st();
-        }
         m_run = m_new;
       }
-      const float neg_m = -m_run;
-      float sum = 0.f;
       uint32_t pk[64];
+      l_run += vr == RF_BLOCK ? row_exp<kBf16, true>(sr, vr, sl2, -m_run, pk)
+                              : row_exp<kBf16, false>(sr, vr, sl2, -m_run, pk);
+      tmem_st32(scol, pk);
+      tmem_st32(scol + 32, pk + 32);
+      if (rescale && i > 0) {
+        // O_w holds this group's earlier P V products: wait for the last one,
+        // then rescale it before P_j is released to the MMA warp.
+        if (!warp_wait(rf_smem_u32(&sm.bar_o_done[wg]), (i - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + o_col + c0, o);
+          tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = c < vr ? rf_ex2(fmaf(__uint_as_float(sr[c]), sl2, neg_m)) : 0.f;
-        const float p1 = c + 1 < vr ? rf_ex2(fmaf(__uint_as_float(sr[c + 1]), sl2, neg_m)) : 0.f;
-        sum += p0 + p1;
-        pk[c >> 1] = rf_pack2<kBf16>(p0, p1);
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(lane_base + o_col + c0, o);
+        }
       }
-      l_run += sum;
-      tmem_st32(lane_base + buf * 128 + 0, pk + 0);
-      tmem_st32(lane_base + buf * 128 + 32, pk + 32);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(rf_smem_u32(&sm.bar_p_full[buf]));
+      mbar_arrive(rf_smem_u32(&sm.bar_p_full[wg]));
     }
     if (!ok) record_timeout(abort, a.status, 3);
-    // Epilogue: O / l -> 16-bit, rows of this query block only.
-    const bool have_o = ok && nv > 0 && warp_wait(rf_smem_u32(&sm.bar_o_done), (nv - 1) & 1, abort);
+
+    // Epilogue: merge the two groups' (max, sum, O) per row, write this group's
+    // half of the columns: O = (2^(m0-m) O_0 + 2^(m1-m) O_1) / (2^(m0-m) l_0 + 2^(m1-m) l_1).
+    sm.row_m[wg][row] = m_run;
+    sm.row_l[wg][row] = l_run;
+    softmax_bar_sync();
+    const bool have_o = ok && nv > 0 && warp_wait(rf_smem_u32(&sm.bar_final), 0, abort);
+    const float m0 = sm.row_m[0][row], m1 = sm.row_m[1][row];
+    const float l0 = sm.row_l[0][row], l1 = sm.row_l[1][row];
+    const float m = fmaxf(m0, m1);
+    const float a0 = l0 > 0.f ? rf_ex2(m0 - m) : 0.f;
+    const float a1 = l1 > 0.f ? rf_ex2(m1 - m) : 0.f;
+    const float l = a0 * l0 + a1 * l1;
+    const float inv = l > 0.f ? 1.0f / l : 0.f;
+    const float s0 = a0 * inv, s1 = a1 * inv;
+    const bool use0 = have_o && nv > 0, use1 = have_o && nv > 1;
     uint16_t* dst = a.o_r + rf_row_offset(g, s, g.n1, n, q_r0 + min(row, q_rows - 1));
-    const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
     if (have_o) tc_fence_after();
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(lane_base + 256 + c0, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] = 0u;
-      }
+    for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
+      uint32_t o0[32], o1[32];
+      if (use0) tmem_ld32(lane_base + 256 + c0, o0);
+      if (use1) tmem_ld32(lane_base + 384 + c0, o1);
+      if (use0 || use1) tmem_wait_ld();
       uint32_t w[16];
 #pragma unroll
-      for (int c = 0; c < 16; ++c)
-        w[c] = rf_pack2<kBf16>(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+      for (int c = 0; c < 16; ++c) {
+        float x0 = 0.f, x1 = 0.f;
+        if (use0) {
+          x0 = s0 * __uint_as_float(o0[2 * c]);
+          x1 = s0 * __uint_as_float(o0[2 * c + 1]);
+        }
+        if (use1) {
+          x0 = fmaf(s1, __uint_as_float(o1[2 * c]), x0);
+          x1 = fmaf(s1, __uint_as_float(o1[2 * c + 1]), x1);
+        }
+        w[c] = rf_pack2<kBf16>(x0, x1);
+      }
       if (row < q_rows) {
         uint4* d4 = reinterpret_cast<uint4*>(dst + c0);
         d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -368,9 +450,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Self-test of the two exponential paths the softmax uses.
+__global__ void rf_exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y_poly,
+                                        float* __restrict__ y_mufu, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    y_poly[i] = rf_exp2_poly(x[i]);
+    y_mufu[i] = rf_ex2(x[i]);
   }
 }
 
@@ -434,6 +526,16 @@ rf_status_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return rf_check_launch("cudaFuncSetAttribute(rf_attn_kernel)");
+  // The warpgroup register split (setmaxnreg) assumes exactly kLaunchRegs per
+  // thread at launch; with fewer, the softmax groups' request could never be
+  // met.  Refuse to launch a build that differs.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess)
+    return rf_check_launch("cudaFuncGetAttributes(rf_attn_kernel)");
+  if (fa.numRegs != kLaunchRegs)
+    return rf_fail(RF_ERR_CUDA, "rf_attn_kernel built with " + std::to_string(fa.numRegs) +
+                                    " registers per thread; the register split needs " +
+                                    std::to_string(kLaunchRegs));
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, args);
   return rf_check_launch("rf_attn_kernel");
 }
@@ -465,4 +567,11 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
               : launch_t<128, false>(mq, mk, mv, args, (unsigned)grid, st);
   return bf ? launch_t<64, true>(mq, mk, mv, args, (unsigned)grid, st)
             : launch_t<64, false>(mq, mk, mv, args, (unsigned)grid, st);
+}
+
+rf_status_t rf_launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                                    cudaStream_t st) {
+  if (n <= 0) return RF_OK;
+  rf_exp2_selftest_kernel<<<1184, 256, 0, st>>>(x, y_poly, y_mufu, (long long)n);
+  return rf_check_launch("rf_exp2_selftest_kernel");
 }

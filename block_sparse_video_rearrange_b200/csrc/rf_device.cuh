@@ -110,8 +110,23 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One test of phase `parity`; the thread may be suspended in hardware (up to
+// RF_SUSPEND_HINT_NS, or until the phase completes) instead of spinning, so a
+// waiting warp does not take issue slots from the warps sharing its scheduler.
+#ifndef RF_SUSPEND_HINT_NS
+#define RF_SUSPEND_HINT_NS 1000000u
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+#if RF_SUSPEND_HINT_NS > 0
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(RF_SUSPEND_HINT_NS)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -119,6 +134,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 
@@ -130,12 +146,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = rf_globaltimer();
 #pragma unroll 1
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort) return false;
-      if (rf_globaltimer() - t0 > RF_WAIT_LIMIT_NS) return false;
-    }
+    if (*abort) return false;
+    if (rf_globaltimer() - t0 > RF_WAIT_LIMIT_NS) return false;
   }
 }
 
@@ -229,6 +243,26 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
+// Register re-allocation between warpgroups (all warps of a warpgroup execute it).
+template <uint32_t kRegs>
+__device__ __forceinline__ void reg_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void reg_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -240,6 +274,29 @@ __device__ __forceinline__ float rf_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes, for the share of the softmax
+// exponentials taken off the MUFU unit.  Range reduction: x = j + r with
+// j = round(x) (adding 1.5 * 2^23 leaves round(x) in the low mantissa bits)
+// and r in [-1/2, 1/2]; 2^r from a degree-3 polynomial with p(0) = 1 whose
+// coefficients were fitted for minimum relative error on [-1/2, 1/2] by
+// csrc/gen_exp2_poly.py (max relative error 1.8e-4 in fp32); 2^j is added to
+// the exponent field.  x is clamped at -125.5 so the result stays a normal
+// number (2^-125.5 instead of 0 for smaller inputs; irrelevant next to the
+// row maximum, whose exponential is >= 2^-8 here).
+__device__ __forceinline__ float rf_exp2_poly(float x) {
+  constexpr float kShifter = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC1 = 0.6933164596557617f, kC2 = 0.24192412197589874f,
+                  kC3 = 0.054602622985839844f;
+  x = fmaxf(x, -125.5f);
+  const float t = x + kShifter;
+  const float r = x - (t - kShifter);
+  const int j = __float_as_int(t) - __float_as_int(kShifter);
+  float p = fmaf(kC3, r, kC2);
+  p = fmaf(p, r, kC1);
+  p = fmaf(p, r, 1.0f);
+  return __int_as_float(__float_as_int(p) + (j << 23));
 }
 
 // Two floats to packed 16-bit (lo = a, hi = b), round to nearest even.

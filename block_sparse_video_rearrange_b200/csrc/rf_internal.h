@@ -71,6 +71,8 @@ rf_status_t rf_launch_pool(const rf_plan* p, const void* q_r, const void* k_r, v
 rf_status_t rf_launch_inverse(const rf_plan* p, const void* o_r, void* o, cudaStream_t st);
 rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_num, void* ws,
                              cudaStream_t st);
+rf_status_t rf_launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                                    cudaStream_t st);
 rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, const void* v_r,
                            const int32_t* sel_idx, const int32_t* sel_num, float scale,
                            void* o_r, void* ws, cudaStream_t st);

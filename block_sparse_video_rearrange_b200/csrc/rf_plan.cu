@@ -355,6 +355,15 @@ rf_status_t rf_forward(const rf_plan_t* p, const void* q, const void* k, const v
   return rf_inverse_rearrange(p, o_r, o, stream);
 }
 
+rf_status_t rf_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                             rf_stream_t stream) {
+  g_last_error.clear();
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_mufu))) return rf_fail(RF_ERR_INVALID_ARG, "bad buffers");
+  rf_status_t st = rf_require_device();
+  if (st != RF_OK) return st;
+  return rf_launch_exp2_selftest(x, y_poly, y_mufu, n, (cudaStream_t)stream);
+}
+
 rf_status_t rf_check_device_status(const rf_plan_t* p, void* ws, uint32_t* flags_out,
                                    rf_stream_t stream) {
   g_last_error.clear();

@@ -18,7 +18,8 @@ from typing import Iterable, List, Optional, Sequence, Tuple
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librf.so")
+# RF_LIBRARY may name another build of librf (same ABI), e.g. to compare builds.
+LIB_PATH = os.environ.get("RF_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "librf.so")
 
 RF_OK = 0
 STATUS_NAMES = {0: "RF_OK", 1: "RF_ERR_INVALID_ARG", 2: "RF_ERR_UNSUPPORTED_DEVICE",
@@ -31,7 +32,8 @@ POOL_MODES = {"from_ws": 0, "recompute": 1}
 
 EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange", "rf_pool_select",
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
-            "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation")
+            "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
+            "rf_selftest_exp2")
 
 
 class RfError(RuntimeError):
@@ -78,6 +80,7 @@ def _load() -> ctypes.CDLL:
         "rf_forward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp, sz, vp],
         "rf_check_device_status": [vp, vp, ctypes.POINTER(ctypes.c_uint32), vp],
         "rf_plan_destroy": [vp],
+        "rf_selftest_exp2": [vp, vp, vp, ctypes.c_int64, vp],
         "rf_plan_permutation": [vp, i32, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64],
         "rf_status_string": [i32],
         "rf_last_error": [],
@@ -245,6 +248,14 @@ def inverse_rearrange(plan: Plan, o_r, o, stream=None) -> None:
     _expect(o, plan.tensor_shape(plan.n1), plan.torch_dtype, "o")
     _check(_lib.rf_inverse_rearrange(plan.handle, _ptr(o_r), _ptr(o), _stream(stream)),
            "rf_inverse_rearrange")
+
+
+def selftest_exp2(x: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(polynomial 2^x, ex2.approx 2^x) of a float32 device tensor, from the kernel's own code paths."""
+    assert x.dtype == torch.float32 and x.is_cuda
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _check(_lib.rf_selftest_exp2(_ptr(x), _ptr(yp), _ptr(ym), x.numel(), _stream(stream)), "rf_selftest_exp2")
+    return yp, ym
 
 
 def check_device_status(plan: Plan, ws, stream=None) -> Tuple[int, Tuple[int, int]]:

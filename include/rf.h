@@ -225,6 +225,13 @@ RF_API rf_status_t rf_plan_permutation(const rf_plan_t* plan, int32_t seq, int64
 RF_API rf_status_t rf_check_device_status(const rf_plan_t* plan, void* ws, uint32_t* flags_out,
                                    rf_stream_t stream);
 
+/* Self-test of the attention kernel's two exponential paths (the pages have no
+ * counterpart; this exists so the polynomial can be checked on the device):
+ * y_poly[i] = the FMA-pipe polynomial 2^x[i], y_mufu[i] = ex2.approx(x[i]),
+ * for n float32 device values.  Asynchronous on `stream`. */
+RF_API rf_status_t rf_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                                    rf_stream_t stream);
+
 /* Frees a plan (NULL is a no-op). */
 RF_API void rf_plan_destroy(rf_plan_t* plan);
 

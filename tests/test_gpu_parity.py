@@ -183,3 +183,22 @@ def test_full_size_parity(name, s):
     assert stats["near_tie"] <= max(1, stats["rows"] // 1000), stats
     items = parity.sample_items(p, np.random.default_rng(7), per_kind=3)
     parity.check_attention(p, w, rbits, gpu, items)
+
+
+def test_exp2_polynomial_against_mufu_and_exact():
+    """The FMA-pipe exponential the softmax uses for part of its columns:
+    relative error <= 2e-4 against the exact 2^x and against ex2.approx,
+    over the range the softmax feeds it (x <= 8)."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 2_000_001, dtype=torch.float32),
+                   torch.tensor([0.0, -0.5, 0.5, -1.0, 1.0, -8.0, 8.0, -20.25], dtype=torch.float32)]).cuda()
+    yp, ym = rf.selftest_exp2(x)
+    torch.cuda.synchronize()
+    exact = torch.exp2(x.double())
+    rel_poly = ((yp.double() - exact).abs() / exact).max().item()
+    rel_mufu = ((ym.double() - exact).abs() / exact).max().item()
+    assert rel_poly <= 2e-4, rel_poly
+    assert rel_mufu <= 1e-5, rel_mufu
+    # integers map to exact powers of two
+    xi = torch.arange(-120, 9, dtype=torch.float32).cuda()
+    yi, _ = rf.selftest_exp2(xi)
+    assert torch.equal(yi.double(), torch.exp2(xi.double()))
