@@ -33,7 +33,7 @@ POOL_MODES = {"from_ws": 0, "recompute": 1}
 EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange", "rf_pool_select",
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
             "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
-            "rf_selftest_exp2")
+            "rf_selftest_exp2", "rf_pool_select_noalloc")
 
 
 class RfError(RuntimeError):
@@ -81,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "rf_check_device_status": [vp, vp, ctypes.POINTER(ctypes.c_uint32), vp],
         "rf_plan_destroy": [vp],
         "rf_selftest_exp2": [vp, vp, vp, ctypes.c_int64, vp],
+        "rf_pool_select_noalloc": [vp, vp, vp, vp, vp, vp],
         "rf_plan_permutation": [vp, i32, ctypes.POINTER(ctypes.c_int64), ctypes.c_int64],
         "rf_status_string": [i32],
         "rf_last_error": [],
@@ -231,6 +232,18 @@ def pool_select(plan: Plan, q_r, k_r, select_idx, select_num, ws, pool_mode: str
     _check(_lib.rf_pool_select(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(select_idx), _ptr(select_num),
                                _ptr(ws), ws.numel() * ws.element_size(), POOL_MODES[pool_mode],
                                _stream(stream)), "rf_pool_select")
+
+
+def pool_select_noalloc(plan: Plan, q_r, k_r, select_idx, select_num, stream=None) -> None:
+    """Selection without any device allocation: the scratch is a static array
+    inside librf (32 MiB per device, set up by the first call on a device).
+    For callers that cannot allocate device memory; same result as
+    pool_select(..., pool_mode="recompute").  Concurrent calls on one device race."""
+    si, sn = plan.select_shapes()
+    _expect(select_idx, si, torch.int32, "select_idx")
+    _expect(select_num, sn, torch.int32, "select_num")
+    _check(_lib.rf_pool_select_noalloc(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(select_idx), _ptr(select_num),
+                                       _stream(stream)), "rf_pool_select_noalloc")
 
 
 def block_sparse_attn(plan: Plan, q_r, k_r, v_r, select_idx, select_num, scale: float, o_r, ws,

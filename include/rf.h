@@ -181,6 +181,27 @@ RF_API rf_status_t rf_pool_select(const rf_plan_t* plan, const void* q_r, const 
                            int32_t* select_idx, int32_t* select_num, void* ws,
                            size_t ws_bytes, rf_pool_mode_t pool_mode, rf_stream_t stream);
 
+/* Steps 2-3 without any device allocation by the caller or the library.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory -- code running inside a host framework whose
+ * device memory belongs to the framework's own allocator (a plugin cannot
+ * cudaMalloc behind its back), or code on a latency-critical path where a
+ * cudaMalloc, which may synchronise the device, is not acceptable.
+ * Same result as rf_pool_select(..., RF_POOL_RECOMPUTE): the block means are
+ * recomputed from q_r and k_r (both required, 16-byte aligned), then ranked.
+ * Scratch: one static device array of 32 MiB inside librf.  It is set up on
+ * the first call on each device (with that device current), which loads it
+ * onto that GPU, where it stays until the process exits; make that first call
+ * before any stream capture.  Problems whose selection scratch
+ * (rf_plan_info().workspace_bytes) exceeds 32 MiB are rejected with
+ * RF_ERR_INVALID_ARG.  Every call on a device shares the array: calls that
+ * overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.  Calls no cudaMalloc, cudaFree or other
+ * allocating routine. */
+RF_API rf_status_t rf_pool_select_noalloc(const rf_plan_t* plan, const void* q_r, const void* k_r,
+                                          int32_t* select_idx, int32_t* select_num,
+                                          rf_stream_t stream);
+
 /* Step 4 ([API] "Formula": Softmax(scale * Q K^T + atten_mask) V, restricted to
  * the key blocks of selectIdx; no user mask is consumed, the only masked keys
  * are rows past the dense prefix in its last, partial block).
