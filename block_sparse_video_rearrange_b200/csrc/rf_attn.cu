@@ -114,39 +114,58 @@ __device__ __forceinline__ void softmax_bar_sync() {
   asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight softmax warps
 }
 
-// Row max of 128 raw scores (the first vr valid), eight independent chains.
+// Row max of 128 raw scores (the first vr valid): three-input max, eight chains.
 template <bool kFull>
 __device__ __forceinline__ float row_max(const uint32_t* sr, int vr) {
   float m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = -INFINITY;
+  if (kFull) {
 #pragma unroll
-  for (int c = 0; c < 128; ++c)
-    if (kFull || c < vr) m[c & 7] = fmaxf(m[c & 7], __uint_as_float(sr[c]));
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+    for (int c = 0; c < 128; c += 2)
+      m[(c >> 1) & 7] = rf_max3(m[(c >> 1) & 7], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+  } else {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (c < vr) m[c & 7] = fmaxf(m[c & 7], __uint_as_float(sr[c]));
+  }
+  return rf_max3(rf_max3(m[0], m[1], m[2]), rf_max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // p = 2^(s * sl2 - m) for 128 scores (the first vr valid), packed pairwise to
-// 16-bit into pk[64]; returns the fp32 sum.  Pairs selected by kEmuPairMask
-// use the FMA-pipe polynomial, the others ex2.approx.
+// 16-bit into pk[64]; returns the fp32 sum.  The scale-and-subtract and the
+// running sums run as paired fp32 instructions (two columns per instruction).
+// Pairs selected by kEmuPairMask use the FMA-pipe polynomial, the others
+// ex2.approx.
 template <bool kBf16, bool kFull>
 __device__ __forceinline__ float row_exp(const uint32_t* sr, int vr, float sl2, float neg_m, uint32_t* pk) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
+  const uint64_t negm2 = rf_f2(__float_as_uint(neg_m), __float_as_uint(neg_m));
+  uint64_t acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = 0ull;
 #pragma unroll
   for (int c = 0; c < 128; c += 2) {
     const bool emu = (kEmuPairMask >> ((c >> 1) & 15)) & 1u;
-    const float x0 = fmaf(__uint_as_float(sr[c]), sl2, neg_m);
-    const float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, neg_m);
+    float x0, x1;
+    rf_f2_split(rf_fma2(rf_f2(sr[c], sr[c + 1]), sl2x2, negm2), x0, x1);
     float p0 = emu ? rf_exp2_poly(x0) : rf_ex2(x0);
     float p1 = emu ? rf_exp2_poly(x1) : rf_ex2(x1);
     if (!kFull) {
       p0 = c < vr ? p0 : 0.f;
       p1 = c + 1 < vr ? p1 : 0.f;
     }
-    acc[(c >> 1) & 3] += p0 + p1;
+    acc[(c >> 1) & 3] = rf_add2(acc[(c >> 1) & 3], rf_f2(__float_as_uint(p0), __float_as_uint(p1)));
     pk[c >> 1] = rf_pack2<kBf16>(p0, p1);
   }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a, b;
+    rf_f2_split(acc[i], a, b);
+    s += a + b;
+  }
+  return s;
 }
 
 template <int D, bool kBf16>
