@@ -18,10 +18,12 @@
 //   warps 0-3  softmax warpgroup 0: the even-numbered selected blocks
 //   warps 4-7  softmax warpgroup 1: the odd-numbered selected blocks
 //              (thread = query row = TMEM lane in both groups)
-//   warp 8     TMA producer: Q once, then K_j / V_j of each selected block;
-//              block j always uses shared-memory stage j % 2
+//   warp 8     TMA producer of Q (once) and K_j through a 3-stage ring
 //   warp 9     TMEM allocation and the single-thread tcgen05.mma issue
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warp 10    TMA producer of V_j through a 2-stage ring (K and V have
+//              separate producers so that a K load never queues behind a V
+//              load that waits for an earlier P V product)
+//   warp 11    idle (it completes the third warpgroup)
 // The kernel launches with 168 registers per thread; the third warpgroup
 // gives registers back (72 each) and the softmax groups take them (216 each),
 // so that a thread holds its whole 128-column score row: 2*128*216 + 128*72
@@ -52,8 +54,9 @@
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kProducerWarp = 8;
+constexpr int kProducerWarp = 8;   // Q and K loads
 constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10; // V loads
 constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
 constexpr uint32_t kSoftmaxRegs = 216;
 constexpr uint32_t kOtherRegs = 72;
@@ -63,7 +66,8 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchReg
 #define RF_EMU_PAIR_MASK 0x0u
 #endif
 constexpr uint32_t kEmuPairMask = RF_EMU_PAIR_MASK;  // bit i: pair i of every 16 column pairs uses rf_exp2_poly
-constexpr int kStages = 2;
+constexpr int kStagesK = 3;  // K ring: K_{j+3} is requested as soon as S_j is done
+constexpr int kStagesV = 2;  // V ring: V_{j+2} is requested as soon as O += P_j V_j is done
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy rescale while growth <= 256x
@@ -72,11 +76,11 @@ template <int D>
 struct __align__(1024) AttnSmem {
   static constexpr int kTileBytes = RF_BLOCK * D * 2;  // 128 rows x D x 16-bit
   uint8_t q[kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t k[kStagesK][kTileBytes];
+  uint8_t v[kStagesV][kTileBytes];
   uint64_t bar_q;
-  uint64_t bar_k_full[kStages], bar_k_empty[kStages];
-  uint64_t bar_v_full[kStages], bar_v_empty[kStages];
+  uint64_t bar_k_full[kStagesK], bar_k_empty[kStagesK];
+  uint64_t bar_v_full[kStagesV], bar_v_empty[kStagesV];
   uint64_t bar_s_full[2], bar_p_full[2], bar_o_done[2];
   uint64_t bar_final;
   uint64_t bar_drain;
@@ -97,12 +101,12 @@ struct AttnArgs {
   float sl2;  // scale * log2(e)
 };
 
-// Warp-uniform bounded wait: lane 0 polls, the result is broadcast.
+// Warp-wide bounded wait: every lane polls the barrier itself (a lane that
+// only waits on a warp shuffle for a polling lane 0 wakes far later), then the
+// warp agrees on the outcome.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  return ok != 0;
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
 }
 
 __device__ __forceinline__ void record_timeout(volatile int* abort, uint32_t* status, int where) {
@@ -193,9 +197,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(rf_smem_u32(&sm.bar_q), 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kStagesK; ++i) {
       mbar_init(rf_smem_u32(&sm.bar_k_full[i]), 1);
       mbar_init(rf_smem_u32(&sm.bar_k_empty[i]), 1);
+    }
+    for (int i = 0; i < kStagesV; ++i) {
       mbar_init(rf_smem_u32(&sm.bar_v_full[i]), 1);
       mbar_init(rf_smem_u32(&sm.bar_v_empty[i]), 1);
     }
@@ -257,110 +263,115 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int vr_last = s.Lp - (s.n_pb - 1) * RF_BLOCK;  // valid rows of the last prefix block
   if (warp >= 8) {
   reg_dealloc<kOtherRegs>();
-  if (warp == kProducerWarp) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0 && nv > 0) {
-      const bool bnsd = g.layout == RF_LAYOUT_BNSD;
-      auto coords = [&](int heads, int head, int r0, int& c1, int& c2) {
-        if (bnsd) { c1 = r0; c2 = s.batch_idx * heads + head; }
-        else      { c1 = head; c2 = (int)s.row_off + r0; }
-      };
-      int c1, c2;
+  if ((warp == kProducerWarp || warp == kVProducerWarp) && lane == 0 && nv > 0) {
+    // ---------------- TMA producers: one thread streams Q then K, another V ----------------
+    const bool is_k = warp == kProducerWarp;
+    const bool bnsd = g.layout == RF_LAYOUT_BNSD;
+    auto coords = [&](int heads, int head, int r0, int& c1, int& c2) {
+      if (bnsd) { c1 = r0; c2 = s.batch_idx * heads + head; }
+      else      { c1 = head; c2 = (int)s.row_off + r0; }
+    };
+    int c1, c2;
+    const uint32_t bq = rf_smem_u32(&sm.bar_q);
+    if (is_k) {
       coords(g.n1, n, q_r0, c1, c2);
-      const uint32_t bq = rf_smem_u32(&sm.bar_q);
       mbar_arrive_expect_tx(bq, kTileBytes);
 #pragma unroll
       for (int x = 0; x < kBoxes; ++x)
         tma_load_3d(rf_smem_u32(sm.q + x * kBoxBytes), &tm_q, bq, x * 64, c1, c2);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < nv; ++j) {
-        const int st = j % kStages;
-        const uint32_t ph = (j / kStages) & 1;
-        if (j >= kStages && !mbar_wait(rf_smem_u32(&sm.bar_k_empty[st]), ph ^ 1, abort)) {
-          record_timeout(abort, a.status, 0);
-          break;
-        }
-        int r0, nr;
-        rf_block_span(s, sm.list[j], r0, nr);
-        coords(g.n2, gk, r0, c1, c2);
-        const uint32_t bk = rf_smem_u32(&sm.bar_k_full[st]);
-        mbar_arrive_expect_tx(bk, kTileBytes);
-#pragma unroll
-        for (int x = 0; x < kBoxes; ++x)
-          tma_load_3d(rf_smem_u32(sm.k[st] + x * kBoxBytes), &tm_k, bk, x * 64, c1, c2);
-        k_issued = j + 1;
-        if (j >= kStages && !mbar_wait(rf_smem_u32(&sm.bar_v_empty[st]), ph ^ 1, abort)) {
-          record_timeout(abort, a.status, 1);
-          break;
-        }
-        const uint32_t bv = rf_smem_u32(&sm.bar_v_full[st]);
-        mbar_arrive_expect_tx(bv, kTileBytes);
-#pragma unroll
-        for (int x = 0; x < kBoxes; ++x)
-          tma_load_3d(rf_smem_u32(sm.v[st] + x * kBoxBytes), &tm_v, bv, x * 64, c1, c2);
-        v_issued = j + 1;
-      }
-      if (*abort) {
-        // Let this CTA's own copies land before its shared memory goes away:
-        // the newest load of each stage completes last on that stage's barrier.
-        volatile int no_abort = 0;
-        mbar_wait(bq, 0, &no_abort);
-        for (int j = (k_issued > kStages ? k_issued - kStages : 0); j < k_issued; ++j)
-          mbar_wait(rf_smem_u32(&sm.bar_k_full[j % kStages]), (j / kStages) & 1, &no_abort);
-        for (int j = (v_issued > kStages ? v_issued - kStages : 0); j < v_issued; ++j)
-          mbar_wait(rf_smem_u32(&sm.bar_v_full[j % kStages]), (j / kStages) & 1, &no_abort);
-      }
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------- tcgen05.mma issue (one thread) ----------------
-    if (lane == 0 && nv > 0) {
-      const uint32_t fmt = kBf16 ? 1u : 0u;
-      const uint32_t idesc_qk = umma_idesc_f16(fmt, 128, 128, 0);
-      const uint32_t idesc_pv = umma_idesc_f16(fmt, 128, D, 1);
-      const uint32_t q_addr = rf_smem_u32(sm.q);
-      // S_j = Q K_j^T into the S buffer of warpgroup j % 2 (stage j % 2).
-      auto issue_qk = [&](int j) -> bool {
-        const int st = j % kStages;
-        if (!mbar_wait(rf_smem_u32(&sm.bar_k_full[st]), (j / kStages) & 1, abort)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = rf_smem_u32(sm.k[st]);
+    const int stages = is_k ? kStagesK : kStagesV;
+    uint8_t* tiles = is_k ? &sm.k[0][0] : &sm.v[0][0];
+    uint64_t* full = is_k ? sm.bar_k_full : sm.bar_v_full;
+    uint64_t* empty = is_k ? sm.bar_k_empty : sm.bar_v_empty;
+    const void* map = is_k ? static_cast<const void*>(&tm_k) : static_cast<const void*>(&tm_v);
+    int issued = 0;
+    for (int j = 0; j < nv; ++j) {
+      const int st = j % stages;
+      const uint32_t ph = (j / stages) & 1;
+      if (j >= stages && !mbar_wait(rf_smem_u32(&empty[st]), ph ^ 1, abort)) {
+        record_timeout(abort, a.status, is_k ? 0 : 1);
+        break;
+      }
+      int r0, nr;
+      rf_block_span(s, sm.list[j], r0, nr);
+      coords(g.n2, gk, r0, c1, c2);
+      const uint32_t bar = rf_smem_u32(&full[st]);
+      mbar_arrive_expect_tx(bar, kTileBytes);
+#pragma unroll
+      for (int x = 0; x < kBoxes; ++x)
+        tma_load_3d(rf_smem_u32(tiles + st * kTileBytes + x * kBoxBytes), map, bar, x * 64, c1, c2);
+      issued = j + 1;
+    }
+    if (*abort) {
+      // Let this thread's own copies land before the CTA's shared memory goes
+      // away: the newest load of each stage completes last on its barrier.
+      volatile int no_abort = 0;
+      if (is_k) mbar_wait(bq, 0, &no_abort);
+      for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+        mbar_wait(rf_smem_u32(&full[j % stages]), (j / stages) & 1, &no_abort);
+    }
+  } else if (warp == kMmaWarp && nv > 0) {
+    // ---------------- tcgen05.mma issue ----------------
+    // The whole warp runs this loop (warp-uniform control flow keeps the
+    // descriptors in uniform registers); one elected lane issues every MMA
+    // and every commit, so the commits track all of them.
+    const uint32_t fmt = kBf16 ? 1u : 0u;
+    const uint32_t idesc_qk = umma_idesc_f16(fmt, 128, 128, 0);
+    const uint32_t idesc_pv = umma_idesc_f16(fmt, 128, D, 1);
+    // Adding (bytes >> 4) to a descriptor moves its 14-bit start-address field.
+    const uint64_t dq = umma_desc_sw128(rf_smem_u32(sm.q), 16, 1024);
+    const uint64_t dk0 = umma_desc_sw128(rf_smem_u32(sm.k[0]), 16, 1024);
+    const uint64_t dv0 = umma_desc_sw128(rf_smem_u32(sm.v[0]), kBoxBytes, 1024);
+    // S_j = Q K_j^T into the S buffer of warpgroup j % 2.
+    auto issue_qk = [&](int j) -> bool {
+      const int st = j % kStagesK;
+      if (!warp_wait(rf_smem_u32(&sm.bar_k_full[st]), (j / kStagesK) & 1, abort)) return false;
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t dk = dk0 + (uint64_t)(st * (kTileBytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          mma_ss(tmem + (j & 1) * 128, umma_desc_sw128(q_addr + off, 16, 1024),
-                 umma_desc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(rf_smem_u32(&sm.bar_s_full[j & 1]));
         tc_commit(rf_smem_u32(&sm.bar_k_empty[st]));
-        return true;
-      };
-      bool ok = mbar_wait(rf_smem_u32(&sm.bar_q), 0, abort);
-      if (ok) ok = issue_qk(0);
-      if (ok && nv > 1) ok = issue_qk(1);
-      for (int j = 0; ok && j < nv; ++j) {
-        const int w = j & 1, i = j >> 1, st = j % kStages;
-        if (!mbar_wait(rf_smem_u32(&sm.bar_p_full[w]), i & 1, abort)) { ok = false; break; }
-        if (!mbar_wait(rf_smem_u32(&sm.bar_v_full[st]), (j / kStages) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t v_addr = rf_smem_u32(sm.v[st]);
+      }
+      __syncwarp();
+      return true;
+    };
+    bool ok = warp_wait(rf_smem_u32(&sm.bar_q), 0, abort);
+    if (ok) ok = issue_qk(0);
+    if (ok && nv > 1) ok = issue_qk(1);
+    for (int j = 0; ok && j < nv; ++j) {
+      const int w = j & 1, i = j >> 1, st = j % kStagesV;
+      if (!warp_wait(rf_smem_u32(&sm.bar_p_full[w]), i & 1, abort)) { ok = false; break; }
+      if (!warp_wait(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      if (elect_one()) {
+        const uint64_t dv = dv0 + (uint64_t)(st * (kTileBytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < RF_BLOCK / 16; ++kk)
-          mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8,
-                 umma_desc_sw128(v_addr + kk * 2048, kBoxBytes, 1024), idesc_pv,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)),
+                 idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(rf_smem_u32(&sm.bar_o_done[w]));
         tc_commit(rf_smem_u32(&sm.bar_v_empty[st]));
-        if (j + 2 < nv && !issue_qk(j + 2)) { ok = false; break; }
       }
-      if (!ok) record_timeout(abort, a.status, 2);
-      // Every MMA issued so far (all of them, on the normal path) completes
-      // before bar_final, which gates the epilogue, and before bar_drain,
-      // which gates freeing TMEM.
+      __syncwarp();
+      if (j + 2 < nv && !issue_qk(j + 2)) { ok = false; break; }
+    }
+    if (!ok && lane == 0) record_timeout(abort, a.status, 2);
+    // Every MMA issued so far (all of them, on the normal path) completes
+    // before bar_final, which gates the epilogue, and before bar_drain,
+    // which gates freeing TMEM.
+    if (elect_one()) {
       tc_commit(rf_smem_u32(&sm.bar_final));
       tc_commit(rf_smem_u32(&sm.bar_drain));
-      volatile int no_abort = 0;
-      mbar_wait(rf_smem_u32(&sm.bar_drain), 0, &no_abort);
     }
+    __syncwarp();
+    volatile int no_abort = 0;
+    warp_wait(rf_smem_u32(&sm.bar_drain), 0, &no_abort);
   }
   } else {
     reg_alloc<kSoftmaxRegs>();
