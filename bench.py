@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="wan", choices=sorted(WORKLOAD_DESC))
     ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--order", default="tile", choices=["tile", "frame_pair"],
+                    help="token order of the aligned video (frame_pair: frames paired into 2x8x8 blocks)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -277,7 +279,7 @@ def main():
     wr = synth.Workload(w.name, w.layout, w.dtype, w.batch, w.seqs, w.n1, w.n2, w.d, w.sparsity, w.seed + 7919 * rank)
     bits = synth.generate_qkv(wr)
     seqs = [(s.prefix_len, s.t, s.h, s.w) for s in w.seqs]
-    plan = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch)
+    plan = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=args.order)
     tdt = plan.torch_dtype
     host = [torch.from_numpy(x.view(np.int16)).view(tdt).pin_memory() for x in bits]
     q, k, v = (h.to(dev) for h in host)
@@ -395,6 +397,7 @@ def main():
             "data": "synthetic (seeded smooth-field + noise per 8x8 cell; no real activations available)",
             "config": {"workload": WORKLOAD_DESC[w.name.split("@")[0]] + (f" [reduced to {w.n1} heads]" if args.heads else ""),
                        "sparsity": sparsity,
+                       **({"token_order": args.order} if args.order != "tile" else {}),
                        "global_batch": w.batch * world, "seq_len": int(plan.info.rows_total),
                        "parallelism": f"independent layer per GPU x{world}",
                        "l2": "inputs larger than L2 (Q+K+V %.2f GB vs 126 MB)" % (

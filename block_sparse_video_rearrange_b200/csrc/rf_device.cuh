@@ -46,6 +46,10 @@ __host__ __device__ __forceinline__ void rf_block_span(const RfSeqDev& s, int b,
 //   rearranged = [text | promoted | sparse]; the video part follows V', the
 //   video tokens in tile order: aligned tokens by (frame, tile row, tile col,
 //   row in tile, col in tile), then the ragged tokens in raster order.
+//   With RF_ORDER_FRAME_PAIR the aligned frames 1..t-1 are taken in pairs
+//   (xllm PR #1867, frame-pairing approach): frame 0 first, then each pair
+//   cube by cube (tile row, tile col; frame in pair, row, col), then an
+//   unpaired last frame in tile order.
 //   Sparse rows are V'[0, S); promoted rows are V'[S, t*h*w).
 __host__ __device__ __forceinline__ int rf_orig_row(const RfSeqDev& s, int r) {
   if (r < s.P) return r;
@@ -53,8 +57,18 @@ __host__ __device__ __forceinline__ int rf_orig_row(const RfSeqDev& s, int r) {
   int y, x, f;
   if (v < s.A) {
     const int frame = s.h8 * s.w8;
-    f = v / frame;
-    const int rem = v - f * frame;
+    int rem;  // position of the token in its frame's single-frame tile order
+    if (s.order == RF_ORDER_FRAME_PAIR && v >= frame && v < frame * (1 + 2 * ((s.t - 1) >> 1))) {
+      // Frame pair (2m+1, 2m+2): cube c holds tile c of both frames, 64 rows each.
+      const int u = v - frame;
+      const int pair = u / (2 * frame);
+      const int c = u - pair * 2 * frame;
+      f = 1 + 2 * pair + ((c >> 6) & 1);
+      rem = ((c >> 7) << 6) | (c & 63);
+    } else {
+      f = v / frame;
+      rem = v - f * frame;
+    }
     const int tile = rem >> 6, within = rem & 63;
     const int tiles_per_row = s.w8 >> 3;
     const int hb = tile / tiles_per_row, wb = tile - hb * tiles_per_row;

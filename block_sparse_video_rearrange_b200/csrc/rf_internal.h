@@ -26,6 +26,7 @@ struct RfSeqDev {
   int Lp;               // dense prefix rows P + promoted
   int L;                // sequence length
   int n_pb, nb, ns, k, dense;
+  int order;            // rf_token_order_t of the aligned video tokens
   int qblk_off;         // first global query block
   int pool_off;         // first pooled block (sum of nb of earlier instances)
 };

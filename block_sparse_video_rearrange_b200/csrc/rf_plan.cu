@@ -29,9 +29,10 @@ int keep_count(int nb, double sparsity) {
 // guide, "Geometry handling"): the sparse region is the largest whole number of
 // 128-row blocks of tokens inside whole 8x8 tiles; every other video token is
 // promoted into the always-dense prefix.
-RfSeqDev seq_geometry(const rf_seq_geom_t& s, double sparsity) {
+RfSeqDev seq_geometry(const rf_seq_geom_t& s, double sparsity, rf_token_order_t order) {
   RfSeqDev d;
   std::memset(&d, 0, sizeof(d));
+  d.order = order;
   d.P = s.prefix_len;
   d.t = s.t;
   d.h = s.h;
@@ -106,8 +107,18 @@ const char* rf_last_error(void) { return g_last_error.c_str(); }
 rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch, int32_t n1,
                            int32_t n2, int32_t d, rf_layout_t layout, rf_dtype_t dtype,
                            double sparsity, int32_t block_q, int32_t block_kv, rf_plan_t** out) {
+  return rf_plan_create_ex(seqs, n_seqs, batch, n1, n2, d, layout, dtype, sparsity, block_q,
+                           block_kv, RF_ORDER_TILE, out);
+}
+
+rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
+                              int32_t n1, int32_t n2, int32_t d, rf_layout_t layout,
+                              rf_dtype_t dtype, double sparsity, int32_t block_q,
+                              int32_t block_kv, rf_token_order_t order, rf_plan_t** out) {
   g_last_error.clear();
   if (!out || !seqs) return rf_fail(RF_ERR_INVALID_ARG, "null seqs or out");
+  if (order != RF_ORDER_TILE && order != RF_ORDER_FRAME_PAIR)
+    return rf_fail(RF_ERR_INVALID_ARG, "token order must be RF_ORDER_TILE or RF_ORDER_FRAME_PAIR");
   if (layout != RF_LAYOUT_BNSD && layout != RF_LAYOUT_TND)
     return rf_fail(RF_ERR_INVALID_ARG, "layout must be BNSD or TND");
   if (dtype != RF_BF16 && dtype != RF_FP16)
@@ -159,7 +170,7 @@ rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t ba
   int max_kv = 0, max_nb = 0;
   for (int i = 0; i < g.n_seqs; ++i) {
     const rf_seq_geom_t& src = seqs[layout == RF_LAYOUT_BNSD ? 0 : i];
-    RfSeqDev s = seq_geometry(src, sparsity);
+    RfSeqDev s = seq_geometry(src, sparsity, order);
     s.batch_idx = layout == RF_LAYOUT_BNSD ? i : 0;
     s.row_off = layout == RF_LAYOUT_BNSD ? 0 : rows;
     s.qblk_off = (int)qblk;

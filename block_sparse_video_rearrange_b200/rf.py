@@ -27,13 +27,14 @@ STATUS_NAMES = {0: "RF_OK", 1: "RF_ERR_INVALID_ARG", 2: "RF_ERR_UNSUPPORTED_DEVI
                 6: "RF_ERR_UNSUPPORTED"}
 LAYOUTS = {"BNSD": 0, "TND": 1}
 DTYPES = {"bf16": 0, "fp16": 1}
+ORDERS = {"tile": 0, "frame_pair": 1}   # rf_token_order_t
 TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 POOL_MODES = {"from_ws": 0, "recompute": 1}
 
 EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange", "rf_pool_select",
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
             "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
-            "rf_selftest_exp2", "rf_pool_select_noalloc")
+            "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex")
 
 
 class RfError(RuntimeError):
@@ -71,6 +72,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "rf_plan_create": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
                            i32, i32, ctypes.POINTER(vp)],
+        "rf_plan_create_ex": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
+                              i32, i32, i32, ctypes.POINTER(vp)],
         "rf_plan_info": [vp, ctypes.POINTER(PlanInfo)],
         "rf_plan_seq_info": [vp, i32, ctypes.POINTER(SeqInfo)],
         "rf_rearrange": [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -113,12 +116,16 @@ class Plan:
 
     def __init__(self, seqs: Sequence[Tuple[int, int, int, int]], n1: int, n2: int, d: int,
                  layout: str = "BNSD", dtype: str = "bf16", sparsity: float = 0.8, batch: int = 1,
-                 block_q: int = 128, block_kv: int = 128):
+                 block_q: int = 128, block_kv: int = 128, order: str = "tile"):
         arr = (SeqGeom * max(1, len(seqs)))(*[SeqGeom(*map(int, s)) for s in seqs])
         handle = ctypes.c_void_p()
-        _check(_lib.rf_plan_create(arr, len(seqs), batch, n1, n2, d, LAYOUTS[layout], DTYPES[dtype],
-                                   float(sparsity), block_q, block_kv, ctypes.byref(handle)),
-               "rf_plan_create")
+        if order not in ORDERS:
+            raise ValueError(f"order must be one of {sorted(ORDERS)}")
+        _check(_lib.rf_plan_create_ex(arr, len(seqs), batch, n1, n2, d, LAYOUTS[layout], DTYPES[dtype],
+                                      float(sparsity), block_q, block_kv, ORDERS[order],
+                                      ctypes.byref(handle)),
+               "rf_plan_create_ex")
+        self.order = order
         self._h = handle
         self._lib = _lib  # kept so that destruction at interpreter exit still finds it
         self.layout, self.dtype, self.sparsity, self.batch = layout, dtype, float(sparsity), batch
@@ -311,20 +318,24 @@ def forward(plan: Plan, q, k, v, bufs: Buffers, scale: Optional[float] = None, s
 def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          seqs: Sequence[Tuple[int, int, int, int]], sparsity: float = 0.8,
                          layout: str = "BNSD", scale: Optional[float] = None,
-                         plan: Optional[Plan] = None, bufs: Optional[Buffers] = None) -> torch.Tensor:
+                         plan: Optional[Plan] = None, bufs: Optional[Buffers] = None,
+                         order: str = "tile") -> torch.Tensor:
     """User-level call: RainFusion v2 block-sparse attention of q, k, v (original token order).
 
     q, k, v may live on the host (pinned or not) or on the GPU; the result is
     returned on the device the inputs came from.  BNSD: q [B, N1, L, D],
     k/v [B, N2, L, D]; TND: q [T, N1, D], k/v [T, N2, D].  `seqs` holds one
     (prefix_len, t, h, w) per sequence (BNSD: one for the whole batch).
+    `order` is the token order of the aligned video ("tile", or "frame_pair"
+    for 2x8x8 blocks over frame pairs); it is ignored when `plan` is given.
     """
     dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[q.dtype]
     if plan is None:
         if layout == "BNSD":
-            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[3], "BNSD", dtype, sparsity, batch=q.shape[0])
+            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[3], "BNSD", dtype, sparsity, batch=q.shape[0],
+                        order=order)
         else:
-            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[2], "TND", dtype, sparsity)
+            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[2], "TND", dtype, sparsity, order=order)
     host = not q.is_cuda
     dev = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     if bufs is None:

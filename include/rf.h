@@ -90,6 +90,20 @@ typedef enum {
   RF_POOL_RECOMPUTE = 1  /* recompute them from q_r / k_r first */
 } rf_pool_mode_t;
 
+/* Token order of the aligned video tokens in the rearranged sequence.
+ *   RF_ORDER_TILE       8x8 spatial tiles of one frame in (frame, tile row,
+ *                       tile column, row, column) order: a 128-row block is
+ *                       two adjacent tiles of one frame ([UG] opening
+ *                       paragraph and "Geometry handling": (t, h, w) order).
+ *   RF_ORDER_FRAME_PAIR the frame-pairing variant of [PR] (change summary:
+ *                       frame-pairing approach, first frame before the rest):
+ *                       frame 0 in tile order, then frames (1,2), (3,4), ...
+ *                       cube by cube, a cube being the same 8x8 tile of both
+ *                       frames (128 rows: frame in pair, row, column), then
+ *                       an unpaired last frame in tile order.
+ * Both orders give the same counts (sparse rows, promoted rows, blocks,
+ * sinks); only the order of the aligned tokens differs. */
+typedef enum { RF_ORDER_TILE = 0, RF_ORDER_FRAME_PAIR = 1 } rf_token_order_t;
 /* One sequence: text/condition prefix length and video latent grid
  * ([UG] "Geometry handling").  t, h, w >= 0; prefix_len >= 0; length > 0. */
 typedef struct {
@@ -145,6 +159,15 @@ RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int
                            rf_dtype_t dtype, double sparsity, int32_t block_q,
                            int32_t block_kv, rf_plan_t** out);
 
+/* rf_plan_create with an explicit token order (rf_plan_create uses
+ * RF_ORDER_TILE).  Every other argument and error as rf_plan_create; an
+ * unknown order is RF_ERR_INVALID_ARG.  Every later call on the plan
+ * (rearrange, pooling, selection, inverse, rf_plan_permutation) follows the
+ * plan's order. */
+RF_API rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
+                                     int32_t n1, int32_t n2, int32_t d, rf_layout_t layout,
+                                     rf_dtype_t dtype, double sparsity, int32_t block_q,
+                                     int32_t block_kv, rf_token_order_t order, rf_plan_t** out);
 /* Sizes of a plan (host only). */
 RF_API rf_status_t rf_plan_info(const rf_plan_t* plan, rf_plan_info_t* out);
 

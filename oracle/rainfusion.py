@@ -59,6 +59,7 @@ class SeqGeometry:
     ns: int           # first-frame sink blocks
     k: int            # ranked key blocks kept per sparse query block
     dense: bool       # the whole sequence runs dense (nb < 32)
+    order: str = "tile"  # token order of the aligned video: "tile" or "frame_pair"
 
     @property
     def n_blocks(self) -> int:
@@ -78,15 +79,22 @@ def keep_count(nb: int, sparsity: float) -> int:
     return max(0, min(nb, k))
 
 
-def geometry(prefix_len: int, t: int, h: int, w: int, sparsity: float) -> SeqGeometry:
+ORDERS = ("tile", "frame_pair")
+
+
+def geometry(prefix_len: int, t: int, h: int, w: int, sparsity: float,
+             order: str = "tile") -> SeqGeometry:
     """Sizes of one sequence under suffix promotion ([UG] "Geometry handling").
 
     Video tokens inside whole 8x8 tiles are "aligned".  The sparse region is the
     largest whole number of 128-row blocks of aligned tokens (taken in tile
     order); every other video token (the ragged edge, plus the aligned tokens
     past that last whole block, reading R2) is promoted to the dense prefix.
-    Nothing is padded.
+    Nothing is padded.  The counts do not depend on `order` (it only reorders
+    the aligned tokens, and the first frame leads in both orders).
     """
+    if order not in ORDERS:
+        raise ValueError(f"order must be one of {ORDERS}")
     h8, w8 = TILE * (h // TILE), TILE * (w // TILE)
     aligned = t * h8 * w8
     sparse = BLOCK * (aligned // BLOCK)
@@ -98,7 +106,7 @@ def geometry(prefix_len: int, t: int, h: int, w: int, sparsity: float) -> SeqGeo
     dense = nb < DENSE_MIN_BLOCKS
     k = nb if dense else keep_count(nb, sparsity)
     return SeqGeometry(prefix_len, t, h, w, h8, w8, aligned, sparse, promoted, lp,
-                       lp + sparse, n_pb, nb, ns, k, dense)
+                       lp + sparse, n_pb, nb, ns, k, dense, order)
 
 
 # --------------------------------------------------------------------------------------
@@ -106,21 +114,46 @@ def geometry(prefix_len: int, t: int, h: int, w: int, sparsity: float) -> SeqGeo
 #         [ABS] insight 2, spatiotemporal-aware token permutation).
 # --------------------------------------------------------------------------------------
 
-def video_order(t: int, h: int, w: int) -> List[int]:
+def video_order(t: int, h: int, w: int, order: str = "tile") -> List[int]:
     """V': video raster indices in rearranged order.
 
-    Reading R1: aligned tokens are ordered by (frame, tile row, tile column,
-    row in tile, column in tile), so every 128-row block is two 8x8 tiles of
-    one frame; ragged tokens follow in raster order.  Built by sorting keys.
+    order == "tile" (reading R1): aligned tokens are ordered by (frame, tile
+    row, tile column, row in tile, column in tile), so every 128-row block is
+    two 8x8 tiles of one frame.
+
+    order == "frame_pair" ([PR] change summary: the frame-pairing approach,
+    with the first frame placed before the rest; reading R17): frame 0 comes
+    first, in the single-frame tile order above; frames 1..t-1 are then taken
+    two at a time, (1,2), (3,4), ..., and each pair is laid out cube by cube
+    (tile row, tile column), a cube holding the 8x8 tile of both frames
+    (frame in pair, row in tile, column in tile) -- 128 tokens, one block.  A
+    last frame left without a partner (t even) follows alone, in tile order.
+
+    Ragged tokens follow the aligned ones in raster order in both cases.
+    Built by sorting keys.
     """
+    if order not in ORDERS:
+        raise ValueError(f"order must be one of {ORDERS}")
     h8, w8 = TILE * (h // TILE), TILE * (w // TILE)
+    n_pairs = (t - 1) // 2 if t > 0 else 0
+
+    def group(tau: int) -> Tuple[int, int]:
+        """(frame group, position of the frame inside its group)."""
+        if order == "tile":
+            return tau, 0
+        if tau == 0:
+            return 0, 0
+        if tau <= 2 * n_pairs:
+            return 1 + (tau - 1) // 2, (tau - 1) % 2
+        return 1 + n_pairs, 0           # the unpaired last frame
 
     def key(v: int):
         tau, rem = divmod(v, h * w)
         y, x = divmod(rem, w)
         if y < h8 and x < w8:
-            return (0, tau, y // TILE, x // TILE, y % TILE, x % TILE)
-        return (1, v, 0, 0, 0, 0)
+            grp, fi = group(tau)
+            return (0, grp, y // TILE, x // TILE, fi, y % TILE, x % TILE)
+        return (1, v, 0, 0, 0, 0, 0)
 
     return sorted(range(t * h * w), key=key)
 
@@ -132,7 +165,7 @@ def permutation(g: SeqGeometry) -> np.ndarray:
     [text (original order) | promoted | sparse], reading R3: promoted rows sit
     right after the text and join the always-kept prefix.
     """
-    vp = video_order(g.t, g.h, g.w)
+    vp = video_order(g.t, g.h, g.w, g.order)
     sparse, promoted = vp[:g.sparse], vp[g.sparse:]
     P = g.prefix_len
     src = list(range(P)) + [P + v for v in promoted] + [P + v for v in sparse]
@@ -302,10 +335,10 @@ class Problem:
 
 
 def make_problem(layout: str, batch: int, seqs: Sequence[Tuple[int, int, int, int]],
-                 n1: int, n2: int, d: int, sparsity: float) -> Problem:
+                 n1: int, n2: int, d: int, sparsity: float, order: str = "tile") -> Problem:
     if n1 % n2:
         raise ValueError("N1 must be a multiple of N2 ([API] constraints)")
-    geoms = [geometry(p, t, h, w, sparsity) for (p, t, h, w) in seqs]
+    geoms = [geometry(p, t, h, w, sparsity, order) for (p, t, h, w) in seqs]
     return Problem(layout, batch, geoms, n1, n2, d)
 
 

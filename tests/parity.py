@@ -26,8 +26,8 @@ def seqs_of(w: synth.Workload):
     return [(s.prefix_len, s.t, s.h, s.w) for s in w.seqs]
 
 
-def problem(w: synth.Workload) -> orc.Problem:
-    return orc.make_problem(w.layout, w.batch, seqs_of(w), w.n1, w.n2, w.d, w.sparsity)
+def problem(w: synth.Workload, order: str = "tile") -> orc.Problem:
+    return orc.make_problem(w.layout, w.batch, seqs_of(w), w.n1, w.n2, w.d, w.sparsity, order)
 
 
 def to_device(bits: np.ndarray, dtype: str) -> torch.Tensor:
@@ -39,9 +39,10 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
     return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "from_ws") -> Dict[str, object]:
+def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "from_ws",
+            order: str = "tile") -> Dict[str, object]:
     """Whole path through the C ABI, one call per step; returns host copies of every result."""
-    plan = rf.Plan(seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch)
+    plan = rf.Plan(seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=order)
     q, k, v = (to_device(b, w.dtype) for b in bits)
     b = rf.Buffers(plan)
     scale = 1.0 / math.sqrt(w.d)

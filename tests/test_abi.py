@@ -122,3 +122,36 @@ def test_kernel_index_math_equals_oracle_permutation(name):
 def test_kernel_index_math_ragged_cases(s):
     plan = rf.Plan([s], 1, 1, 64)
     assert np.array_equal(plan.permutation(0), orc.permutation(orc.geometry(*s, 0.8)))
+
+
+# ---------------- frame-pair token order (rf_plan_create_ex) ----------------
+
+@pytest.mark.parametrize("s", [(512, 21, 30, 52), (256, 62, 24, 42), (128, 9, 16, 32), (384, 21, 24, 40),
+                               (77, 9, 17, 33), (0, 6, 24, 40), (5, 3, 7, 9), (1, 2, 8, 8), (0, 1, 3, 3),
+                               (64, 4, 31, 9), (0, 8, 16, 16)])
+def test_frame_pair_index_math_equals_oracle_permutation(s):
+    """The kernels' frame-pair row mapping (run on the host) against the oracle's
+    key sort, bit for bit, with the counts unchanged from the tile order."""
+    plan = rf.Plan([s], 1, 1, 64, order="frame_pair")
+    g = orc.geometry(*s, 0.8, "frame_pair")
+    assert np.array_equal(plan.permutation(0), orc.permutation(g))
+    tile = rf.Plan([s], 1, 1, 64)
+    a, b = plan.seq_info[0], tile.seq_info[0]
+    assert (a.length, a.lp, a.sparse, a.promoted, a.n_pb, a.nb, a.ns, a.k) == \
+           (b.length, b.lp, b.sparse, b.promoted, b.n_pb, b.nb, b.ns, b.k)
+
+
+def test_frame_pair_tnd_sequences_each_follow_the_order():
+    seqs = [(256, 13, 32, 48), (384, 21, 24, 40)]
+    plan = rf.Plan(seqs, 32, 8, 128, "TND", "fp16", 0.8, order="frame_pair")
+    for i, s in enumerate(seqs):
+        assert np.array_equal(plan.permutation(i), orc.permutation(orc.geometry(*s, 0.8, "frame_pair")))
+
+
+def test_unknown_token_order_is_rejected():
+    arr = (rf.SeqGeom * 1)(rf.SeqGeom(128, 9, 16, 32))
+    h = ctypes.c_void_p()
+    st = rf.lib().rf_plan_create_ex(arr, 1, 1, 2, 2, 64, 0, 0, ctypes.c_double(0.8), 128, 128, 7, ctypes.byref(h))
+    assert st == 1 and not h.value
+    with pytest.raises(ValueError):
+        rf.Plan([(128, 9, 16, 32)], 2, 2, 64, order="zigzag")

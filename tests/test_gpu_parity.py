@@ -185,6 +185,49 @@ def test_full_size_parity(name, s):
     parity.check_attention(p, w, rbits, gpu, items)
 
 
+# ------------------------------------------------------------------------------------------
+# Frame-pair token order (xllm PR #1867, frame-pairing approach): the whole path with the
+# permutation of rf_plan_create_ex(RF_ORDER_FRAME_PAIR), against the oracle in the same order.
+# ------------------------------------------------------------------------------------------
+
+FRAME_PAIR = [
+    ("tiny", SMALL["tiny"]),                      # 9 frames: 4 pairs after frame 0
+    ("ragged_d128", SMALL["ragged_d128"]),        # ragged edge promoted, 9 frames
+    ("no_prefix", SMALL["no_prefix"]),            # 6 frames: the last one is unpaired
+    ("tnd_gqa_small", SMALL["tnd_gqa_small"]),    # two sequences, 9 and 10 frames
+]
+
+
+@pytest.mark.parametrize("name,w", FRAME_PAIR, ids=[n for n, _ in FRAME_PAIR])
+def test_frame_pair_small_full_parity(name, w):
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w, order="frame_pair")
+    gpu = parity.run_gpu(w, bits, order="frame_pair")
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 100)
+    parity.check_attention(p, w, rbits, gpu)
+
+
+@pytest.mark.parametrize("name,s", [("wan", None), ("minimax", 0.8)])
+def test_frame_pair_full_size_parity(name, s):
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w, order="frame_pair")
+    gpu = parity.run_gpu(w, bits, order="frame_pair")
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 1000), stats
+    items = parity.sample_items(p, np.random.default_rng(8), per_kind=3)
+    parity.check_attention(p, w, rbits, gpu, items)
+
+
 def test_exp2_polynomial_against_mufu_and_exact():
     """The FMA-pipe exponential the softmax uses for part of its columns:
     relative error <= 2e-4 against the exact 2^x and against ex2.approx,

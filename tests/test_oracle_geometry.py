@@ -144,3 +144,112 @@ def test_short_video_runs_dense():
     assert g.dense and g.k == g.nb
     g = rf.geometry(64, 8, 16, 32, 0.9)             # 32 blocks: not dense
     assert not g.dense and g.nb == 32
+
+
+# ---------------- frame-pair token order ([PR] change summary, reading R17) ----------------
+
+def _nested_loop_frame_pair_order(t, h, w):
+    """Frame-pair order written as explicit loops: frame 0 in tile order, then
+    each frame pair cube by cube (frame in pair inside the cube), then an
+    unpaired last frame in tile order, then the ragged tokens in raster order."""
+    h8, w8 = 8 * (h // 8), 8 * (w // 8)
+
+    def one_frame(tau):
+        out = []
+        for hb in range(h8 // 8):
+            for wb in range(w8 // 8):
+                for hi in range(8):
+                    for wi in range(8):
+                        out.append(tau * h * w + (8 * hb + hi) * w + 8 * wb + wi)
+        return out
+
+    order = one_frame(0) if t > 0 else []
+    tau = 1
+    while tau + 1 < t:
+        for hb in range(h8 // 8):
+            for wb in range(w8 // 8):
+                for fi in range(2):
+                    for hi in range(8):
+                        for wi in range(8):
+                            order.append((tau + fi) * h * w + (8 * hb + hi) * w + 8 * wb + wi)
+        tau += 2
+    if tau < t:
+        order += one_frame(tau)
+    for tau in range(t):
+        for y in range(h):
+            for x in range(w):
+                if y >= h8 or x >= w8:
+                    order.append(tau * h * w + y * w + x)
+    return order
+
+
+@pytest.mark.parametrize("t,h,w", [(1, 8, 8), (2, 16, 24), (3, 13, 21), (4, 30, 52), (5, 8, 16),
+                                   (6, 7, 9), (7, 17, 40), (0, 8, 8)])
+def test_frame_pair_order_equals_nested_loops(t, h, w):
+    assert rf.video_order(t, h, w, "frame_pair") == _nested_loop_frame_pair_order(t, h, w)
+
+
+def test_frame_pair_order_of_one_or_two_frames_is_tile_order():
+    # with t <= 2 no pair exists: frame 0 alone, then (t = 2) the unpaired frame 1
+    for (t, h, w) in [(1, 16, 24), (2, 16, 24), (2, 13, 21)]:
+        assert rf.video_order(t, h, w, "frame_pair") == rf.video_order(t, h, w, "tile")
+
+
+@pytest.mark.parametrize("p,t,h,w", [(128, 9, 16, 32), (512, 3, 30, 52), (0, 4, 24, 42), (7, 1, 5, 5),
+                                     (384, 21, 24, 40), (1, 6, 17, 9)])
+def test_frame_pair_permutation_round_trips_and_keeps_counts(p, t, h, w):
+    g_tile = rf.geometry(p, t, h, w, 0.8)
+    g = rf.geometry(p, t, h, w, 0.8, "frame_pair")
+    # the order changes nothing but the order: every count is the tile order's
+    assert dataclasses_replace_order(g_tile) == g
+    src = rf.permutation(g)
+    assert sorted(src.tolist()) == list(range(g.length))
+    assert np.array_equal(src[:p], np.arange(p))
+    x = np.random.default_rng(1).standard_normal((g.length, 2))
+    assert np.array_equal(rf.inverse_rows(rf.rearrange_rows(x, src), src), x)
+    # the promoted ragged edge is the same set of rows in both orders
+    assert set(src[p:g.lp].tolist()) >= set(
+        v for v in range(p, g.length) if ((v - p) % (h * w)) // w >= g.h8 or (v - p) % w >= g.w8)
+
+
+def dataclasses_replace_order(g):
+    import dataclasses
+    return dataclasses.replace(g, order="frame_pair")
+
+
+def test_frame_pair_blocks_are_spatiotemporal_cubes():
+    # Wan2.2-shaped grid: a frame holds 9 whole blocks, so after the 9 first-frame
+    # (sink) blocks every sparse block is one 2x8x8 cube of two consecutive frames.
+    p, t, h, w = 512, 21, 30, 52
+    g = rf.geometry(p, t, h, w, 0.8, "frame_pair")
+    assert (g.nb, g.ns, g.promoted) == (189, 9, 8568)
+    src = rf.permutation(g)
+    for i in range(g.nb):
+        rows = src[g.lp + 128 * i: g.lp + 128 * (i + 1)] - p
+        tau = rows // (h * w)
+        y = (rows % (h * w)) // w
+        x = rows % w
+        cells = set(zip((y // 8).tolist(), (x // 8).tolist()))
+        frames = sorted(set(tau.tolist()))
+        if i < g.ns:
+            assert frames == [0] and len(cells) == 2       # first frame: two tiles of frame 0
+        else:
+            assert len(cells) == 1                          # one 8x8 spatial tile ...
+            assert frames == [frames[0], frames[0] + 1] and frames[0] % 2 == 1   # ... of frames (2m+1, 2m+2)
+            assert np.array_equal(tau[:64], np.full(64, frames[0]))
+
+
+def test_frame_pair_sinks_cover_exactly_the_first_frame():
+    for (p, t, h, w) in [(128, 9, 16, 32), (256, 62, 24, 42), (512, 21, 30, 52), (0, 4, 8, 16)]:
+        g = rf.geometry(p, t, h, w, 0.8, "frame_pair")
+        src = rf.permutation(g)
+        frame = (src[g.lp:] - p) // (h * w)
+        first_frame_blocks = {i // 128 for i in np.nonzero(frame == 0)[0].tolist()}
+        assert first_frame_blocks == set(range(g.ns))
+
+
+def test_unknown_order_is_rejected():
+    with pytest.raises(ValueError):
+        rf.geometry(0, 2, 8, 8, 0.8, "zigzag")
+    with pytest.raises(ValueError):
+        rf.video_order(2, 8, 8, "zigzag")
