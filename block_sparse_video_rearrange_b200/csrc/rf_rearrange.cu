@@ -13,7 +13,8 @@
 // One CTA moves one 128-row block of one head of one tensor: 16-byte vector
 // loads and stores, whole rows per group of D/8 threads, every load of a
 // thread issued before its first store.  The source of a rearranged row is
-// computed from the geometry (no index table in memory).
+// computed from the geometry (no index table in memory), once per row into
+// shared memory, so that the copy loop runs no index arithmetic.
 #include <cuda_fp16.h>
 
 #include "rf_device.cuh"
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(kThreads)
   constexpr int kRowLanes = kThreads / kChunks;   // rows handled in parallel
   constexpr int kRowsPerThread = RF_BLOCK / kRowLanes;
   __shared__ float red[kRowLanes][D + 4];
+  __shared__ long long src_off[RF_BLOCK], dst_off[RF_BLOCK];  // row offsets in 16-byte units
 
   const int tb = blockIdx.x % g.t_qblk;           // global block
   const int th = blockIdx.x / g.t_qblk;           // tensor-major head index
@@ -71,55 +73,62 @@ __global__ void __launch_bounds__(kThreads)
   const int ch = threadIdx.x % kChunks;
   const int rl = threadIdx.x / kChunks;
 
+  // Source and destination of every row, computed once per row (not once per
+  // 16-byte chunk): the permutation's divisions stay off the copy loop.
+  if (threadIdx.x < nrows) {
+    const int r = r0 + (int)threadIdx.x;
+    const int from = (MODE == kRearrange) ? rf_orig_row(s, r) : r;
+    const int to = (MODE == kInverse) ? rf_orig_row(s, r) : r;
+    src_off[threadIdx.x] = (long long)(rf_row_offset(g, s, heads, head, from) / 8);
+    dst_off[threadIdx.x] = (long long)(rf_row_offset(g, s, heads, head, to) / 8);
+  }
+  __syncthreads();
+
   uint4 val[kRowsPerThread];
 #pragma unroll
   for (int i = 0; i < kRowsPerThread; ++i) {
     const int rr = rl + i * kRowLanes;
     val[i] = make_uint4(0, 0, 0, 0);
-    if (rr < nrows) {
-      const int r = r0 + rr;
-      const int from = (MODE == kRearrange) ? rf_orig_row(s, r) : r;
-      val[i] = __ldg(src + rf_row_offset(g, s, heads, head, from) / 8 + ch);
-    }
+    if (rr < nrows) val[i] = __ldg(src + src_off[rr] + ch);
   }
   if (MODE != kPoolOnly) {
 #pragma unroll
     for (int i = 0; i < kRowsPerThread; ++i) {
       const int rr = rl + i * kRowLanes;
-      if (rr < nrows) {
-        const int r = r0 + rr;
-        const int to = (MODE == kInverse) ? rf_orig_row(s, r) : r;
-        dst[rf_row_offset(g, s, heads, head, to) / 8 + ch] = val[i];
+      if (rr < nrows) dst[dst_off[rr] + ch] = val[i];
+    }
+  }
+  if constexpr (MODE == kInverse) {
+    return;
+  } else {
+    if (!pool) return;  // uniform over the CTA
+
+    // Column sums of the block in fp32 and a fixed order (a lane's rows in
+    // order, then the lanes in order), then the mean.
+    float acc[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[2 * c] += Dec::lo(w[c]);
+        acc[2 * c + 1] += Dec::hi(w[c]);
       }
     }
-  }
-  if (!pool) return;  // uniform over the CTA
-
-  // Column sums of the block in fp32 and a fixed order (a lane's rows in
-  // order, then the lanes in order), then the mean.
-  float acc[8];
 #pragma unroll
-  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-#pragma unroll
-  for (int i = 0; i < kRowsPerThread; ++i) {
-    const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      acc[2 * c] += Dec::lo(w[c]);
-      acc[2 * c + 1] += Dec::hi(w[c]);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float sum = 0.f;
+    for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
+    __syncthreads();
+    if (threadIdx.x < D) {
+      float sum = 0.f;
 #pragma unroll 4
-    for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
-    float* out = tensor == 0 ? pooled_q : pooled_k;
-    const size_t idx =
-        ((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x;
-    out[idx] = sum * (1.0f / RF_BLOCK);
+      for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
+      float* out = tensor == 0 ? pooled_q : pooled_k;
+      const size_t idx =
+          ((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x;
+      out[idx] = sum * (1.0f / RF_BLOCK);
+    }
   }
 }
 

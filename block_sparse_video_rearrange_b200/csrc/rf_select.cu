@@ -12,11 +12,13 @@
 //
 // Two kernels:
 //  1. rf_scores_kernel: per sparse sequence and query head n, the fp32 matrix
-//     scores[i][j] = qbar[n][i] . kbar[n / G][j] (64 x 64 tiles, 4 x 4 per
-//     thread, D chunks staged through shared memory).
+//     scores[i][j] = qbar[n][i] . kbar[n / G][j] (128 x 128 or 64 x 64
+//     tiles, 8 x 8 or 4 x 4 per thread, D chunks double-buffered through
+//     shared memory).
 //  2. rf_topk_kernel: one warp per selectIdx row.  Keys are the scores mapped
 //     to order-preserving 32-bit integers, held in registers (32 lanes x M).
-//     A 32-step radix select finds the k-th largest key; ties at the
+//     A bitwise radix select (over the bits below the keys' common prefix)
+//     finds the k-th largest key; ties at the
 //     threshold go to the lowest block index; sinks are added; the row is
 //     written in ascending order with a ballot prefix sum.  No sorting, no
 //     shared memory, no atomics.
@@ -24,14 +26,24 @@
 
 namespace {
 
-constexpr int kTile = 64;
-constexpr int kKc = 32;
+constexpr int kKc = 16;  // D chunk staged through shared memory (double-buffered)
 
-__global__ void __launch_bounds__(256)
+// One CTA computes a (16 TT) x (16 TT) tile of scores for one (sequence, query
+// head): 256 threads, TT x TT results each (rows q*64 + ty*4 + {0..3} for the
+// TT/4 quadrants q, columns likewise with tx), so every inner step is TT/2
+// 16-byte shared loads feeding TT*TT fp32 FMAs.  The next D chunk is fetched
+// into registers while the current one is multiplied.  TT = 8 (128 x 128
+// tiles) for large problems, TT = 4 (64 x 64) when the large tiles would not
+// fill the GPU twice over.
+template <int TT>
+__global__ void __launch_bounds__(256, 2)
     rf_scores_kernel(const RfGeomDev g, const float* __restrict__ pq, const float* __restrict__ pk,
                      float* __restrict__ scores) {
-  __shared__ float As[kKc][kTile + 4];
-  __shared__ float Bs[kKc][kTile + 4];
+  constexpr int kTile = 16 * TT;
+  constexpr int kQ = TT / 4;                       // 64-row quadrants per tile edge
+  constexpr int kReps = kTile * kKc / 4 / 256;     // float4 per thread per operand chunk
+  __shared__ __align__(16) float As[2][kKc][kTile + 4];
+  __shared__ __align__(16) float Bs[2][kKc][kTile + 4];
   // Decode blockIdx.x into (instance, head, tile row, tile col) over the
   // non-dense instances in order.
   int rem = blockIdx.x;
@@ -54,47 +66,71 @@ __global__ void __launch_bounds__(256)
   const float* B = pk + ((size_t)gk * g.pooled_total + s.pool_off) * g.d;
   const int i0 = tr * kTile, j0 = tc * kTile;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
 
-  for (int k0 = 0; k0 < g.d; k0 += kKc) {
-    // 64 rows x 32 k of A and of B: 512 float4 each, 2 per thread.
+  float4 pa[kReps], pb[kReps];
+  auto fetch = [&](int k0) {
 #pragma unroll
-    for (int rep = 0; rep < 2; ++rep) {
+    for (int rep = 0; rep < kReps; ++rep) {
       const int e = threadIdx.x + rep * 256;
-      const int row = e / (kKc / 4), c4 = e % (kKc / 4);
-      float4 va = make_float4(0.f, 0.f, 0.f, 0.f), vb = va;
-      if (i0 + row < s.nb) va = *reinterpret_cast<const float4*>(A + (size_t)(i0 + row) * g.d + k0 + 4 * c4);
-      if (j0 + row < s.nb) vb = *reinterpret_cast<const float4*>(B + (size_t)(j0 + row) * g.d + k0 + 4 * c4);
-      As[4 * c4 + 0][row] = va.x; As[4 * c4 + 1][row] = va.y;
-      As[4 * c4 + 2][row] = va.z; As[4 * c4 + 3][row] = va.w;
-      Bs[4 * c4 + 0][row] = vb.x; Bs[4 * c4 + 1][row] = vb.y;
-      Bs[4 * c4 + 2][row] = vb.z; Bs[4 * c4 + 3][row] = vb.w;
+      const int row = e >> 2, c4 = e & 3;
+      pa[rep] = make_float4(0.f, 0.f, 0.f, 0.f);
+      pb[rep] = pa[rep];
+      if (i0 + row < s.nb) pa[rep] = *reinterpret_cast<const float4*>(A + (size_t)(i0 + row) * g.d + k0 + 4 * c4);
+      if (j0 + row < s.nb) pb[rep] = *reinterpret_cast<const float4*>(B + (size_t)(j0 + row) * g.d + k0 + 4 * c4);
     }
-    __syncthreads();
-#pragma unroll 8
+  };
+  auto stash = [&](int buf) {
+#pragma unroll
+    for (int rep = 0; rep < kReps; ++rep) {
+      const int e = threadIdx.x + rep * 256;
+      const int row = e >> 2, c4 = e & 3;
+      As[buf][4 * c4 + 0][row] = pa[rep].x; As[buf][4 * c4 + 1][row] = pa[rep].y;
+      As[buf][4 * c4 + 2][row] = pa[rep].z; As[buf][4 * c4 + 3][row] = pa[rep].w;
+      Bs[buf][4 * c4 + 0][row] = pb[rep].x; Bs[buf][4 * c4 + 1][row] = pb[rep].y;
+      Bs[buf][4 * c4 + 2][row] = pb[rep].z; Bs[buf][4 * c4 + 3][row] = pb[rep].w;
+    }
+  };
+
+  float acc[TT][TT];
+#pragma unroll
+  for (int a = 0; a < TT; ++a)
+#pragma unroll
+    for (int b = 0; b < TT; ++b) acc[a][b] = 0.f;
+
+  fetch(0);
+  stash(0);
+  __syncthreads();
+  const int chunks = g.d / kKc;
+#pragma unroll 1
+  for (int c = 0; c < chunks; ++c) {
+    const int buf = c & 1;
+    if (c + 1 < chunks) fetch((c + 1) * kKc);
+#pragma unroll
     for (int kk = 0; kk < kKc; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+      float av[TT], bv[TT];
 #pragma unroll
-      for (int x = 0; x < 4; ++x)
+      for (int q = 0; q < kQ; ++q) {
+        const float4 a4 = *reinterpret_cast<const float4*>(&As[buf][kk][q * 64 + ty * 4]);
+        const float4 b4 = *reinterpret_cast<const float4*>(&Bs[buf][kk][q * 64 + tx * 4]);
+        av[4 * q] = a4.x; av[4 * q + 1] = a4.y; av[4 * q + 2] = a4.z; av[4 * q + 3] = a4.w;
+        bv[4 * q] = b4.x; bv[4 * q + 1] = b4.y; bv[4 * q + 2] = b4.z; bv[4 * q + 3] = b4.w;
+      }
 #pragma unroll
-        for (int y = 0; y < 4; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
+      for (int x = 0; x < TT; ++x)
+#pragma unroll
+        for (int y = 0; y < TT; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
+    if (c + 1 < chunks) stash(buf ^ 1);
     __syncthreads();
   }
   float* C = scores + s.score_off + (size_t)n * s.nb * s.nb;
 #pragma unroll
-  for (int x = 0; x < 4; ++x) {
-    const int i = i0 + ty * 4 + x;
+  for (int x = 0; x < TT; ++x) {
+    const int i = i0 + (x >> 2) * 64 + ty * 4 + (x & 3);
     if (i >= s.nb) continue;
 #pragma unroll
-    for (int y = 0; y < 4; ++y) {
-      const int j = j0 + tx * 4 + y;
+    for (int y = 0; y < TT; ++y) {
+      const int j = j0 + (y >> 2) * 64 + tx * 4 + (y & 3);
       if (j < s.nb) C[(size_t)i * s.nb + j] = acc[x][y];
     }
   }
@@ -138,10 +174,24 @@ __global__ void __launch_bounds__(256)
   const int k = s.k;
   unsigned long long sel = 0;  // bit m: block lane + 32m is kept
   if (k > 0) {
-    // Largest T with #{key >= T} >= k, one bit at a time from the top.
-    uint32_t T = 0;
+    // Largest T with #{key >= T} >= k, one bit at a time from the top.  All
+    // keys of the row share the bits above the highest bit in which the
+    // smallest and the largest differ, so T starts as that common prefix and
+    // the search runs over the bits below it only.
+    uint32_t kmax = 0u, kmin = 0xFFFFFFFFu;
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+      if (lane + 32 * m < s.nb) {
+        kmax = max(kmax, key[m]);
+        kmin = min(kmin, key[m]);
+      }
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    const uint32_t diff = kmax ^ kmin;
+    const int top = diff ? 31 - __clz(diff) : -1;
+    uint32_t T = diff ? (kmin & ~((2u << top) - 1u)) : kmin;
 #pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
+    for (int bit = top; bit >= 0; --bit) {
       const uint32_t cand = T | (1u << bit);
       int cnt = 0;
 #pragma unroll
@@ -191,14 +241,22 @@ rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_nu
   const float* pq = reinterpret_cast<const float*>(static_cast<char*>(ws) + p->off_pq);
   const float* pk = reinterpret_cast<const float*>(static_cast<char*>(ws) + p->off_pk);
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + p->off_scores);
-  long long tiles = 0;
+  // Tiles of 128 x 128 once they fill the GPU at least twice over (two CTAs
+  // per SM), else 64 x 64 tiles for more parallelism.
+  long long tiles64 = 0, tiles128 = 0;
   for (int i = 0; i < g.n_seqs; ++i) {
     if (g.seq[i].dense) continue;
-    const long long tn = (g.seq[i].nb + kTile - 1) / kTile;
-    tiles += (long long)g.n1 * tn * tn;
+    const long long t64 = (g.seq[i].nb + 63) / 64, t128 = (g.seq[i].nb + 127) / 128;
+    tiles64 += (long long)g.n1 * t64 * t64;
+    tiles128 += (long long)g.n1 * t128 * t128;
   }
-  if (tiles > 0) {
-    rf_scores_kernel<<<(unsigned)tiles, 256, 0, st>>>(g, pq, pk, scores);
+  if (tiles64 > 0) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaGetLastError();
+    if (tiles128 >= 4ll * sms) rf_scores_kernel<8><<<(unsigned)tiles128, 256, 0, st>>>(g, pq, pk, scores);
+    else                       rf_scores_kernel<4><<<(unsigned)tiles64, 256, 0, st>>>(g, pq, pk, scores);
     rf_status_t s = rf_check_launch("rf_scores_kernel");
     if (s != RF_OK) return s;
   }
@@ -207,6 +265,7 @@ rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_nu
   const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
   if (g.max_nb <= 256)       rf_topk_kernel<8><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
   else if (g.max_nb <= 512)  rf_topk_kernel<16><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nb <= 640)  rf_topk_kernel<20><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
   else if (g.max_nb <= 1024) rf_topk_kernel<32><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
   else                       rf_topk_kernel<64><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
   return rf_check_launch("rf_topk_kernel");
