@@ -450,3 +450,95 @@ def kept_flops(p: Problem, idx: np.ndarray, num: np.ndarray) -> int:
             kv = sum(len(block_rows(g, int(j))) for j in idx[t, n, :num[t, n]])
             total += 4 * p.d * mq * kv
     return total
+
+
+# --------------------------------------------------------------------------------------
+# "mix" kernel precision ([UG] "Configuration": precision "bf16" | "fp8" | "mix";
+# "Wan2.2 T2V quantization on Ascend": FP8 block-sparse attention).  The pages give the
+# names only; reading R18: in "mix", Q and K are quantized to FP8 E4M3 with one scale per
+# (head, 128-row block) and Q K^T runs on those codes; P and V stay 16-bit.
+# --------------------------------------------------------------------------------------
+
+E4M3_MAX = 448.0     # largest finite E4M3 magnitude (S.1111.110)
+
+
+def e4m3_value(code: int) -> float:
+    """Value of an FP8 E4M3 code: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa
+    bits, subnormals at exponent 0, no infinities, S.1111.111 is NaN."""
+    sign = -1.0 if code & 0x80 else 1.0
+    e = (code >> 3) & 0xF
+    m = code & 0x7
+    if e == 0xF and m == 0x7:
+        return math.nan
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+_E4M3_POS = np.array([e4m3_value(c) for c in range(0x7F)], dtype=np.float64)  # codes 0..126, increasing
+
+
+def e4m3_round(x: np.ndarray) -> np.ndarray:
+    """uint8 E4M3 codes of x: round to the nearest representable value, ties to the
+    even code (mantissa LSB 0), magnitudes beyond 448 saturate to 448; the sign bit
+    follows the sign of x (negative zero included)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, len(_E4M3_POS) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo = a - _E4M3_POS[lo]
+    d_hi = _E4M3_POS[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    return code | np.where(np.signbit(x), np.uint8(0x80), np.uint8(0))
+
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """float64 values of E4M3 codes (finite codes only)."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    mag = _E4M3_POS[np.minimum(codes & 0x7F, 0x7E)]
+    return np.where(codes & 0x80, -mag, mag)
+
+
+def quantize_block_e4m3(x: np.ndarray) -> Tuple[np.ndarray, np.float32]:
+    """One block (rows x D) of 16-bit values, given as float32: E4M3 codes and the
+    float32 dequantization scale, in the arithmetic reading R18 fixes:
+    amax = max |x|; inv = 448 / amax and scale = amax / 448 (each one float32
+    division, round to nearest even); codes = E4M3(x * inv) with the product a
+    float32 multiply.  An all-zero block has inv = scale = 1."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    if amax == 0:
+        inv, scale = np.float32(1), np.float32(1)
+    else:
+        inv = np.float32(np.float32(E4M3_MAX) / amax)
+        scale = np.float32(amax / np.float32(E4M3_MAX))
+    y = (x * inv).astype(np.float32)
+    return e4m3_round(y), scale
+
+
+def quantize_e4m3(p: Problem, x_r: np.ndarray, heads: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Per (head, block) E4M3 quantization of a rearranged tensor (float32 values in
+    the BNSD or TND layout of x_r): uint8 codes shaped like x_r and float32 scales
+    [heads, T_qblk] indexed by global query-block number."""
+    codes = np.zeros(x_r.shape, dtype=np.uint8)
+    scales = np.ones((heads, p.t_qblk), dtype=np.float32)
+    for t, (s, g, b) in enumerate(qblock_table(p)):
+        r = block_rows(g, b)
+        for n in range(heads):
+            src = p.head_rows(x_r, s, n)
+            c, sc = quantize_block_e4m3(src[r.start:r.stop])
+            p.head_rows(codes, s, n)[r.start:r.stop] = c
+            scales[n, t] = sc
+    return codes, scales
+
+
+def dequantize_e4m3(p: Problem, codes: np.ndarray, scales: np.ndarray, heads: int) -> np.ndarray:
+    """float64 values code * scale of its (head, block), in the layout of codes."""
+    out = np.zeros(codes.shape, dtype=np.float64)
+    for t, (s, g, b) in enumerate(qblock_table(p)):
+        r = block_rows(g, b)
+        for n in range(heads):
+            v = e4m3_decode(p.head_rows(codes, s, n)[r.start:r.stop]) * np.float64(scales[n, t])
+            p.head_rows(out, s, n)[r.start:r.stop] = v
+    return out
