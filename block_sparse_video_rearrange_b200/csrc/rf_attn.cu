@@ -67,17 +67,21 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchReg
 #endif
 constexpr uint32_t kEmuPairMask = RF_EMU_PAIR_MASK;  // bit i: pair i of every 16 column pairs uses rf_exp2_poly
 constexpr int kStagesK = 3;  // K ring: K_{j+3} is requested as soon as S_j is done
-constexpr int kStagesV = 2;  // V ring: V_{j+2} is requested as soon as O += P_j V_j is done
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy rescale while growth <= 256x
 
-template <int D>
+// kQk8: Q and K tiles hold E4M3 codes (precision "mix"), one byte per element.
+template <int D, bool kQk8>
 struct __align__(1024) AttnSmem {
-  static constexpr int kTileBytes = RF_BLOCK * D * 2;  // 128 rows x D x 16-bit
-  uint8_t q[kTileBytes];
-  uint8_t k[kStagesK][kTileBytes];
-  uint8_t v[kStagesV][kTileBytes];
+  static constexpr int kQkTileBytes = RF_BLOCK * D * (kQk8 ? 1 : 2);
+  static constexpr int kVTileBytes = RF_BLOCK * D * 2;   // 128 rows x D x 16-bit
+  // V ring: V_{j+kStagesV} is requested as soon as O += P_j V_j is done.  The
+  // one-byte Q and K tiles leave room for a third V stage.
+  static constexpr int kStagesV = kQk8 ? 3 : 2;
+  uint8_t q[kQkTileBytes];
+  uint8_t k[kStagesK][kQkTileBytes];
+  uint8_t v[kStagesV][kVTileBytes];
   uint64_t bar_q;
   uint64_t bar_k_full[kStagesK], bar_k_empty[kStagesK];
   uint64_t bar_v_full[kStagesV], bar_v_empty[kStagesV];
@@ -90,6 +94,7 @@ struct __align__(1024) AttnSmem {
   float row_m[2][RF_BLOCK];
   float row_l[2][RF_BLOCK];
   int list[RF_MAX_KV_LIST];
+  float kscale[kQk8 ? RF_MAX_KV_LIST : 1];  // dequantization scale of K block list[j]
 };
 
 struct AttnArgs {
@@ -98,6 +103,8 @@ struct AttnArgs {
   const int32_t* sel_num;
   uint16_t* o_r;
   uint32_t* status;
+  const float* q_scale;  // precision "mix": E4M3 scales [n1][t_qblk] and [n2][t_qblk]
+  const float* k_scale;
   float sl2;  // scale * log2(e)
 };
 
@@ -172,15 +179,20 @@ __device__ __forceinline__ float row_exp(const uint32_t* sr, int vr, float sl2, 
   return s;
 }
 
-template <int D, bool kBf16>
+template <int D, bool kBf16, bool kQk8>
 __global__ void __launch_bounds__(kThreads, 1)
     rf_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
+  using Smem = AttnSmem<D, kQk8>;
   extern __shared__ uint8_t smem_raw[];
-  AttnSmem<D>& sm = *reinterpret_cast<AttnSmem<D>*>(
+  Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  constexpr int kBoxes = D / 64;  // 64-column (128-byte) swizzle boxes per tile row
-  constexpr uint32_t kTileBytes = AttnSmem<D>::kTileBytes;
+  // Tiles are read as 128-byte-wide swizzle boxes of 128 rows.
+  constexpr int kQkBoxes = D * (kQk8 ? 1 : 2) / 128;  // boxes per Q or K tile
+  constexpr int kVBoxes = D * 2 / 128;                // boxes per V tile
+  constexpr uint32_t kQkTileBytes = Smem::kQkTileBytes;
+  constexpr uint32_t kVTileBytes = Smem::kVTileBytes;
+  constexpr int kStagesV = Smem::kStagesV;
   constexpr uint32_t kBoxBytes = RF_BLOCK * 128;
 
   const RfGeomDev& g = a.g;
@@ -243,7 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = c < num && v >= 0 && v < nblk;
       if (c < num && v != -1 && !ok) ++bad;
       const uint32_t ball = __ballot_sync(0xffffffffu, ok);
-      if (ok) sm.list[cnt + __popc(ball & lt)] = v;
+      if (ok) {
+        sm.list[cnt + __popc(ball & lt)] = v;
+        if constexpr (kQk8) sm.kscale[cnt + __popc(ball & lt)] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
+      }
       cnt += __popc(ball);
     }
     bad = __reduce_add_sync(0xffffffffu, bad);
@@ -275,12 +290,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bq = rf_smem_u32(&sm.bar_q);
     if (is_k) {
       coords(g.n1, n, q_r0, c1, c2);
-      mbar_arrive_expect_tx(bq, kTileBytes);
+      mbar_arrive_expect_tx(bq, kQkTileBytes);
 #pragma unroll
-      for (int x = 0; x < kBoxes; ++x)
+      for (int x = 0; x < kQkBoxes; ++x)
         tma_load_3d(rf_smem_u32(sm.q + x * kBoxBytes), &tm_q, bq, x * 64, c1, c2);
     }
     const int stages = is_k ? kStagesK : kStagesV;
+    const uint32_t tile_bytes = is_k ? kQkTileBytes : kVTileBytes;
+    const int boxes = is_k ? kQkBoxes : kVBoxes;
     uint8_t* tiles = is_k ? &sm.k[0][0] : &sm.v[0][0];
     uint64_t* full = is_k ? sm.bar_k_full : sm.bar_v_full;
     uint64_t* empty = is_k ? sm.bar_k_empty : sm.bar_v_empty;
@@ -297,10 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       rf_block_span(s, sm.list[j], r0, nr);
       coords(g.n2, gk, r0, c1, c2);
       const uint32_t bar = rf_smem_u32(&full[st]);
-      mbar_arrive_expect_tx(bar, kTileBytes);
-#pragma unroll
-      for (int x = 0; x < kBoxes; ++x)
-        tma_load_3d(rf_smem_u32(tiles + st * kTileBytes + x * kBoxBytes), map, bar, x * 64, c1, c2);
+      mbar_arrive_expect_tx(bar, tile_bytes);
+      for (int x = 0; x < boxes; ++x)
+        tma_load_3d(rf_smem_u32(tiles + st * tile_bytes + x * kBoxBytes), map, bar, x * 64, c1, c2);
       issued = j + 1;
     }
     if (*abort) {
@@ -317,23 +333,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // descriptors in uniform registers); one elected lane issues every MMA
     // and every commit, so the commits track all of them.
     const uint32_t fmt = kBf16 ? 1u : 0u;
-    const uint32_t idesc_qk = umma_idesc_f16(fmt, 128, 128, 0);
+    // kind::f8f6f4 takes E4M3 as format 0 in the same descriptor fields.
+    const uint32_t idesc_qk = umma_idesc_f16(kQk8 ? 0u : fmt, 128, 128, 0);
     const uint32_t idesc_pv = umma_idesc_f16(fmt, 128, D, 1);
     // Adding (bytes >> 4) to a descriptor moves its 14-bit start-address field.
     const uint64_t dq = umma_desc_sw128(rf_smem_u32(sm.q), 16, 1024);
     const uint64_t dk0 = umma_desc_sw128(rf_smem_u32(sm.k[0]), 16, 1024);
     const uint64_t dv0 = umma_desc_sw128(rf_smem_u32(sm.v[0]), kBoxBytes, 1024);
-    // S_j = Q K_j^T into the S buffer of warpgroup j % 2.
+    // S_j = Q K_j^T into the S buffer of warpgroup j % 2.  Every MMA takes a
+    // 32-byte slice of the reduction (16 bf16/fp16 or 32 E4M3 elements).
     auto issue_qk = [&](int j) -> bool {
       const int st = j % kStagesK;
       if (!warp_wait(rf_smem_u32(&sm.bar_k_full[st]), (j / kStagesK) & 1, abort)) return false;
       tc_fence_after();
       if (elect_one()) {
-        const uint64_t dk = dk0 + (uint64_t)(st * (kTileBytes >> 4));
+        const uint64_t dk = dk0 + (uint64_t)(st * (kQkTileBytes >> 4));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < (int)(kQkTileBytes / RF_BLOCK / 32); ++kk) {
           const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
-          mma_ss(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+          if constexpr (kQk8)
+            mma_ss_f8(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(rf_smem_u32(&sm.bar_s_full[j & 1]));
         tc_commit(rf_smem_u32(&sm.bar_k_empty[st]));
@@ -350,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       if (elect_one()) {
-        const uint64_t dv = dv0 + (uint64_t)(st * (kTileBytes >> 4));
+        const uint64_t dv = dv0 + (uint64_t)(st * (kVTileBytes >> 4));
 #pragma unroll
         for (int kk = 0; kk < RF_BLOCK / 16; ++kk)
           mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)),
@@ -380,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = (warp & 3) * 32 + lane;   // query row = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t s_col = wg * 128, o_col = 256 + wg * 128;
-    const float sl2 = a.sl2;
+    // precision "mix": S_j carries the E4M3 scales of the Q block and of K block j
+    const float sl2_q = kQk8 ? a.sl2 * a.q_scale[(size_t)n * g.t_qblk + tb] : a.sl2;
     const int my_blocks = (nv + 1 - wg) >> 1;  // blocks j < nv with j % 2 == wg
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -389,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!warp_wait(rf_smem_u32(&sm.bar_s_full[wg]), i & 1, abort)) { ok = false; break; }
       tc_fence_after();
       const int vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;  // uniform over the CTA
+      const float sl2 = kQk8 ? sl2_q * sm.kscale[j] : sl2_q;
       const uint32_t scol = lane_base + s_col;
       uint32_t sr[128];
       tmem_ld32(scol, sr);
@@ -517,26 +540,30 @@ EncodeTiledFn encode_fn() {
 }
 
 // Tensor map over [rows, heads, D] (TND) or [B*heads, rows, D] (BNSD) with a
-// 128-row x 64-column box and 128-byte swizzle.
-rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int heads) {
+// 128-row x 128-byte box and 128-byte swizzle: 64 columns of a 16-bit tensor,
+// or 128 columns of a one-byte (E4M3) tensor.
+rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int heads, bool one_byte) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return rf_fail(RF_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const RfGeomDev& g = p->g;
   const cuuint64_t d = (cuuint64_t)g.d;
+  const cuuint64_t esz = one_byte ? 1 : 2;
+  const cuuint32_t box_cols = one_byte ? 128 : 64;
   cuuint64_t dims[3], strides[2];
   cuuint32_t box[3], estr[3] = {1, 1, 1};
   if (g.layout == RF_LAYOUT_BNSD) {
     const cuuint64_t L = (cuuint64_t)g.seq[0].L;
     dims[0] = d; dims[1] = L; dims[2] = (cuuint64_t)p->batch * heads;
-    strides[0] = d * 2; strides[1] = L * d * 2;
-    box[0] = 64; box[1] = RF_BLOCK; box[2] = 1;
+    strides[0] = d * esz; strides[1] = L * d * esz;
+    box[0] = box_cols; box[1] = RF_BLOCK; box[2] = 1;
   } else {
     dims[0] = d; dims[1] = (cuuint64_t)heads; dims[2] = (cuuint64_t)p->rows_total;
-    strides[0] = d * 2; strides[1] = (cuuint64_t)heads * d * 2;
-    box[0] = 64; box[1] = 1; box[2] = RF_BLOCK;
+    strides[0] = d * esz; strides[1] = (cuuint64_t)heads * d * esz;
+    box[0] = box_cols; box[1] = 1; box[2] = RF_BLOCK;
   }
-  const CUtensorMapDataType dt =
-      p->dtype == RF_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType dt = one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : p->dtype == RF_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -545,14 +572,14 @@ rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int hea
   return RF_OK;
 }
 
-template <int D, bool kBf16>
+template <int D, bool kBf16, bool kQk8>
 rf_status_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const AttnArgs& args, unsigned grid, cudaStream_t st) {
-  size_t smem = sizeof(AttnSmem<D>) + 1024;
+  size_t smem = sizeof(AttnSmem<D, kQk8>) + 1024;
   // D = 64 tiles are small: ask for enough shared memory that one CTA holds
   // an SM, since each CTA takes all 512 TMEM columns.
   if (smem < 120 * 1024) smem = 120 * 1024;
-  auto kern = rf_attn_kernel<D, kBf16>;
+  auto kern = rf_attn_kernel<D, kBf16, kQk8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return rf_check_launch("cudaFuncSetAttribute(rf_attn_kernel)");
@@ -581,22 +608,33 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   if (grid > 0x7FFFFFFFll) return rf_fail(RF_ERR_INVALID_ARG, "grid too large");
   CUtensorMap mq, mk, mv;
   rf_status_t s;
-  if ((s = make_map(&mq, p, q_r, g.n1)) != RF_OK) return s;
-  if ((s = make_map(&mk, p, k_r, g.n2)) != RF_OK) return s;
-  if ((s = make_map(&mv, p, v_r, g.n2)) != RF_OK) return s;
+  // precision "mix": Q K^T reads the E4M3 copies rf_rearrange wrote into ws.
+  const bool mix = p->precision == RF_PRECISION_MIX;
+  char* w = static_cast<char*>(ws);
+  const void* qsrc = mix ? static_cast<const void*>(w + p->off_q8) : q_r;
+  const void* ksrc = mix ? static_cast<const void*>(w + p->off_k8) : k_r;
+  if ((s = make_map(&mq, p, qsrc, g.n1, mix)) != RF_OK) return s;
+  if ((s = make_map(&mk, p, ksrc, g.n2, mix)) != RF_OK) return s;
+  if ((s = make_map(&mv, p, v_r, g.n2, false)) != RF_OK) return s;
   AttnArgs args;
   args.g = g;
   args.sel_idx = sel_idx;
   args.sel_num = sel_num;
   args.o_r = static_cast<uint16_t*>(o_r);
-  args.status = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + p->off_status);
+  args.status = reinterpret_cast<uint32_t*>(w + p->off_status);
+  args.q_scale = mix ? reinterpret_cast<const float*>(w + p->off_qs) : nullptr;
+  args.k_scale = mix ? reinterpret_cast<const float*>(w + p->off_ks) : nullptr;
   args.sl2 = scale * kLog2e;
   const bool bf = p->dtype == RF_BF16;
-  if (g.d == 128)
-    return bf ? launch_t<128, true>(mq, mk, mv, args, (unsigned)grid, st)
-              : launch_t<128, false>(mq, mk, mv, args, (unsigned)grid, st);
-  return bf ? launch_t<64, true>(mq, mk, mv, args, (unsigned)grid, st)
-            : launch_t<64, false>(mq, mk, mv, args, (unsigned)grid, st);
+  if (g.d == 128) {
+    if (mix)
+      return bf ? launch_t<128, true, true>(mq, mk, mv, args, (unsigned)grid, st)
+                : launch_t<128, false, true>(mq, mk, mv, args, (unsigned)grid, st);
+    return bf ? launch_t<128, true, false>(mq, mk, mv, args, (unsigned)grid, st)
+              : launch_t<128, false, false>(mq, mk, mv, args, (unsigned)grid, st);
+  }
+  return bf ? launch_t<64, true, false>(mq, mk, mv, args, (unsigned)grid, st)
+            : launch_t<64, false, false>(mq, mk, mv, args, (unsigned)grid, st);
 }
 
 rf_status_t rf_launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,

@@ -108,17 +108,31 @@ rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t ba
                            int32_t n2, int32_t d, rf_layout_t layout, rf_dtype_t dtype,
                            double sparsity, int32_t block_q, int32_t block_kv, rf_plan_t** out) {
   return rf_plan_create_ex(seqs, n_seqs, batch, n1, n2, d, layout, dtype, sparsity, block_q,
-                           block_kv, RF_ORDER_TILE, out);
+                           block_kv, nullptr, out);
 }
 
 rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
                               int32_t n1, int32_t n2, int32_t d, rf_layout_t layout,
                               rf_dtype_t dtype, double sparsity, int32_t block_q,
-                              int32_t block_kv, rf_token_order_t order, rf_plan_t** out) {
+                              int32_t block_kv, const rf_plan_options_t* options,
+                              rf_plan_t** out) {
   g_last_error.clear();
   if (!out || !seqs) return rf_fail(RF_ERR_INVALID_ARG, "null seqs or out");
-  if (order != RF_ORDER_TILE && order != RF_ORDER_FRAME_PAIR)
+  rf_plan_options_t opt;
+  std::memset(&opt, 0, sizeof(opt));
+  if (options) opt = *options;
+  for (int i = 0; i < 6; ++i)
+    if (opt.reserved[i] != 0) return rf_fail(RF_ERR_INVALID_ARG, "reserved option fields must be zero");
+  if (opt.token_order != RF_ORDER_TILE && opt.token_order != RF_ORDER_FRAME_PAIR)
     return rf_fail(RF_ERR_INVALID_ARG, "token order must be RF_ORDER_TILE or RF_ORDER_FRAME_PAIR");
+  if (opt.precision != RF_PRECISION_NATIVE && opt.precision != RF_PRECISION_MIX &&
+      opt.precision != RF_PRECISION_FP8)
+    return rf_fail(RF_ERR_INVALID_ARG, "unknown precision");
+  if (opt.precision == RF_PRECISION_FP8)
+    return rf_fail(RF_ERR_UNSUPPORTED, "precision fp8 (FP8 P V) is not built; use mix");
+  if (opt.precision == RF_PRECISION_MIX && d != 128)
+    return rf_fail(RF_ERR_UNSUPPORTED, "precision mix is built for head dim 128 only");
+  const rf_token_order_t order = (rf_token_order_t)opt.token_order;
   if (layout != RF_LAYOUT_BNSD && layout != RF_LAYOUT_TND)
     return rf_fail(RF_ERR_INVALID_ARG, "layout must be BNSD or TND");
   if (dtype != RF_BF16 && dtype != RF_FP16)
@@ -227,6 +241,21 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   off = align_up(off + (int64_t)n2 * pooled * d * 4, 256);
   p->off_scores = off;
   off = align_up(off + scores * 4, 256);
+  // RF_PRECISION_MIX: E4M3 copies of Q' and K' (one byte per element, the
+  // layouts of q_r / k_r) and their fp32 scales per (head, query block).
+  p->precision = (rf_precision_t)opt.precision;
+  p->token_order = order;
+  p->off_q8 = p->off_k8 = p->off_qs = p->off_ks = -1;
+  if (p->precision == RF_PRECISION_MIX) {
+    p->off_q8 = off;
+    off = align_up(off + p->rows_total * n1 * d, 256);
+    p->off_k8 = off;
+    off = align_up(off + p->rows_total * n2 * d, 256);
+    p->off_qs = off;
+    off = align_up(off + (int64_t)n1 * qblk * 4, 256);
+    p->off_ks = off;
+    off = align_up(off + (int64_t)n2 * qblk * 4, 256);
+  }
   p->ws_bytes = off;
   *out = p;
   return RF_OK;
@@ -246,6 +275,12 @@ rf_status_t rf_plan_info(const rf_plan_t* p, rf_plan_info_t* out) {
   out->n1 = p->g.n1;
   out->n2 = p->g.n2;
   out->d = p->g.d;
+  out->precision = p->precision;
+  out->token_order = p->token_order;
+  out->ws_q8 = p->off_q8;
+  out->ws_k8 = p->off_k8;
+  out->ws_q_scale = p->off_qs;
+  out->ws_k_scale = p->off_ks;
   return RF_OK;
 }
 
@@ -293,6 +328,20 @@ rf_status_t rf_rearrange(const rf_plan_t* p, const void* q, const void* k, const
   if (st != RF_OK) return st;
   if ((st = rf_require_device()) != RF_OK) return st;
   return rf_launch_rearrange(p, q, k, v, q_r, k_r, v_r, ws, (cudaStream_t)stream);
+}
+
+rf_status_t rf_quantize_qk(const rf_plan_t* p, const void* q_r, const void* k_r, void* ws,
+                           size_t ws_bytes, rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (p->precision != RF_PRECISION_MIX)
+    return rf_fail(RF_ERR_INVALID_ARG, "rf_quantize_qk needs a plan with precision mix");
+  if (!q_r || !k_r || !aligned16(q_r) || !aligned16(k_r))
+    return rf_fail(RF_ERR_INVALID_ARG, "q_r and k_r must be non-null and 16-byte aligned");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  return rf_launch_quantize(p, q_r, k_r, ws, (cudaStream_t)stream);
 }
 
 rf_status_t rf_pool_select(const rf_plan_t* p, const void* q_r, const void* k_r,

@@ -1,7 +1,7 @@
 // Token permutation kernels (HBM-bound): rf_rearrange for Q, K and V in one
 // launch with the block means of Q and K fused in, the inverse permutation of
-// the output, and a stand-alone block-mean pass over already-rearranged
-// tensors.
+// the output, and stand-alone block-mean and E4M3 passes over
+// already-rearranged tensors.
 //
 // "RainFusion Attention" user guide, opening paragraph and "Geometry
 // handling": video tokens are arranged in (t, h, w) order with a misaligned
@@ -9,6 +9,9 @@
 // permuted in one call and an inverse restores the original order;
 // RainFusion2.0 abstract, insight 1: block means serve as the representative
 // token of each 128-token block.
+//
+// With precision "mix" the rearrange also writes an E4M3 copy of each Q and K
+// block with its fp32 scale (amax / 448) while the block is in registers.
 //
 // One CTA moves one 128-row block of one head of one tensor: 16-byte vector
 // loads and stores, whole rows per group of D/8 threads, every load of a
@@ -21,7 +24,25 @@
 
 namespace {
 
-enum Mode { kRearrange = 0, kInverse = 1, kPoolOnly = 2 };
+enum Mode { kRearrange = 0, kInverse = 1, kPoolOnly = 2, kQuantOnly = 3 };
+
+// Outputs of the fused E4M3 quantization (precision "mix"): one-byte copies of
+// Q' and K' in their layouts, and one fp32 scale per (head, global block).
+struct QuantOut {
+  uint8_t* q8;
+  uint8_t* k8;
+  float* q_scale;
+  float* k_scale;
+};
+
+// Four floats to four E4M3 codes (round to nearest even, saturating at
+// +-448), the first in the lowest byte.
+__device__ __forceinline__ uint32_t rf_e4m3x4(float a, float b, float c, float d) {
+  unsigned short lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
+  return (uint32_t)lo | ((uint32_t)hi << 16);
+}
 
 constexpr int kThreads = 256;
 
@@ -39,17 +60,18 @@ struct DecodeF16 {
   }
 };
 
-template <int D, int MODE, class Dec>
+template <int D, int MODE, class Dec, bool kQuant>
 __global__ void __launch_bounds__(kThreads)
     rf_permute_kernel(const RfGeomDev g, const uint4* __restrict__ q, const uint4* __restrict__ k,
                       const uint4* __restrict__ v, uint4* __restrict__ q_out,
                       uint4* __restrict__ k_out, uint4* __restrict__ v_out,
-                      float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
+                      float* __restrict__ pooled_q, float* __restrict__ pooled_k, const QuantOut qo) {
   constexpr int kChunks = D / 8;                  // 16-byte chunks per row
   constexpr int kRowLanes = kThreads / kChunks;   // rows handled in parallel
   constexpr int kRowsPerThread = RF_BLOCK / kRowLanes;
   __shared__ float red[kRowLanes][D + 4];
   __shared__ long long src_off[RF_BLOCK], dst_off[RF_BLOCK];  // row offsets in 16-byte units
+  __shared__ float amax_w[kThreads / 32];
 
   const int tb = blockIdx.x % g.t_qblk;           // global block
   const int th = blockIdx.x / g.t_qblk;           // tensor-major head index
@@ -65,7 +87,7 @@ __global__ void __launch_bounds__(kThreads)
   const int b = tb - s.qblk_off;
   int r0, nrows;
   rf_block_span(s, b, r0, nrows);
-  const bool pool = (MODE != kInverse) && tensor < 2 && b >= s.n_pb;
+  const bool pool = (MODE == kRearrange || MODE == kPoolOnly) && tensor < 2 && b >= s.n_pb;
   if (MODE == kPoolOnly && !pool) return;
 
   const uint4* src = tensor == 0 ? q : (tensor == 1 ? k : v);
@@ -91,14 +113,52 @@ __global__ void __launch_bounds__(kThreads)
     val[i] = make_uint4(0, 0, 0, 0);
     if (rr < nrows) val[i] = __ldg(src + src_off[rr] + ch);
   }
-  if (MODE != kPoolOnly) {
+  if (MODE == kRearrange || MODE == kInverse) {
 #pragma unroll
     for (int i = 0; i < kRowsPerThread; ++i) {
       const int rr = rl + i * kRowLanes;
       if (rr < nrows) dst[dst_off[rr] + ch] = val[i];
     }
   }
-  if constexpr (MODE == kInverse) {
+  if constexpr (kQuant && (MODE == kRearrange || MODE == kQuantOnly)) {
+    if (tensor < 2) {  // uniform over the CTA: Q and K blocks get an E4M3 copy
+      // amax over the block's valid rows (rows past nrows hold zeros).
+      float mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) mx = fmaxf(mx, fmaxf(fabsf(Dec::lo(w[c])), fabsf(Dec::hi(w[c]))));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if ((threadIdx.x & 31) == 0) amax_w[threadIdx.x >> 5] = mx;
+      __syncthreads();
+      float amax = amax_w[0];
+#pragma unroll
+      for (int i = 1; i < kThreads / 32; ++i) amax = fmaxf(amax, amax_w[i]);
+      const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
+      uint8_t* dst8 = tensor == 0 ? qo.q8 : qo.k8;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int rr = rl + i * kRowLanes;
+        if (rr < nrows) {
+          const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+          const uint32_t lo = rf_e4m3x4(__fmul_rn(Dec::lo(w[0]), inv), __fmul_rn(Dec::hi(w[0]), inv),
+                                        __fmul_rn(Dec::lo(w[1]), inv), __fmul_rn(Dec::hi(w[1]), inv));
+          const uint32_t hi = rf_e4m3x4(__fmul_rn(Dec::lo(w[2]), inv), __fmul_rn(Dec::hi(w[2]), inv),
+                                        __fmul_rn(Dec::lo(w[3]), inv), __fmul_rn(Dec::hi(w[3]), inv));
+          // dst_off is in 16-byte units of the 16-bit tensor: 8 elements each.
+          *reinterpret_cast<uint2*>(dst8 + dst_off[rr] * 8 + ch * 8) = make_uint2(lo, hi);
+        }
+      }
+      if (threadIdx.x == 0) {
+        float* sc = tensor == 0 ? qo.q_scale : qo.k_scale;
+        sc[(size_t)head * g.t_qblk + tb] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      }
+    }
+  }
+  if constexpr (MODE == kInverse || MODE == kQuantOnly) {
     return;
   } else {
     if (!pool) return;  // uniform over the CTA
@@ -139,8 +199,17 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
   const long long grid = (long long)g.t_qblk * tensor_heads;
   if (grid == 0) return RF_OK;
   if (grid > 0x7FFFFFFFll) return rf_fail(RF_ERR_INVALID_ARG, "grid too large");
-  float* pq = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + p->off_pq) : nullptr;
-  float* pk = ws ? reinterpret_cast<float*>(static_cast<char*>(ws) + p->off_pk) : nullptr;
+  char* w = static_cast<char*>(ws);
+  float* pq = ws ? reinterpret_cast<float*>(w + p->off_pq) : nullptr;
+  float* pk = ws ? reinterpret_cast<float*>(w + p->off_pk) : nullptr;
+  const bool quant = (MODE == kRearrange || MODE == kQuantOnly) && p->precision == RF_PRECISION_MIX;
+  QuantOut qout{nullptr, nullptr, nullptr, nullptr};
+  if (quant) {
+    qout.q8 = reinterpret_cast<uint8_t*>(w + p->off_q8);
+    qout.k8 = reinterpret_cast<uint8_t*>(w + p->off_k8);
+    qout.q_scale = reinterpret_cast<float*>(w + p->off_qs);
+    qout.k_scale = reinterpret_cast<float*>(w + p->off_ks);
+  }
   const uint4* a = static_cast<const uint4*>(q);
   const uint4* b = static_cast<const uint4*>(k);
   const uint4* c = static_cast<const uint4*>(v);
@@ -150,11 +219,17 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
   const bool bf = p->dtype == RF_BF16;
   dim3 grd((unsigned)grid), blk(kThreads);
   if (g.d == 128) {
-    if (bf) rf_permute_kernel<128, MODE, DecodeBf16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
-    else    rf_permute_kernel<128, MODE, DecodeF16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
+    if (quant) {
+      // precision mix is built for D = 128 only (checked when the plan is made)
+      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, true><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      else    rf_permute_kernel<128, MODE, DecodeF16, true><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    } else {
+      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      else    rf_permute_kernel<128, MODE, DecodeF16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    }
   } else {
-    if (bf) rf_permute_kernel<64, MODE, DecodeBf16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
-    else    rf_permute_kernel<64, MODE, DecodeF16><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk);
+    if (bf) rf_permute_kernel<64, MODE, DecodeBf16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    else    rf_permute_kernel<64, MODE, DecodeF16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
   }
   return rf_check_launch("rf_permute_kernel");
 }
@@ -170,6 +245,12 @@ rf_status_t rf_launch_pool(const rf_plan* p, const void* q_r, const void* k_r, v
                            cudaStream_t st) {
   return launch<kPoolOnly>(p, q_r, k_r, nullptr, nullptr, nullptr, nullptr, ws, st,
                            p->g.n1 + p->g.n2);
+}
+
+rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_r, void* ws,
+                               cudaStream_t st) {
+  return launch<kQuantOnly>(p, q_r, k_r, nullptr, nullptr, nullptr, nullptr, ws, st,
+                            p->g.n1 + p->g.n2);
 }
 
 rf_status_t rf_launch_inverse(const rf_plan* p, const void* o_r, void* o, cudaStream_t st) {

@@ -28,13 +28,14 @@ STATUS_NAMES = {0: "RF_OK", 1: "RF_ERR_INVALID_ARG", 2: "RF_ERR_UNSUPPORTED_DEVI
 LAYOUTS = {"BNSD": 0, "TND": 1}
 DTYPES = {"bf16": 0, "fp16": 1}
 ORDERS = {"tile": 0, "frame_pair": 1}   # rf_token_order_t
+PRECISIONS = {"native": 0, "mix": 1, "fp8": 2}   # rf_precision_t
 TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 POOL_MODES = {"from_ws": 0, "recompute": 1}
 
 EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange", "rf_pool_select",
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
             "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
-            "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex")
+            "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex", "rf_quantize_qk")
 
 
 class RfError(RuntimeError):
@@ -54,7 +55,14 @@ class PlanInfo(ctypes.Structure):
                 ("pooled_blocks", ctypes.c_int64), ("kept_flops_upper", ctypes.c_int64),
                 ("ws_pooled_q", ctypes.c_int64), ("ws_pooled_k", ctypes.c_int64),
                 ("n_seqs", ctypes.c_int32), ("n1", ctypes.c_int32), ("n2", ctypes.c_int32),
-                ("d", ctypes.c_int32)]
+                ("d", ctypes.c_int32), ("precision", ctypes.c_int32), ("token_order", ctypes.c_int32),
+                ("ws_q8", ctypes.c_int64), ("ws_k8", ctypes.c_int64),
+                ("ws_q_scale", ctypes.c_int64), ("ws_k_scale", ctypes.c_int64)]
+
+
+class PlanOptions(ctypes.Structure):
+    _fields_ = [("token_order", ctypes.c_int32), ("precision", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
 
 
 class SeqInfo(ctypes.Structure):
@@ -73,7 +81,8 @@ def _load() -> ctypes.CDLL:
         "rf_plan_create": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
                            i32, i32, ctypes.POINTER(vp)],
         "rf_plan_create_ex": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
-                              i32, i32, i32, ctypes.POINTER(vp)],
+                              i32, i32, ctypes.POINTER(PlanOptions), ctypes.POINTER(vp)],
+        "rf_quantize_qk": [vp, vp, vp, vp, sz, vp],
         "rf_plan_info": [vp, ctypes.POINTER(PlanInfo)],
         "rf_plan_seq_info": [vp, i32, ctypes.POINTER(SeqInfo)],
         "rf_rearrange": [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -116,16 +125,20 @@ class Plan:
 
     def __init__(self, seqs: Sequence[Tuple[int, int, int, int]], n1: int, n2: int, d: int,
                  layout: str = "BNSD", dtype: str = "bf16", sparsity: float = 0.8, batch: int = 1,
-                 block_q: int = 128, block_kv: int = 128, order: str = "tile"):
+                 block_q: int = 128, block_kv: int = 128, order: str = "tile", precision: str = "native"):
         arr = (SeqGeom * max(1, len(seqs)))(*[SeqGeom(*map(int, s)) for s in seqs])
         handle = ctypes.c_void_p()
         if order not in ORDERS:
             raise ValueError(f"order must be one of {sorted(ORDERS)}")
+        if precision not in PRECISIONS:
+            raise ValueError(f"precision must be one of {sorted(PRECISIONS)}")
+        opts = PlanOptions(ORDERS[order], PRECISIONS[precision])
         _check(_lib.rf_plan_create_ex(arr, len(seqs), batch, n1, n2, d, LAYOUTS[layout], DTYPES[dtype],
-                                      float(sparsity), block_q, block_kv, ORDERS[order],
+                                      float(sparsity), block_q, block_kv, ctypes.byref(opts),
                                       ctypes.byref(handle)),
                "rf_plan_create_ex")
         self.order = order
+        self.precision = precision
         self._h = handle
         self._lib = _lib  # kept so that destruction at interpreter exit still finds it
         self.layout, self.dtype, self.sparsity, self.batch = layout, dtype, float(sparsity), batch
@@ -263,6 +276,14 @@ def block_sparse_attn(plan: Plan, q_r, k_r, v_r, select_idx, select_num, scale: 
            "rf_block_sparse_attn")
 
 
+def quantize_qk(plan: Plan, q_r, k_r, ws, stream=None) -> None:
+    """Precision "mix": E4M3 copies of rearranged q_r / k_r and their scales into ws."""
+    _expect(q_r, plan.tensor_shape(plan.n1), plan.torch_dtype, "q_r")
+    _expect(k_r, plan.tensor_shape(plan.n2), plan.torch_dtype, "k_r")
+    _check(_lib.rf_quantize_qk(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(ws), ws.numel() * ws.element_size(),
+                               _stream(stream)), "rf_quantize_qk")
+
+
 def inverse_rearrange(plan: Plan, o_r, o, stream=None) -> None:
     """Scatter the output back to the original token order."""
     _expect(o, plan.tensor_shape(plan.n1), plan.torch_dtype, "o")
@@ -319,7 +340,7 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          seqs: Sequence[Tuple[int, int, int, int]], sparsity: float = 0.8,
                          layout: str = "BNSD", scale: Optional[float] = None,
                          plan: Optional[Plan] = None, bufs: Optional[Buffers] = None,
-                         order: str = "tile") -> torch.Tensor:
+                         order: str = "tile", precision: str = "native") -> torch.Tensor:
     """User-level call: RainFusion v2 block-sparse attention of q, k, v (original token order).
 
     q, k, v may live on the host (pinned or not) or on the GPU; the result is
@@ -327,15 +348,17 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     k/v [B, N2, L, D]; TND: q [T, N1, D], k/v [T, N2, D].  `seqs` holds one
     (prefix_len, t, h, w) per sequence (BNSD: one for the whole batch).
     `order` is the token order of the aligned video ("tile", or "frame_pair"
-    for 2x8x8 blocks over frame pairs); it is ignored when `plan` is given.
+    for 2x8x8 blocks over frame pairs) and `precision` the kernel precision
+    ("native", or "mix" for E4M3 Q K^T); both are ignored when `plan` is given.
     """
     dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[q.dtype]
     if plan is None:
         if layout == "BNSD":
             plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[3], "BNSD", dtype, sparsity, batch=q.shape[0],
-                        order=order)
+                        order=order, precision=precision)
         else:
-            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[2], "TND", dtype, sparsity, order=order)
+            plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[2], "TND", dtype, sparsity, order=order,
+                        precision=precision)
     host = not q.is_cuda
     dev = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     if bufs is None:

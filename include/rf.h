@@ -123,6 +123,13 @@ typedef struct {
   int64_t ws_pooled_k;     /* byte offset in ws of the K block means, fp32 [n2][pooled_blocks][d] */
   int32_t n_seqs;          /* sequences (BNSD: batch elements) */
   int32_t n1, n2, d;
+  int32_t precision;       /* rf_precision_t of the plan */
+  int32_t token_order;     /* rf_token_order_t of the plan */
+  /* RF_PRECISION_MIX only (else -1): byte offsets in ws of the E4M3 copies of
+   * Q' and K' (uint8, same layout and strides as q_r / k_r with one byte per
+   * element) and of their scales (fp32 [n1][t_qblk] and [n2][t_qblk], indexed
+   * by global query-block number). */
+  int64_t ws_q8, ws_k8, ws_q_scale, ws_k_scale;
 } rf_plan_info_t;
 
 /* Per-sequence geometry under suffix promotion ([UG] "Geometry handling"). */
@@ -159,15 +166,40 @@ RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int
                            rf_dtype_t dtype, double sparsity, int32_t block_q,
                            int32_t block_kv, rf_plan_t** out);
 
-/* rf_plan_create with an explicit token order (rf_plan_create uses
- * RF_ORDER_TILE).  Every other argument and error as rf_plan_create; an
- * unknown order is RF_ERR_INVALID_ARG.  Every later call on the plan
- * (rearrange, pooling, selection, inverse, rf_plan_permutation) follows the
- * plan's order. */
+/* Kernel precision ([UG] "Configuration": precision "bf16" | "fp8" | "mix").
+ *   RF_PRECISION_NATIVE  Q K^T and P V in the inputs' 16-bit type (the pages'
+ *                        "bf16"; fp16 inputs stay fp16).
+ *   RF_PRECISION_MIX     Q K^T on FP8 E4M3 copies of Q' and K' with one fp32
+ *                        scale per (head, 128-row block); P V stays 16-bit.
+ *                        rf_rearrange writes the E4M3 copies and scales into the
+ *                        workspace (amax = max |x| over the block's valid rows,
+ *                        inv = 448 / amax, codes = E4M3(x * inv) rounded to
+ *                        nearest even with saturation, scale = amax / 448; an
+ *                        all-zero block has inv = scale = 1), and
+ *                        rf_block_sparse_attn multiplies each S tile by
+ *                        scale_q * scale_k.  Head dim 128 only.
+ *   RF_PRECISION_FP8     FP8 for P V as well: not built (RF_ERR_UNSUPPORTED).
+ * The pages name the three modes and nothing more; the E4M3 format, the block
+ * granularity and the scale rule above are this library's reading. */
+typedef enum { RF_PRECISION_NATIVE = 0, RF_PRECISION_MIX = 1, RF_PRECISION_FP8 = 2 } rf_precision_t;
+/* Options of rf_plan_create_ex; zero-initialised means the defaults. */
+typedef struct {
+  int32_t token_order;  /* rf_token_order_t, default RF_ORDER_TILE */
+  int32_t precision;    /* rf_precision_t, default RF_PRECISION_NATIVE */
+  int32_t reserved[6];  /* must be zero */
+} rf_plan_options_t;
+/* rf_plan_create with options (rf_plan_create is rf_plan_create_ex with
+ * options == NULL, i.e. tile order and native precision).  Every other
+ * argument and error as rf_plan_create; an unknown option value or a non-zero
+ * reserved field is RF_ERR_INVALID_ARG; RF_PRECISION_FP8, or RF_PRECISION_MIX
+ * with d != 128, is RF_ERR_UNSUPPORTED.  Every later call on the plan
+ * (rearrange, pooling, selection, attention, inverse, rf_plan_permutation)
+ * follows the plan's options. */
 RF_API rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
                                      int32_t n1, int32_t n2, int32_t d, rf_layout_t layout,
                                      rf_dtype_t dtype, double sparsity, int32_t block_q,
-                                     int32_t block_kv, rf_token_order_t order, rf_plan_t** out);
+                                     int32_t block_kv, const rf_plan_options_t* options,
+                                     rf_plan_t** out);
 /* Sizes of a plan (host only). */
 RF_API rf_status_t rf_plan_info(const rf_plan_t* plan, rf_plan_info_t* out);
 
@@ -181,12 +213,20 @@ RF_API rf_status_t rf_plan_seq_info(const rf_plan_t* plan, int32_t seq, rf_seq_i
  *               Must not alias the inputs.
  * ws          : workspace of at least workspace_bytes; receives the fp32
  *               block means of the sparse blocks of Q and K (the fused
- *               pooling of [UG] opening paragraph / [ABS] insight 1).
+ *               pooling of [UG] opening paragraph / [ABS] insight 1) and, with
+ *               precision "mix", the E4M3 copies of Q' and K' and their scales.
  * Bit-exact copy; deterministic. */
 RF_API rf_status_t rf_rearrange(const rf_plan_t* plan, const void* q, const void* k, const void* v,
                          void* q_r, void* k_r, void* v_r, void* ws, size_t ws_bytes,
                          rf_stream_t stream);
 
+/* Precision "mix" only: the E4M3 copies of already-rearranged q_r and k_r and
+ * their scales, written into ws exactly as rf_rearrange writes them (see
+ * rf_precision_t).  rf_rearrange already does this in the same pass; this call
+ * is for callers that produce q_r / k_r themselves.  RF_ERR_INVALID_ARG for a
+ * plan with another precision. */
+RF_API rf_status_t rf_quantize_qk(const rf_plan_t* plan, const void* q_r, const void* k_r, void* ws,
+                                  size_t ws_bytes, rf_stream_t stream);
 /* Steps 2-3 ([UG] opening paragraphs and "Configuration"; [API] selectIdx and
  * selectNum constraints).
  * q_r, k_r    : rearranged Q and K (read only when pool_mode == RF_POOL_RECOMPUTE;
@@ -236,6 +276,9 @@ RF_API rf_status_t rf_pool_select_noalloc(const rf_plan_t* plan, const void* q_r
  * scale       : > 0 and finite (typically 1/sqrt(D)).
  * inner_precise : 0 = fp32 softmax ([API]: 1 = fp16 softmax is not allowed with
  *               bf16 and is not built here: RF_ERR_UNSUPPORTED).
+ * Precision "mix": Q K^T reads the E4M3 copies of Q' and K' and their scales in
+ *               ws (written by rf_rearrange or rf_quantize_qk on this ws), not
+ *               q_r / k_r; P V reads v_r as usual.
  * Deterministic: no split-K, no atomics. */
 RF_API rf_status_t rf_block_sparse_attn(const rf_plan_t* plan, const void* q_r, const void* k_r,
                                  const void* v_r, const int32_t* select_idx,

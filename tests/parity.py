@@ -40,9 +40,10 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
 
 
 def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "from_ws",
-            order: str = "tile") -> Dict[str, object]:
+            order: str = "tile", precision: str = "native") -> Dict[str, object]:
     """Whole path through the C ABI, one call per step; returns host copies of every result."""
-    plan = rf.Plan(seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=order)
+    plan = rf.Plan(seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=order,
+                   precision=precision)
     q, k, v = (to_device(b, w.dtype) for b in bits)
     b = rf.Buffers(plan)
     scale = 1.0 / math.sqrt(w.d)
@@ -58,9 +59,45 @@ def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "fro
     oq, ok_ = int(plan.info.ws_pooled_q), int(plan.info.ws_pooled_k)
     pq = ws8[oq:oq + w.n1 * pooled * w.d * 4].view(torch.float32).reshape(w.n1, pooled, w.d).cpu().numpy()
     pk = ws8[ok_:ok_ + w.n2 * pooled * w.d * 4].view(torch.float32).reshape(w.n2, pooled, w.d).cpu().numpy()
-    return dict(plan=plan, q_r=to_bits(b.q_r), k_r=to_bits(b.k_r), v_r=to_bits(b.v_r), o_r=to_bits(b.o_r),
-                o=to_bits(b.o), idx=b.select_idx.cpu().numpy(), num=b.select_num.cpu().numpy(),
-                pooled_q=pq, pooled_k=pk, scale=scale)
+    out = dict(plan=plan, q_r=to_bits(b.q_r), k_r=to_bits(b.k_r), v_r=to_bits(b.v_r), o_r=to_bits(b.o_r),
+               o=to_bits(b.o), idx=b.select_idx.cpu().numpy(), num=b.select_num.cpu().numpy(),
+               pooled_q=pq, pooled_k=pk, scale=scale)
+    if precision == "mix":
+        out.update(mix_buffers(plan, b.ws))
+    return out
+
+
+def mix_buffers(plan: rf.Plan, ws: torch.Tensor) -> Dict[str, np.ndarray]:
+    """Host copies of the E4M3 copies of Q' / K' and their scales in a mix-precision workspace."""
+    info = plan.info
+    ws8 = ws.view(torch.uint8)
+    rows, t, d = int(info.rows_total), int(info.t_qblk), plan.d
+
+    def region(off, n):
+        return ws8[int(off):int(off) + n].cpu().numpy()
+    q8 = region(info.ws_q8, rows * plan.n1 * d).reshape(plan.tensor_shape(plan.n1))
+    k8 = region(info.ws_k8, rows * plan.n2 * d).reshape(plan.tensor_shape(plan.n2))
+    qs = region(info.ws_q_scale, plan.n1 * t * 4).view(np.float32).reshape(plan.n1, t)
+    ks = region(info.ws_k_scale, plan.n2 * t * 4).view(np.float32).reshape(plan.n2, t)
+    return dict(q8=q8, k8=k8, q_scale=qs, k_scale=ks)
+
+
+def check_mix_quantization(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu) -> None:
+    """E4M3 codes and scales of Q' and K' bit-exact against the oracle's quantization."""
+    for name, x, heads in (("q", rbits[0], w.n1), ("k", rbits[1], w.n2)):
+        xf = synth.bits_to_float64(x, w.dtype).astype(np.float32)   # exact: 16-bit values
+        codes, scales = orc.quantize_e4m3(p, xf, heads)
+        assert np.array_equal(gpu[name + "_scale"], scales), f"{name} scales differ"
+        got = gpu[name + "8"]
+        diff = got != codes
+        assert not diff.any(), f"{name} E4M3 codes differ at {int(diff.sum())} elements"
+
+
+def mix_reference_inputs(p: orc.Problem, w: synth.Workload, gpu, rbits: Sequence[np.ndarray]):
+    """float64 Q', K' as the mix precision sees them (E4M3 code x scale) and exact V'."""
+    qf = orc.dequantize_e4m3(p, gpu["q8"], gpu["q_scale"], w.n1)
+    kf = orc.dequantize_e4m3(p, gpu["k8"], gpu["k_scale"], w.n2)
+    return qf, kf, synth.bits_to_float64(rbits[2], w.dtype)
 
 
 def oracle_rearranged_bits(p: orc.Problem, bits: np.ndarray) -> np.ndarray:
@@ -129,9 +166,12 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
 
 
 def check_attention(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu,
-                    items: Sequence[Tuple[int, int]] | None = None) -> Dict[str, float]:
-    """GPU o_r against the oracle run on the GPU's selectIdx, for (q-block, head) items."""
-    qf, kf, vf = (synth.bits_to_float64(x, w.dtype) for x in rbits)
+                    items: Sequence[Tuple[int, int]] | None = None, values=None,
+                    check: bool = True) -> Dict[str, float]:
+    """GPU o_r against the oracle run on the GPU's selectIdx, for (q-block, head) items.
+    `values` replaces the float64 (Q', K', V') decoded from rbits (mix precision);
+    with check=False the errors are returned without asserting the bars."""
+    qf, kf, vf = values if values is not None else (synth.bits_to_float64(x, w.dtype) for x in rbits)
     ref = orc.attention(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items)
     o_r = synth.bits_to_float64(gpu["o_r"], w.dtype)
     table = orc.qblock_table(p)
@@ -146,8 +186,9 @@ def check_attention(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarra
         num += float(np.sum(d * d))
         den += float(np.sum(rows * rows))
     rel = math.sqrt(num / max(den, 1e-300))
-    assert mx <= MAX_ABS, f"max abs err {mx}"
-    assert rel <= REL_L2, f"rel L2 err {rel}"
+    if check:
+        assert mx <= MAX_ABS, f"max abs err {mx}"
+        assert rel <= REL_L2, f"rel L2 err {rel}"
     return dict(max_abs=mx, rel_l2=rel, items=len(ref))
 
 

@@ -148,10 +148,55 @@ def test_frame_pair_tnd_sequences_each_follow_the_order():
         assert np.array_equal(plan.permutation(i), orc.permutation(orc.geometry(*s, 0.8, "frame_pair")))
 
 
-def test_unknown_token_order_is_rejected():
+def _create_ex(opts, d=64):
     arr = (rf.SeqGeom * 1)(rf.SeqGeom(128, 9, 16, 32))
     h = ctypes.c_void_p()
-    st = rf.lib().rf_plan_create_ex(arr, 1, 1, 2, 2, 64, 0, 0, ctypes.c_double(0.8), 128, 128, 7, ctypes.byref(h))
-    assert st == 1 and not h.value
+    st = rf.lib().rf_plan_create_ex(arr, 1, 1, 2, 2, d, 0, 0, ctypes.c_double(0.8), 128, 128,
+                                    ctypes.byref(opts) if opts is not None else None, ctypes.byref(h))
+    if h.value:
+        rf.lib().rf_plan_destroy(h)
+    return st, bool(h.value)
+
+
+def test_plan_options_are_validated():
+    assert _create_ex(None) == (0, True)                          # NULL options: the defaults
+    assert _create_ex(rf.PlanOptions(0, 0)) == (0, True)
+    assert _create_ex(rf.PlanOptions(7, 0)) == (1, False)         # unknown token order
+    assert _create_ex(rf.PlanOptions(0, 9)) == (1, False)         # unknown precision
+    bad = rf.PlanOptions(0, 0)
+    bad.reserved[3] = 1
+    assert _create_ex(bad) == (1, False)                          # reserved fields must be zero
+    assert _create_ex(rf.PlanOptions(0, 2), d=128) == (6, False)  # fp8 P V: not built
+    assert _create_ex(rf.PlanOptions(0, 1), d=64) == (6, False)   # mix: head dim 128 only
+    assert _create_ex(rf.PlanOptions(1, 1), d=128) == (0, True)
     with pytest.raises(ValueError):
         rf.Plan([(128, 9, 16, 32)], 2, 2, 64, order="zigzag")
+    with pytest.raises(ValueError):
+        rf.Plan([(128, 9, 16, 32)], 2, 2, 128, precision="int4")
+
+
+@pytest.mark.parametrize("layout,seqs,n1,n2", [("BNSD", [(512, 21, 30, 52)], 40, 40),
+                                               ("TND", [(256, 13, 32, 48), (384, 21, 24, 40)], 32, 8)])
+def test_mix_precision_workspace_layout(layout, seqs, n1, n2):
+    """The E4M3 copies and scales sit after the native workspace, 256-byte aligned,
+    sized one byte per element of Q' / K' and one float per (head, query block)."""
+    nat = rf.Plan(seqs, n1, n2, 128, layout, "bf16", 0.8)
+    mix = rf.Plan(seqs, n1, n2, 128, layout, "bf16", 0.8, precision="mix")
+    a, b = nat.info, mix.info
+    assert (a.precision, b.precision) == (0, 1)
+    assert a.ws_q8 == a.ws_k8 == a.ws_q_scale == a.ws_k_scale == -1
+    rows, t = int(b.rows_total), int(b.t_qblk)
+    assert b.ws_q8 >= a.workspace_bytes and b.ws_q8 % 256 == 0
+    assert b.ws_k8 >= b.ws_q8 + rows * n1 * 128 and b.ws_k8 % 256 == 0
+    assert b.ws_q_scale >= b.ws_k8 + rows * n2 * 128
+    assert b.ws_k_scale >= b.ws_q_scale + n1 * t * 4
+    assert b.workspace_bytes >= b.ws_k_scale + n2 * t * 4
+    for f in ("rows_total", "t_qblk", "max_kv_blocks", "pooled_blocks", "ws_pooled_q", "ws_pooled_k"):
+        assert getattr(a, f) == getattr(b, f), f
+
+
+def test_quantize_needs_a_mix_plan():
+    plan = rf.Plan([(128, 9, 16, 32)], 2, 2, 128)
+    fake = ctypes.c_void_p(1 << 20)
+    st = rf.lib().rf_quantize_qk(plan.handle, fake, fake, fake, plan.workspace_bytes, None)
+    assert st == 1

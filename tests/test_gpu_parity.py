@@ -228,6 +228,61 @@ def test_frame_pair_full_size_parity(name, s):
     parity.check_attention(p, w, rbits, gpu, items)
 
 
+# ------------------------------------------------------------------------------------------
+# Precision "mix" (E4M3 Q K^T, 16-bit P V): the E4M3 copies and scales bit-exact against the
+# oracle's quantization; the output against the oracle run on the dequantized Q', K' (the
+# inputs this precision defines) within the same bars as the native path.
+# ------------------------------------------------------------------------------------------
+
+MIX_SMALL = ["ragged_d128", "tnd_gqa_small", "dense", "s_one"]
+
+
+@pytest.mark.parametrize("name", MIX_SMALL)
+def test_mix_small_parity(name):
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision="mix")
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    parity.check_mix_quantization(p, w, rbits, gpu)
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)             # pooling still reads the 16-bit values
+    parity.check_selection(p, qbars, kbars, gpu)
+    parity.check_attention(p, w, rbits, gpu, values=parity.mix_reference_inputs(p, w, gpu, rbits))
+
+
+@pytest.mark.parametrize("name,s", [("wan", None), ("tnd_gqa", None)])
+def test_mix_full_size_parity(name, s):
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision="mix")
+    rbits = [orc.rearrange(p, x) for x in bits]
+    parity.check_mix_quantization(p, w, rbits, gpu)
+    items = parity.sample_items(p, np.random.default_rng(9), per_kind=3)
+    parity.check_attention(p, w, rbits, gpu, items, values=parity.mix_reference_inputs(p, w, gpu, rbits))
+    # the quantization error itself, against the unquantized oracle: reported, and bounded
+    # loosely (E4M3 keeps 3 mantissa bits)
+    err = parity.check_attention(p, w, rbits, gpu, items, check=False)
+    assert err["rel_l2"] <= 0.1, err
+
+
+def test_mix_quantize_entry_point_equals_fused_quantization():
+    w = SMALL["tnd_gqa_small"]
+    bits = synth.generate_qkv(w)
+    fused = parity.run_gpu(w, bits, precision="mix")
+    plan = fused["plan"]
+    b = rf.Buffers(plan)
+    q_r = parity.to_device(fused["q_r"], w.dtype)
+    k_r = parity.to_device(fused["k_r"], w.dtype)
+    rf.quantize_qk(plan, q_r, k_r, b.ws)
+    torch.cuda.synchronize()
+    alone = parity.mix_buffers(plan, b.ws)
+    for key in ("q8", "k8", "q_scale", "k_scale"):
+        assert np.array_equal(alone[key], fused[key]), key
+
+
 def test_exp2_polynomial_against_mufu_and_exact():
     """The FMA-pipe exponential the softmax uses for part of its columns:
     relative error <= 2e-4 against the exact 2^x and against ex2.approx,
