@@ -77,7 +77,7 @@ def kernel_sha(name):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def profiled_traffic(workload, sparsity):
+def profiled_traffic(workload, sparsity, tag=""):
     """DRAM bytes per attention launch from the committed ncu summary, if it still
     describes the current kernel source (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.md")
@@ -88,7 +88,7 @@ def profiled_traffic(workload, sparsity):
         for line in f:
             parts = line.strip().strip("|").split("|")
             parts = [p.strip() for p in parts]
-            if len(parts) >= 5 and parts[0] == "rf_attn_kernel" and parts[1] == f"{workload}@{sparsity:g}" \
+            if len(parts) >= 5 and parts[0] == "rf_attn_kernel" and parts[1] == f"{workload}@{sparsity:g}{tag}" \
                     and parts[2] == sha:
                 try:
                     return float(parts[3])
@@ -393,7 +393,8 @@ def main():
         front_ms = float(np.mean(per[:, 0] + per[:, 1]))
         inv_ms = float(np.mean(per[:, 3]))
         value = flops_all / (ms_step * 1e-3) / 1e12
-        traffic = profiled_traffic(w.name.split("@")[0], sparsity)
+        traffic = (profiled_traffic(w.name.split("@")[0], sparsity, "/mix" if args.precision == "mix" else "")
+                   if args.order == "tile" and not args.heads else None)
         line = {
             "metric": METRIC,
             "value": round(value, 3),
@@ -424,7 +425,7 @@ def main():
             "attn_tflops": round(achieved, 2),
             "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4),
-                         "traffic": traffic if args.precision == "native" and args.order == "tile" else None,
+                         "traffic": traffic,
                          "peak_source": peak_note},
             "hbm_roofline": {"kernels": "rf_rearrange + rf_pool_select", "achieved": round(front_bytes / (front_ms * 1e-3) / 1e9, 1),
                              "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -2,11 +2,13 @@
 
 The compute path lives in the CUDA library `librf.so` (built from `csrc/`),
 reached through `block_sparse_video_rearrange_b200.rf` (ctypes binding).
-`synth` holds the seeded synthetic input generator.
+`ulysses` shards one layer over a process group by heads (sequence <-> head
+all-to-all around the path).  `synth` holds the seeded synthetic input
+generator.
 """
 import importlib
 
-__all__ = ["rf", "synth"]
+__all__ = ["rf", "synth", "ulysses"]
 
 
 def __getattr__(name):

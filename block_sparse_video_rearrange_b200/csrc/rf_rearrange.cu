@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(kThreads)
   constexpr int kRowsPerThread = RF_BLOCK / kRowLanes;
   __shared__ float red[kRowLanes][D + 4];
   __shared__ long long src_off[RF_BLOCK], dst_off[RF_BLOCK];  // row offsets in 16-byte units
-  __shared__ float amax_w[kThreads / 32];
+  __shared__ uint32_t amax_w[kThreads / 32];
 
   const int tb = blockIdx.x % g.t_qblk;           // global block
   const int th = blockIdx.x / g.t_qblk;           // tensor-major head index
@@ -122,32 +122,39 @@ __global__ void __launch_bounds__(kThreads)
   }
   if constexpr (kQuant && (MODE == kRearrange || MODE == kQuantOnly)) {
     if (tensor < 2) {  // uniform over the CTA: Q and K blocks get an E4M3 copy
-      // amax over the block's valid rows (rows past nrows hold zeros).
-      float mx = 0.f;
+      // amax over the block's valid rows (rows past nrows hold zeros).  For
+      // finite bf16 and fp16 alike |x| orders as the 15-bit magnitude field,
+      // so a packed unsigned 16-bit max of the masked words finds the largest
+      // magnitude two elements at a time.
+      uint32_t mb = 0u;
 #pragma unroll
       for (int i = 0; i < kRowsPerThread; ++i) {
-        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
-#pragma unroll
-        for (int c = 0; c < 4; ++c) mx = fmaxf(mx, fmaxf(fabsf(Dec::lo(w[c])), fabsf(Dec::hi(w[c]))));
+        mb = __vmaxu2(mb, val[i].x & 0x7FFF7FFFu);
+        mb = __vmaxu2(mb, val[i].y & 0x7FFF7FFFu);
+        mb = __vmaxu2(mb, val[i].z & 0x7FFF7FFFu);
+        mb = __vmaxu2(mb, val[i].w & 0x7FFF7FFFu);
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if ((threadIdx.x & 31) == 0) amax_w[threadIdx.x >> 5] = mx;
+      mb = __reduce_max_sync(0xffffffffu, max(mb & 0xFFFFu, mb >> 16));
+      if ((threadIdx.x & 31) == 0) amax_w[threadIdx.x >> 5] = mb;
       __syncthreads();
-      float amax = amax_w[0];
 #pragma unroll
-      for (int i = 1; i < kThreads / 32; ++i) amax = fmaxf(amax, amax_w[i]);
+      for (int i = 0; i < kThreads / 32; ++i) mb = max(mb, amax_w[i]);
+      const float amax = Dec::lo(mb);
       const float inv = amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f;
+      const uint64_t inv2 = rf_f2(__float_as_uint(inv), __float_as_uint(inv));
       uint8_t* dst8 = tensor == 0 ? qo.q8 : qo.k8;
 #pragma unroll
       for (int i = 0; i < kRowsPerThread; ++i) {
         const int rr = rl + i * kRowLanes;
         if (rr < nrows) {
           const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
-          const uint32_t lo = rf_e4m3x4(__fmul_rn(Dec::lo(w[0]), inv), __fmul_rn(Dec::hi(w[0]), inv),
-                                        __fmul_rn(Dec::lo(w[1]), inv), __fmul_rn(Dec::hi(w[1]), inv));
-          const uint32_t hi = rf_e4m3x4(__fmul_rn(Dec::lo(w[2]), inv), __fmul_rn(Dec::hi(w[2]), inv),
-                                        __fmul_rn(Dec::lo(w[3]), inv), __fmul_rn(Dec::hi(w[3]), inv));
+          float y[8];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)   // x * inv, one IEEE fp32 multiply per element, two per instruction
+            rf_f2_split(rf_mul2(rf_f2(__float_as_uint(Dec::lo(w[c])), __float_as_uint(Dec::hi(w[c]))), inv2),
+                        y[2 * c], y[2 * c + 1]);
+          const uint32_t lo = rf_e4m3x4(y[0], y[1], y[2], y[3]);
+          const uint32_t hi = rf_e4m3x4(y[4], y[5], y[6], y[7]);
           // dst_off is in 16-byte units of the 16-bit tensor: 8 elements each.
           *reinterpret_cast<uint2*>(dst8 + dst_off[rr] * 8 + ch * 8) = make_uint2(lo, hi);
         }
