@@ -35,9 +35,12 @@
 // half of the blocks; the epilogue merges the two halves (a fixed split, so
 // the result is deterministic).  MMA issue order: S_0, S_1, then for every j:
 // O_{j%2} += P_j V_j followed by S_{j+2}, so one group's softmax overlaps the
-// other group's matrix products.
+// other group's matrix products.  P_j V_j goes in two halves of the key rows:
+// the softmax releases the first 64 columns of P_j before computing the rest.
 // The softmax works in the exp2 domain; O_w is rescaled only when a row max
-// grows by more than 2^8 (a warp-uniform decision).  Column pairs selected by
+// grows by more than 2^8 (a warp-uniform decision), right after the row max,
+// before any of P_j is released (O_w is at rest then: S_j completes after the
+// group's previous P V).  Column pairs selected by
 // RF_EMU_PAIR_MASK take their exponentials from a polynomial on the FMA pipe
 // (rf_exp2_poly) instead of the MUFU unit.  Measured on the Wan2.2-shaped
 // layer, offloading 12.5% or 25% of them was slower than none (the extra
@@ -85,7 +88,7 @@ struct __align__(1024) AttnSmem {
   uint64_t bar_q;
   uint64_t bar_k_full[kStagesK], bar_k_empty[kStagesK];
   uint64_t bar_v_full[kStagesV], bar_v_empty[kStagesV];
-  uint64_t bar_s_full[2], bar_p_full[2], bar_o_done[2];
+  uint64_t bar_s_full[2], bar_p_half[2], bar_p_full[2];
   uint64_t bar_final;
   uint64_t bar_drain;
   uint32_t tmem_base;
@@ -110,9 +113,12 @@ struct AttnArgs {
 
 // Warp-wide bounded wait: every lane polls the barrier itself (a lane that
 // only waits on a warp shuffle for a polling lane 0 wakes far later), then the
-// warp agrees on the outcome.
+// warp agrees on the outcome.  kPoll = true drops the suspend hint: the MMA
+// warp's hand-offs (P ready, V and K tiles landed) sit on the critical path,
+// and polling them measured about 2% faster overall than sleeping on them.
+template <bool kPoll = false>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+  const bool ok = mbar_wait<kPoll>(bar, parity, abort);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -143,32 +149,35 @@ __device__ __forceinline__ float row_max(const uint32_t* sr, int vr) {
   return rf_max3(rf_max3(m[0], m[1], m[2]), rf_max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// p = 2^(s * sl2 - m) for 128 scores (the first vr valid), packed pairwise to
-// 16-bit into pk[64]; returns the fp32 sum.  The scale-and-subtract and the
-// running sums run as paired fp32 instructions (two columns per instruction).
-// Pairs selected by kEmuPairMask use the FMA-pipe polynomial, the others
-// ex2.approx.
+// p = 2^(s * sl2 - m) for the 64 scores c0 .. c0 + 63 of a row (the first vr
+// of the row valid), packed pairwise to 16-bit into pk[32]; the fp32 sums go
+// to the four paired accumulators acc (a column pair's accumulator does not
+// depend on c0, so two halves sum in the same order as one pass would).  The
+// scale-and-subtract and the sums run as paired fp32 instructions (two columns
+// per instruction).  Pairs selected by kEmuPairMask use the FMA-pipe
+// polynomial, the others ex2.approx.
 template <bool kBf16, bool kFull>
-__device__ __forceinline__ float row_exp(const uint32_t* sr, int vr, float sl2, float neg_m, uint32_t* pk) {
+__device__ __forceinline__ void half_row_exp(const uint32_t* sr, int c0, int vr, float sl2, float neg_m,
+                                             uint32_t* pk, uint64_t* acc) {
   const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
   const uint64_t negm2 = rf_f2(__float_as_uint(neg_m), __float_as_uint(neg_m));
-  uint64_t acc[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = 0ull;
-#pragma unroll
-  for (int c = 0; c < 128; c += 2) {
+  for (int c = 0; c < 64; c += 2) {
     const bool emu = (kEmuPairMask >> ((c >> 1) & 15)) & 1u;
     float x0, x1;
-    rf_f2_split(rf_fma2(rf_f2(sr[c], sr[c + 1]), sl2x2, negm2), x0, x1);
+    rf_f2_split(rf_fma2(rf_f2(sr[c0 + c], sr[c0 + c + 1]), sl2x2, negm2), x0, x1);
     float p0 = emu ? rf_exp2_poly(x0) : rf_ex2(x0);
     float p1 = emu ? rf_exp2_poly(x1) : rf_ex2(x1);
     if (!kFull) {
-      p0 = c < vr ? p0 : 0.f;
-      p1 = c + 1 < vr ? p1 : 0.f;
+      p0 = c0 + c < vr ? p0 : 0.f;
+      p1 = c0 + c + 1 < vr ? p1 : 0.f;
     }
     acc[(c >> 1) & 3] = rf_add2(acc[(c >> 1) & 3], rf_f2(__float_as_uint(p0), __float_as_uint(p1)));
     pk[c >> 1] = rf_pack2<kBf16>(p0, p1);
   }
+}
+
+__device__ __forceinline__ float acc_sum(const uint64_t* acc) {
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -219,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(rf_smem_u32(&sm.bar_s_full[i]), 1);
+      mbar_init(rf_smem_u32(&sm.bar_p_half[i]), 128);
       mbar_init(rf_smem_u32(&sm.bar_p_full[i]), 128);
-      mbar_init(rf_smem_u32(&sm.bar_o_done[i]), 1);
     }
     mbar_init(rf_smem_u32(&sm.bar_final), 1);
     mbar_init(rf_smem_u32(&sm.bar_drain), 1);
@@ -344,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // 32-byte slice of the reduction (16 bf16/fp16 or 32 E4M3 elements).
     auto issue_qk = [&](int j) -> bool {
       const int st = j % kStagesK;
-      if (!warp_wait(rf_smem_u32(&sm.bar_k_full[st]), (j / kStagesK) & 1, abort)) return false;
+      if (!warp_wait<true>(rf_smem_u32(&sm.bar_k_full[st]), (j / kStagesK) & 1, abort)) return false;
       tc_fence_after();
       if (elect_one()) {
         const uint64_t dk = dk0 + (uint64_t)(st * (kQkTileBytes >> 4));
@@ -362,21 +371,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       return true;
     };
-    bool ok = warp_wait(rf_smem_u32(&sm.bar_q), 0, abort);
+    bool ok = warp_wait<true>(rf_smem_u32(&sm.bar_q), 0, abort);
     if (ok) ok = issue_qk(0);
     if (ok && nv > 1) ok = issue_qk(1);
     for (int j = 0; ok && j < nv; ++j) {
       const int w = j & 1, i = j >> 1, st = j % kStagesV;
-      if (!warp_wait(rf_smem_u32(&sm.bar_p_full[w]), i & 1, abort)) { ok = false; break; }
-      if (!warp_wait(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
+      const uint64_t dv = dv0 + (uint64_t)(st * (kVTileBytes >> 4));
+      // O_w += P_j V_j in two halves of the key rows: the first as soon as the
+      // softmax has stored the first 64 columns of P_j, the second when all of
+      // P_j is in.
+      if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_half[w]), i & 1, abort)) { ok = false; break; }
+      if (!warp_wait<true>(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
       tc_fence_after();
       if (elect_one()) {
-        const uint64_t dv = dv0 + (uint64_t)(st * (kVTileBytes >> 4));
 #pragma unroll
-        for (int kk = 0; kk < RF_BLOCK / 16; ++kk)
+        for (int kk = 0; kk < RF_BLOCK / 32; ++kk)
           mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)),
                  idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(rf_smem_u32(&sm.bar_o_done[w]));
+      }
+      __syncwarp();
+      if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_full[w]), i & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = RF_BLOCK / 32; kk < RF_BLOCK / 16; ++kk)
+          mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)),
+                 idesc_pv, 1u);
         tc_commit(rf_smem_u32(&sm.bar_v_empty[st]));
       }
       __syncwarp();
@@ -421,33 +441,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
       const float mx_t = (vr == RF_BLOCK ? row_max<true>(sr, vr) : row_max<false>(sr, vr)) * sl2;
       const bool rescale = __any_sync(0xffffffffu, mx_t > m_run + kRescaleThreshold);
-      float alpha = 1.f;
       if (rescale) {
         const float m_new = fmaxf(m_run, mx_t);
-        alpha = rf_ex2(m_run - m_new);
+        const float alpha = rf_ex2(m_run - m_new);
         l_run *= alpha;
         m_run = m_new;
-      }
-      uint32_t pk[64];
-      l_run += vr == RF_BLOCK ? row_exp<kBf16, true>(sr, vr, sl2, -m_run, pk)
-                              : row_exp<kBf16, false>(sr, vr, sl2, -m_run, pk);
-      tmem_st32(scol, pk);
-      tmem_st32(scol + 32, pk + 32);
-      if (rescale && i > 0) {
-        // O_w holds this group's earlier P V products: wait for the last one,
-        // then rescale it before P_j is released to the MMA warp.
-        if (!warp_wait(rf_smem_u32(&sm.bar_o_done[wg]), (i - 1) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
+        if (i > 0) {
+          // O_w holds this group's earlier P V products and is at rest: S_j
+          // was issued after the last of them, and S_j is complete.  Rescale
+          // it before any of P_j is released to the MMA warp.
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + o_col + c0, o);
-          tmem_wait_ld();
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + o_col + c0, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(lane_base + o_col + c0, o);
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(lane_base + o_col + c0, o);
+          }
         }
       }
+      // P_j over the first 64 columns of S_j (already in registers), one half
+      // at a time: the first half is released to the MMA warp while the second
+      // is being computed.
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[32];
+      if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 0, vr, sl2, -m_run, pk, acc);
+      else                half_row_exp<kBf16, false>(sr, 0, vr, sl2, -m_run, pk, acc);
+      tmem_st32(scol, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(rf_smem_u32(&sm.bar_p_half[wg]));
+      if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 64, vr, sl2, -m_run, pk, acc);
+      else                half_row_exp<kBf16, false>(sr, 64, vr, sl2, -m_run, pk, acc);
+      l_run += acc_sum(acc);
+      tmem_st32(scol + 32, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(rf_smem_u32(&sm.bar_p_full[wg]));

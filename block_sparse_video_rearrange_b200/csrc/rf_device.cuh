@@ -152,16 +152,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One test of phase `parity` without a suspend hint: the thread polls.
+__device__ __forceinline__ bool mbar_try_wait_poll(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` of barrier `bar` to complete, for at most
 // RF_WAIT_LIMIT_NS; gives up early once *abort is set.  Returns false when it
-// gave up (the caller records it and unwinds).
+// gave up (the caller records it and unwinds).  kPoll: poll without the
+// suspend hint (for a warp whose wake-up latency is on the critical path).
 #define RF_WAIT_LIMIT_NS 1000000000ull
+template <bool kPoll = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() { return kPoll ? mbar_try_wait_poll(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
   const uint64_t t0 = rf_globaltimer();
 #pragma unroll 1
   for (;;) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (test()) return true;
     if (*abort) return false;
     if (rf_globaltimer() - t0 > RF_WAIT_LIMIT_NS) return false;
   }

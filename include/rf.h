@@ -256,8 +256,8 @@ RF_API rf_status_t rf_pool_select(const rf_plan_t* plan, const void* q_r, const 
  * the first call on each device (with that device current), which loads it
  * onto that GPU, where it stays until the process exits; make that first call
  * before any stream capture.  Problems whose selection scratch
- * (rf_plan_info().workspace_bytes) exceeds 32 MiB are rejected with
- * RF_ERR_INVALID_ARG.  Every call on a device shares the array: calls that
+ * (rf_plan_info().workspace_bytes; for a precision "mix" plan the part before
+ * ws_q8) exceeds 32 MiB are rejected with RF_ERR_INVALID_ARG.  Every call on a device shares the array: calls that
  * overlap on the GPU (other streams, other threads) race and must be
  * serialised by the caller.  Calls no cudaMalloc, cudaFree or other
  * allocating routine. */

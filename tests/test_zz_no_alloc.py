@@ -64,3 +64,21 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     st = rf.lib().rf_pool_select_noalloc(plan.handle, p, p, p, p, None)
     assert st == 1                            # RF_ERR_INVALID_ARG
     assert b"scratch" in rf.lib().rf_last_error()
+
+
+def test_noalloc_accepts_a_mix_plan_whose_selection_part_fits():
+    """A mix-precision plan's workspace also holds the E4M3 copies of Q' and K';
+    selection needs only the part before them, which is what must fit."""
+    w = CASES["wan"]
+    bits = synth.generate_qkv(w)
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, precision="mix")
+    assert plan.workspace_bytes > 32 << 20 and plan.info.ws_q8 <= 32 << 20
+    q, k, v = (parity.to_device(x, w.dtype) for x in bits)
+    b = rf.Buffers(plan)
+    rf.rearrange(plan, q, k, v, b.q_r, b.k_r, b.v_r, b.ws)
+    rf.pool_select(plan, b.q_r, b.k_r, b.select_idx, b.select_num, b.ws, pool_mode="recompute")
+    idx = torch.full_like(b.select_idx, 7)
+    num = torch.full_like(b.select_num, 7)
+    rf.pool_select_noalloc(plan, b.q_r, b.k_r, idx, num)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, b.select_idx) and torch.equal(num, b.select_num)
