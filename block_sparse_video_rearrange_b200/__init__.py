@@ -3,12 +3,13 @@
 The compute path lives in the CUDA library `librf.so` (built from `csrc/`),
 reached through `block_sparse_video_rearrange_b200.rf` (ctypes binding).
 `ulysses` shards one layer over a process group by heads (sequence <-> head
-all-to-all around the path).  `synth` holds the seeded synthetic input
+all-to-all around the path); `pipeline` runs host tensors in head chunks
+whose copies overlap the compute.  `synth` holds the seeded synthetic input
 generator.
 """
 import importlib
 
-__all__ = ["rf", "synth", "ulysses"]
+__all__ = ["rf", "synth", "ulysses", "pipeline"]
 
 
 def __getattr__(name):

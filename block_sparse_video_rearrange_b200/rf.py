@@ -336,11 +336,15 @@ def forward(plan: Plan, q, k, v, bufs: Buffers, scale: Optional[float] = None, s
     return b.o
 
 
+_PIPELINES = {}
+
+
 def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          seqs: Sequence[Tuple[int, int, int, int]], sparsity: float = 0.8,
                          layout: str = "BNSD", scale: Optional[float] = None,
                          plan: Optional[Plan] = None, bufs: Optional[Buffers] = None,
-                         order: str = "tile", precision: str = "native") -> torch.Tensor:
+                         order: str = "tile", precision: str = "native",
+                         chunks: Optional[int] = None) -> torch.Tensor:
     """User-level call: RainFusion v2 block-sparse attention of q, k, v (original token order).
 
     q, k, v may live on the host (pinned or not) or on the GPU; the result is
@@ -350,8 +354,30 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     `order` is the token order of the aligned video ("tile", or "frame_pair"
     for 2x8x8 blocks over frame pairs) and `precision` the kernel precision
     ("native", or "mix" for E4M3 Q K^T); both are ignored when `plan` is given.
+
+    Host inputs run through `pipeline.HostPipeline` (made once per problem
+    shape and kept): head chunks whose copies to and from the GPU overlap
+    the compute of other chunks; `chunks` overrides its default.  The result
+    is the same, bit for bit, as one pass over all heads.
     """
     dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[q.dtype]
+    if not q.is_cuda and plan is None and bufs is None:
+        from .pipeline import HostPipeline
+        if layout == "BNSD":
+            n1, n2, d, batch = q.shape[1], k.shape[1], q.shape[3], q.shape[0]
+        else:
+            n1, n2, d, batch = q.shape[1], k.shape[1], q.shape[2], 1
+        dev = torch.device("cuda", torch.cuda.current_device())
+        key = (tuple(map(tuple, seqs)), n1, n2, d, layout, dtype, float(sparsity), batch, order, precision,
+               chunks, dev.index)
+        pipe = _PIPELINES.get(key)
+        if pipe is None:
+            pipe = HostPipeline(seqs, n1, n2, d, layout, dtype, sparsity, batch, chunks, order, precision, dev)
+            _PIPELINES[key] = pipe
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        pipe(q, k, v, out, scale)
+        torch.cuda.current_stream(dev).synchronize()
+        return out
     if plan is None:
         if layout == "BNSD":
             plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[3], "BNSD", dtype, sparsity, batch=q.shape[0],

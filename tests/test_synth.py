@@ -39,3 +39,11 @@ def test_video_rows_share_their_cell_offset():
     same = np.corrcoef(q[0], q[1])[0, 1]          # (0,0) and (0,1): same cell
     other = np.corrcoef(q[0], q[8])[0, 1]         # (0,0) and (0,8): neighbouring cell
     assert same > 0.6 and abs(other) < 0.3
+
+
+def test_pipeline_default_chunks_divide_the_heads():
+    from block_sparse_video_rearrange_b200 import pipeline
+    for n2 in (1, 2, 3, 4, 6, 8, 12, 24, 40, 7, 9, 32):
+        c = pipeline.default_chunks(n2)
+        assert n2 % c == 0 and 1 <= c <= 8
+    assert pipeline.default_chunks(40) == 8 and pipeline.default_chunks(24) == 8 and pipeline.default_chunks(9) == 3
