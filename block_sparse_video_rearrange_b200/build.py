@@ -11,7 +11,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librf.so")
-SOURCES = ["rf_plan.cu", "rf_rearrange.cu", "rf_select.cu", "rf_attn.cu", "rf_noalloc.cu"]
+SOURCES = ["rf_plan.cu", "rf_rearrange.cu", "rf_select.cu", "rf_attn.cu", "rf_noalloc.cu", "rf_selftest.cu"]
 
 
 def nvcc_path():

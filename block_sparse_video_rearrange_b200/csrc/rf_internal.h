@@ -77,6 +77,7 @@ rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_
                                cudaStream_t st);
 rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_num, void* ws,
                              cudaStream_t st);
+rf_status_t rf_launch_expired_wait_selftest(const rf_plan* p, void* ws, cudaStream_t st);
 rf_status_t rf_launch_exp2_selftest(const float* x, float* y_poly, float* y_mufu, int64_t n,
                                     cudaStream_t st);
 rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, const void* v_r,

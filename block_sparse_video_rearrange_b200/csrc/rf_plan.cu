@@ -424,6 +424,16 @@ rf_status_t rf_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64
   return rf_launch_exp2_selftest(x, y_poly, y_mufu, n, (cudaStream_t)stream);
 }
 
+rf_status_t rf_selftest_expired_wait(const rf_plan_t* p, void* ws, size_t ws_bytes,
+                                    rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  return rf_launch_expired_wait_selftest(p, ws, (cudaStream_t)stream);
+}
+
 rf_status_t rf_check_device_status(const rf_plan_t* p, void* ws, uint32_t* flags_out,
                                    rf_stream_t stream) {
   g_last_error.clear();

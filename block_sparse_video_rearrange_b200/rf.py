@@ -35,7 +35,8 @@ POOL_MODES = {"from_ws": 0, "recompute": 1}
 EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange", "rf_pool_select",
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
             "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
-            "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex", "rf_quantize_qk")
+            "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex", "rf_quantize_qk",
+            "rf_selftest_expired_wait")
 
 
 class RfError(RuntimeError):
@@ -83,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "rf_plan_create_ex": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
                               i32, i32, ctypes.POINTER(PlanOptions), ctypes.POINTER(vp)],
         "rf_quantize_qk": [vp, vp, vp, vp, sz, vp],
+        "rf_selftest_expired_wait": [vp, vp, sz, vp],
         "rf_plan_info": [vp, ctypes.POINTER(PlanInfo)],
         "rf_plan_seq_info": [vp, i32, ctypes.POINTER(SeqInfo)],
         "rf_rearrange": [vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -297,6 +299,12 @@ def selftest_exp2(x: torch.Tensor, stream=None) -> Tuple[torch.Tensor, torch.Ten
     yp, ym = torch.empty_like(x), torch.empty_like(x)
     _check(_lib.rf_selftest_exp2(_ptr(x), _ptr(yp), _ptr(ym), x.numel(), _stream(stream)), "rf_selftest_exp2")
     return yp, ym
+
+
+def selftest_expired_wait(plan: Plan, ws, stream=None) -> None:
+    """Provoke one expired bounded wait (about 1 s on the device) recorded in ws's status words."""
+    _check(_lib.rf_selftest_expired_wait(plan.handle, _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "rf_selftest_expired_wait")
 
 
 def check_device_status(plan: Plan, ws, stream=None) -> Tuple[int, Tuple[int, int]]:

@@ -319,6 +319,15 @@ RF_API rf_status_t rf_check_device_status(const rf_plan_t* plan, void* ws, uint3
 RF_API rf_status_t rf_selftest_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n,
                                     rf_stream_t stream);
 
+/* Self-test of the failure path of the kernels' bounded waits (the pages have
+ * no counterpart): one thread waits on a barrier that nothing completes, gives
+ * up after the same limit as every wait in rf_block_sparse_attn (1 s), and
+ * records the expiry in ws's status words as an attention CTA would (bit 31
+ * of the expired-wait word).  The next rf_check_device_status reports
+ * RF_ERR_DEVICE_FAULT and clears the words; the CUDA context stays usable.
+ * Takes about one second of device time; asynchronous on `stream`. */
+RF_API rf_status_t rf_selftest_expired_wait(const rf_plan_t* plan, void* ws, size_t ws_bytes,
+                                            rf_stream_t stream);
 /* Frees a plan (NULL is a no-op). */
 RF_API void rf_plan_destroy(rf_plan_t* plan);
 

@@ -49,6 +49,7 @@ def test_status_strings():
     (dict(seqs=[(-1, 2, 8, 8)]), 1),
     (dict(seqs=[(0, 2, 8, 8), (0, 2, 8, 8)]), 1),  # BNSD takes one geometry
     (dict(layout="TND", batch=2), 1),
+    (dict(seqs=[(0, 33, 64, 128)]), 6),       # 2,112 sparse blocks: beyond the 2,048 the kernels take
 ])
 def test_plan_validation(kwargs, status):
     args = dict(seqs=[(128, 9, 16, 32)], n1=2, n2=2, d=64, layout="BNSD", dtype="bf16", sparsity=0.8,

@@ -31,6 +31,10 @@ SMALL = {
     "s_one": W("s_one", "BNSD", "bf16", 1, (S(40, 9, 16, 32),), 2, 2, 128, 1.0, 15),
     # no text prefix at all, odd tile column count
     "no_prefix": W("no_prefix", "BNSD", "fp16", 1, (S(0, 6, 24, 40),), 2, 2, 64, 0.5, 16),
+    # text only: no video at all, three prefix blocks, the last one partial (44 rows)
+    "text_only": W("text_only", "BNSD", "bf16", 1, (S(300, 0, 0, 0),), 2, 2, 64, 0.8, 31),
+    # TND: a grid under 8 rows high (every video token promoted) next to a 2-block video
+    "all_promoted": W("all_promoted", "TND", "fp16", 1, (S(64, 3, 5, 9), S(0, 2, 16, 16)), 2, 1, 128, 0.8, 32),
 }
 
 
@@ -234,7 +238,7 @@ def test_frame_pair_full_size_parity(name, s):
 # inputs this precision defines) within the same bars as the native path.
 # ------------------------------------------------------------------------------------------
 
-MIX_SMALL = ["ragged_d128", "tnd_gqa_small", "dense", "s_one"]
+MIX_SMALL = ["ragged_d128", "tnd_gqa_small", "dense", "s_one", "all_promoted"]
 
 
 @pytest.mark.parametrize("name", MIX_SMALL)
@@ -281,6 +285,26 @@ def test_mix_quantize_entry_point_equals_fused_quantization():
     alone = parity.mix_buffers(plan, b.ws)
     for key in ("q8", "k8", "q_scale", "k_scale"):
         assert np.array_equal(alone[key], fused[key]), key
+
+
+def test_maximum_size_sequence():
+    """One sequence at the largest sizes the kernels take: 2,048 sparse blocks (the top-k
+    kernel's widest rows) and 2,048 key blocks per selectIdx row (the attention kernel's
+    list), 64 first-frame sinks, k = 410."""
+    w = W("maxsize", "BNSD", "bf16", 1, (S(0, 32, 64, 128),), 1, 1, 64, 0.8, 33)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    g = p.geoms[0]
+    assert (g.nb, g.n_blocks, g.ns, g.k) == (2048, 2048, 64, 410)
+    gpu = parity.run_gpu(w, bits)
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 1000), stats
+    items = [(0, 0), (63, 0), (64, 0), (1000, 0), (2047, 0)]     # sink, last sink, first sparse, middle, last
+    parity.check_attention(p, w, rbits, gpu, items)
 
 
 def test_exp2_polynomial_against_mufu_and_exact():
