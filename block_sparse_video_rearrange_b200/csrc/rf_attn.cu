@@ -217,7 +217,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(rf_smem_u32(&sm.bar_q), 1);
     for (int i = 0; i < kStagesK; ++i) {
       mbar_init(rf_smem_u32(&sm.bar_k_full[i]), 1);
       mbar_init(rf_smem_u32(&sm.bar_k_empty[i]), 1);
@@ -237,7 +236,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == kProducerWarp && lane == 0) {
+    // The Q tile does not depend on the selection: request it first thing.
+    mbar_init(rf_smem_u32(&sm.bar_q), 1);
+    fence_mbar_init();
     tma_prefetch_desc(&tm_q);
+    int c1, c2;
+    if (g.layout == RF_LAYOUT_BNSD) { c1 = q_r0; c2 = s.batch_idx * g.n1 + n; }
+    else                            { c1 = n; c2 = (int)s.row_off + q_r0; }
+    mbar_arrive_expect_tx(rf_smem_u32(&sm.bar_q), kQkTileBytes);
+#pragma unroll
+    for (int x = 0; x < kQkBoxes; ++x)
+      tma_load_3d(rf_smem_u32(sm.q + x * kBoxBytes), &tm_q, rf_smem_u32(&sm.bar_q), x * 64, c1, c2);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
@@ -245,28 +254,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(rf_smem_u32(&sm.tmem_base), kTmemCols);
     tmem_relinquish();
   }
+  // The selectIdx row (and, with E4M3 Q and K, each entry's K scale) into
+  // shared memory: every thread loads, so the row costs one round trip.
+  const size_t row_id = (size_t)tb * g.n1 + n;
+  const int32_t* row = a.sel_idx + row_id * g.max_kv;
+  const int num_raw = a.sel_num[row_id];
+  const int num = num_raw < 0 ? 0 : (num_raw > g.max_kv ? g.max_kv : num_raw);
+  for (int c = threadIdx.x; c < num; c += kThreads) {
+    const int v = row[c];
+    sm.list[c] = v;
+    if constexpr (kQk8)
+      if (v >= 0 && v < nblk) sm.kscale[c] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
+  }
+  __syncthreads();
   if (warp == 0) {
-    // Compact the selectIdx row: keep in-range entries in order, skip -1
-    // (an unused slot), count anything else as a bad index.
-    const size_t row_id = (size_t)tb * g.n1 + n;
-    const int32_t* row = a.sel_idx + row_id * g.max_kv;
-    int num = a.sel_num[row_id];
-    int bad = 0;
-    if (num < 0 || num > g.max_kv) {
-      bad = 1;
-      num = num < 0 ? 0 : g.max_kv;
-    }
+    // Compact the row in place: keep in-range entries in order, skip -1 (an
+    // unused slot), count anything else as a bad index.  A lane writes at or
+    // below its own read position, and every lane reads before the ballot.
+    int bad = (lane == 0 && num != num_raw) ? 1 : 0;
     int cnt = 0;
     const uint32_t lt = (1u << lane) - 1u;
     for (int c0 = 0; c0 < num; c0 += 32) {
       const int c = c0 + lane;
-      const int v = c < num ? row[c] : -1;
+      const int v = c < num ? sm.list[c] : -1;
+      float ks = 0.f;
+      if constexpr (kQk8) ks = c < num ? sm.kscale[c] : 0.f;
       const bool ok = c < num && v >= 0 && v < nblk;
       if (c < num && v != -1 && !ok) ++bad;
       const uint32_t ball = __ballot_sync(0xffffffffu, ok);
       if (ok) {
         sm.list[cnt + __popc(ball & lt)] = v;
-        if constexpr (kQk8) sm.kscale[cnt + __popc(ball & lt)] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
+        if constexpr (kQk8) sm.kscale[cnt + __popc(ball & lt)] = ks;
       }
       cnt += __popc(ball);
     }
@@ -297,13 +315,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     int c1, c2;
     const uint32_t bq = rf_smem_u32(&sm.bar_q);
-    if (is_k) {
-      coords(g.n1, n, q_r0, c1, c2);
-      mbar_arrive_expect_tx(bq, kQkTileBytes);
-#pragma unroll
-      for (int x = 0; x < kQkBoxes; ++x)
-        tma_load_3d(rf_smem_u32(sm.q + x * kBoxBytes), &tm_q, bq, x * 64, c1, c2);
-    }
     const int stages = is_k ? kStagesK : kStagesV;
     const uint32_t tile_bytes = is_k ? kQkTileBytes : kVTileBytes;
     const int boxes = is_k ? kQkBoxes : kVBoxes;
@@ -413,6 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     volatile int no_abort = 0;
     warp_wait(rf_smem_u32(&sm.bar_drain), 0, &no_abort);
+  }
+  if (warp == kProducerWarp && lane == 0 && nv == 0) {
+    // Nothing to compute (an empty row, or a recorded expiry): the Q copy
+    // requested at the start still has to land before the CTA exits.
+    volatile int no_abort = 0;
+    mbar_wait(rf_smem_u32(&sm.bar_q), 0, &no_abort);
   }
   } else {
     reg_alloc<kSoftmaxRegs>();
