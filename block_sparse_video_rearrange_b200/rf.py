@@ -344,7 +344,8 @@ def forward(plan: Plan, q, k, v, bufs: Buffers, scale: Optional[float] = None, s
     return b.o
 
 
-_PIPELINES = {}
+_PIPELINES = {}        # host pipelines (with their device buffers) of recent problem shapes
+_PIPELINES_KEPT = 4
 
 
 def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
@@ -378,10 +379,12 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         dev = torch.device("cuda", torch.cuda.current_device())
         key = (tuple(map(tuple, seqs)), n1, n2, d, layout, dtype, float(sparsity), batch, order, precision,
                chunks, dev.index)
-        pipe = _PIPELINES.get(key)
+        pipe = _PIPELINES.pop(key, None)
         if pipe is None:
             pipe = HostPipeline(seqs, n1, n2, d, layout, dtype, sparsity, batch, chunks, order, precision, dev)
-            _PIPELINES[key] = pipe
+            while len(_PIPELINES) >= _PIPELINES_KEPT:      # drop the least recently used shape
+                _PIPELINES.pop(next(iter(_PIPELINES)))
+        _PIPELINES[key] = pipe                               # most recently used last
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
         pipe(q, k, v, out, scale)
         torch.cuda.current_stream(dev).synchronize()
