@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--order", default="tile", choices=["tile", "frame_pair"],
                     help="token order of the aligned video (frame_pair: frames paired into 2x8x8 blocks)")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--chunks", type=int, default=None,
+                    help="head chunks of the host pipeline in the e2e measurement (default: the library's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--heads", type=int, default=None,
@@ -351,7 +353,7 @@ def main():
         def e2e_step():
             nonlocal out_host
             out_host = rf.rainfusion_attention(host[0], host[1], host[2], seqs, w.sparsity, w.layout, scale,
-                                               order=args.order, precision=args.precision)
+                                               order=args.order, precision=args.precision, chunks=args.chunks)
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(dev)

@@ -31,8 +31,14 @@ except ImportError:  # pragma: no cover - older cuda-python layout
         _cudart = None
 
 
-def default_chunks(n2: int, limit: int = 8) -> int:
-    """Largest divisor of the key/value head count not above `limit`."""
+def default_chunks(n2: int, limit: int = 20) -> int:
+    """Largest divisor of the key/value head count not above `limit`.
+
+    More chunks shorten the pipeline's fill and drain (the first chunk's copy in
+    and the last chunk's compute and copy out run alone), until a chunk holds so
+    few heads that its launches stop filling the GPU: on a 40-head layer with
+    bf16 D = 128 and 33k rows, 20 chunks beat 8 by about 4 % and 40 chunks lose.
+    """
     return max(c for c in range(1, min(n2, limit) + 1) if n2 % c == 0)
 
 

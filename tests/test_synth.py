@@ -45,5 +45,6 @@ def test_pipeline_default_chunks_divide_the_heads():
     from block_sparse_video_rearrange_b200 import pipeline
     for n2 in (1, 2, 3, 4, 6, 8, 12, 24, 40, 7, 9, 32):
         c = pipeline.default_chunks(n2)
-        assert n2 % c == 0 and 1 <= c <= 8
-    assert pipeline.default_chunks(40) == 8 and pipeline.default_chunks(24) == 8 and pipeline.default_chunks(9) == 3
+        assert n2 % c == 0 and 1 <= c <= 20
+    assert pipeline.default_chunks(40) == 20 and pipeline.default_chunks(24) == 12 and pipeline.default_chunks(9) == 9
+    assert pipeline.default_chunks(7) == 7 and pipeline.default_chunks(64) == 16
