@@ -51,8 +51,9 @@ def parse():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="wan", choices=sorted(WORKLOAD_DESC))
     ap.add_argument("--sparsity", type=float, default=None)
-    ap.add_argument("--precision", default="native", choices=["native", "mix"],
-                    help="kernel precision (mix: E4M3 Q K^T with per-block scales, 16-bit P V)")
+    ap.add_argument("--precision", default="native", choices=["native", "mix", "mxfp4"],
+                    help="kernel precision (mix: E4M3 Q K^T with per-block scales, 16-bit P V; "
+                         "mxfp4: MXFP4 operands with UOS scaling and PNQ, on the 16-bit tensor cores)")
     ap.add_argument("--order", default="tile", choices=["tile", "frame_pair"],
                     help="token order of the aligned video (frame_pair: frames paired into 2x8x8 blocks)")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -133,6 +134,9 @@ def algorithmic_bytes(plan, elem=2):
     inv = 2 * rows * plan.n1 * plan.d * elem
     # precision "mix": the rearrange also writes one-byte copies of Q' and K' and their scales
     quant = rows * (plan.n1 + plan.n2) * plan.d + 4 * t * (plan.n1 + plan.n2) if plan.precision == "mix" else 0
+    # precision "mxfp4": 16-bit MXFP4-rounded copies of Q', K' and V'
+    if plan.precision == "mxfp4":
+        quant = rows * (plan.n1 + 2 * plan.n2) * plan.d * 2
     return 2 * qkv + sel + quant, inv
 
 
@@ -391,11 +395,14 @@ def main():
             # rate: the harmonic combination is 4/3 of the 16-bit peak.
             peak = round(peak * 4.0 / 3.0, 1)
             peak_note += "; mix: QK^T at 2x (fp8, nominal ratio), PV at 1x -> 4/3 x"
+        if args.precision == "mxfp4":
+            peak_note += "; mxfp4: both products run on the 16-bit tensor cores -> 1x"
         front_bytes, inv_bytes = algorithmic_bytes(plan)
         front_ms = float(np.mean(per[:, 0] + per[:, 1]))
         inv_ms = float(np.mean(per[:, 3]))
         value = flops_all / (ms_step * 1e-3) / 1e12
-        traffic = (profiled_traffic(w.name.split("@")[0], sparsity, "/mix" if args.precision == "mix" else "")
+        traffic = (profiled_traffic(w.name.split("@")[0], sparsity,
+                                    "" if args.precision == "native" else "/" + args.precision)
                    if args.order == "tile" and not args.heads else None)
         line = {
             "metric": METRIC,
@@ -408,12 +415,14 @@ def main():
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": ("e4m3+" if args.precision == "mix" else "") + ("bf16" if w.dtype == "bf16" else "fp16"),
+            "dtype": {"mix": "e4m3+", "mxfp4": "mxfp4 on "}.get(args.precision, "") + ("bf16" if w.dtype == "bf16" else "fp16"),
             "data": "synthetic (seeded smooth-field + noise per 8x8 cell; no real activations available)",
             "config": {"workload": WORKLOAD_DESC[w.name.split("@")[0]] + (f" [reduced to {w.n1} heads]" if args.heads else ""),
                        "sparsity": sparsity,
                        **({"token_order": args.order} if args.order != "tile" else {}),
                        **({"precision": "mix (E4M3 QK^T, 16-bit PV)"} if args.precision == "mix" else {}),
+                       **({"precision": "mxfp4 (UOS Qmax 7.25, PNQ; MXFP4 values on the 16-bit tensor cores)"}
+                          if args.precision == "mxfp4" else {}),
                        "global_batch": w.batch * world, "seq_len": int(plan.info.rows_total),
                        "parallelism": f"independent layer per GPU x{world}",
                        "l2": "inputs larger than L2 (Q+K+V %.2f GB vs 126 MB)" % (

@@ -48,7 +48,19 @@
 // the default mask is 0.
 // Every wait is bounded: on expiry the CTA records it in the status words and
 // unwinds (waiting, again bounded, for its own copies and MMAs in flight).
+//
+// Precision "mxfp4" (kMx; MXAttention abstract: MXFP4 attention with UOS
+// scaling and Pre-Normalization Quantization): Q, K and V arrive already
+// rounded to MXFP4 (exact 16-bit values; V as f16).  The softmax keeps its
+// running max an integer (log2 units) and, for every group of 32 keys, takes
+// the exponentials against m + e, e the group's UOS exponent, so that they
+// land in (3.625, 7.25] at the top; it rounds them to E2M1 in hardware,
+// accumulates the row sum from the rounded values (PNQ) and hands P V the
+// rounded values times 2^e as f16.  Power-of-two scales make the rounded P
+// independent of which integer the running max is, so the result does not
+// depend on the order the blocks are visited in.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <mutex>
 
@@ -177,6 +189,72 @@ __device__ __forceinline__ void half_row_exp(const uint32_t* sr, int c0, int vr,
   }
 }
 
+// Maxima of the four 32-column groups of a row of raw scores (the first vr
+// valid; a group with no valid column gives -inf).
+template <bool kFull>
+__device__ __forceinline__ void group_max4(const uint32_t* sr, int vr, float* gm) {
+#pragma unroll
+  for (int gi = 0; gi < 4; ++gi) {
+    float m[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 32 * gi; c < 32 * gi + 32; c += 2) {
+      if (kFull) {
+        m[(c >> 1) & 1] = rf_max3(m[(c >> 1) & 1], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+      } else {
+        if (c < vr) m[0] = fmaxf(m[0], __uint_as_float(sr[c]));
+        if (c + 1 < vr) m[1] = fmaxf(m[1], __uint_as_float(sr[c + 1]));
+      }
+    }
+    gm[gi] = fmaxf(m[0], m[1]);
+  }
+}
+
+// Precision "mxfp4": P over the 64 scores c0 .. c0 + 63 of a row (two groups
+// of 32 keys), rounded to MXFP4 per group and packed as f16 pairs into
+// pk[32]; the rounded values are summed into lsum.  m is the integer running
+// max; gm2 the two groups' raw score maxima.  Group exponent (UOS):
+// e = ceil(log2(amax / 7.25)) with log2(amax) = gmax * sl2 - m; the
+// exponentials are taken as 2^(s * sl2 - (m + e)), rounded to E2M1 (the
+// hardware conversion saturates at 6), summed exactly in f16 (at most 32
+// values of at most 6 on a 0.5 grid) and scaled by 2^e.
+template <bool kFull>
+__device__ __forceinline__ void half_row_exp_mx(const uint32_t* sr, int c0, int vr, float sl2, float m,
+                                                const float* gm2, uint32_t* pk, float& lsum) {
+  const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int cb = c0 + 32 * h;
+    const bool live = kFull || cb < vr;
+    const int e = live ? (int)ceilf(fmaf(gm2[h], sl2, -m) - kMxLog2Qmax) : 0;
+    const float neg_me = -(m + (float)e);
+    const uint64_t negme2 = rf_f2(__float_as_uint(neg_me), __float_as_uint(neg_me));
+    // 2^e as f16 (normal from 2^-14, subnormal down to 2^-24; a group whose
+    // scale is below that rounds to zero in f16, as its P V terms would)
+    const unsigned short hb = e >= -14 ? (unsigned short)((15 + e) << 10)
+                                       : (e >= -24 ? (unsigned short)(1u << (e + 24)) : (unsigned short)0);
+    const __half2 up2 = __half2half2(__ushort_as_half(hb));
+    __half2 acc0 = __float2half2_rn(0.f), acc1 = acc0;
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+      float x0, x1;
+      rf_f2_split(rf_fma2(rf_f2(sr[cb + c], sr[cb + c + 1]), sl2x2, negme2), x0, x1);
+      float y0 = rf_ex2(x0), y1 = rf_ex2(x1);
+      if (!kFull) {
+        y0 = cb + c < vr ? y0 : 0.f;
+        y1 = cb + c + 1 < vr ? y1 : 0.f;
+      }
+      const uint32_t r = rf_e2m1x2_round(y0, y1);
+      const __half2 rh = *reinterpret_cast<const __half2*>(&r);
+      if (c & 2) acc1 = __hadd2(acc1, rh);
+      else       acc0 = __hadd2(acc0, rh);
+      const __half2 ph = __hmul2(rh, up2);
+      pk[(cb - c0 + c) >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
+    }
+    const float2 sum = __half22float2(__hadd2(acc0, acc1));
+    if (live && e >= -126) lsum = fmaf(sum.x + sum.y, rf_pow2(e), lsum);
+  }
+}
+
 __device__ __forceinline__ float acc_sum(const uint64_t* acc) {
   float s = 0.f;
 #pragma unroll
@@ -188,7 +266,7 @@ __device__ __forceinline__ float acc_sum(const uint64_t* acc) {
   return s;
 }
 
-template <int D, bool kBf16, bool kQk8>
+template <int D, bool kBf16, bool kQk8, bool kMx>
 __global__ void __launch_bounds__(kThreads, 1)
     rf_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
@@ -355,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t fmt = kBf16 ? 1u : 0u;
     // kind::f8f6f4 takes E4M3 as format 0 in the same descriptor fields.
     const uint32_t idesc_qk = umma_idesc_f16(kQk8 ? 0u : fmt, 128, 128, 0);
-    const uint32_t idesc_pv = umma_idesc_f16(fmt, 128, D, 1);
+    // precision "mxfp4": P and V are f16 whatever the input type
+    const uint32_t idesc_pv = umma_idesc_f16(kMx ? 0u : fmt, 128, D, 1);
     // Adding (bytes >> 4) to a descriptor moves its 14-bit start-address field.
     const uint64_t dq = umma_desc_sw128(rf_smem_u32(sm.q), 16, 1024);
     const uint64_t dk0 = umma_desc_sw128(rf_smem_u32(sm.k[0]), 16, 1024);
@@ -456,10 +535,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(scol + 64, sr + 64);
       tmem_ld32(scol + 96, sr + 96);
       tmem_wait_ld();
-      const float mx_t = (vr == RF_BLOCK ? row_max<true>(sr, vr) : row_max<false>(sr, vr)) * sl2;
+      float gm[4];
+      float mx_t;
+      if constexpr (kMx) {
+        if (vr == RF_BLOCK) group_max4<true>(sr, vr, gm);
+        else                group_max4<false>(sr, vr, gm);
+        mx_t = fmaxf(fmaxf(gm[0], gm[1]), fmaxf(gm[2], gm[3])) * sl2;
+      } else {
+        mx_t = (vr == RF_BLOCK ? row_max<true>(sr, vr) : row_max<false>(sr, vr)) * sl2;
+      }
       const bool rescale = __any_sync(0xffffffffu, mx_t > m_run + kRescaleThreshold);
       if (rescale) {
-        const float m_new = fmaxf(m_run, mx_t);
+        // mxfp4: the running max stays an integer
+        const float m_new = kMx ? ceilf(fmaxf(m_run, mx_t)) : fmaxf(m_run, mx_t);
         const float alpha = rf_ex2(m_run - m_new);
         l_run *= alpha;
         m_run = m_new;
@@ -482,16 +570,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       // at a time: the first half is released to the MMA warp while the second
       // is being computed.
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      float lsum = 0.f;
       uint32_t pk[32];
-      if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 0, vr, sl2, -m_run, pk, acc);
-      else                half_row_exp<kBf16, false>(sr, 0, vr, sl2, -m_run, pk, acc);
+      if constexpr (kMx) {
+        if (vr == RF_BLOCK) half_row_exp_mx<true>(sr, 0, vr, sl2, m_run, gm, pk, lsum);
+        else                half_row_exp_mx<false>(sr, 0, vr, sl2, m_run, gm, pk, lsum);
+      } else {
+        if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 0, vr, sl2, -m_run, pk, acc);
+        else                half_row_exp<kBf16, false>(sr, 0, vr, sl2, -m_run, pk, acc);
+      }
       tmem_st32(scol, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(rf_smem_u32(&sm.bar_p_half[wg]));
-      if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 64, vr, sl2, -m_run, pk, acc);
-      else                half_row_exp<kBf16, false>(sr, 64, vr, sl2, -m_run, pk, acc);
-      l_run += acc_sum(acc);
+      if constexpr (kMx) {
+        if (vr == RF_BLOCK) half_row_exp_mx<true>(sr, 64, vr, sl2, m_run, gm + 2, pk, lsum);
+        else                half_row_exp_mx<false>(sr, 64, vr, sl2, m_run, gm + 2, pk, lsum);
+        l_run += lsum;
+      } else {
+        if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 64, vr, sl2, -m_run, pk, acc);
+        else                half_row_exp<kBf16, false>(sr, 64, vr, sl2, -m_run, pk, acc);
+        l_run += acc_sum(acc);
+      }
       tmem_st32(scol + 32, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -584,10 +684,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Element type of a tensor map: the plan's 16-bit type, E4M3 bytes, or f16.
+enum MapElem { kElemPlan = 0, kElemByte = 1, kElemF16 = 2 };
+
 // Tensor map over [rows, heads, D] (TND) or [B*heads, rows, D] (BNSD) with a
 // 128-row x 128-byte box and 128-byte swizzle: 64 columns of a 16-bit tensor,
 // or 128 columns of a one-byte (E4M3) tensor.
-rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int heads, bool one_byte) {
+rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int heads, MapElem elem) {
+  const bool one_byte = elem == kElemByte;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return rf_fail(RF_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const RfGeomDev& g = p->g;
@@ -607,8 +711,8 @@ rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int hea
     box[0] = box_cols; box[1] = 1; box[2] = RF_BLOCK;
   }
   const CUtensorMapDataType dt = one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8
-                                 : p->dtype == RF_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+                                 : (p->dtype == RF_BF16 && elem == kElemPlan) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -617,14 +721,14 @@ rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int hea
   return RF_OK;
 }
 
-template <int D, bool kBf16, bool kQk8>
+template <int D, bool kBf16, bool kQk8, bool kMx = false>
 rf_status_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const AttnArgs& args, unsigned grid, cudaStream_t st) {
   size_t smem = sizeof(AttnSmem<D, kQk8>) + 1024;
   // D = 64 tiles are small: ask for enough shared memory that one CTA holds
   // an SM, since each CTA takes all 512 TMEM columns.
   if (smem < 120 * 1024) smem = 120 * 1024;
-  auto kern = rf_attn_kernel<D, kBf16, kQk8>;
+  auto kern = rf_attn_kernel<D, kBf16, kQk8, kMx>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return rf_check_launch("cudaFuncSetAttribute(rf_attn_kernel)");
@@ -653,14 +757,18 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   if (grid > 0x7FFFFFFFll) return rf_fail(RF_ERR_INVALID_ARG, "grid too large");
   CUtensorMap mq, mk, mv;
   rf_status_t s;
-  // precision "mix": Q K^T reads the E4M3 copies rf_rearrange wrote into ws.
+  // precision "mix": Q K^T reads the E4M3 copies rf_rearrange wrote into ws;
+  // precision "mxfp4": every operand reads the MXFP4 copies in ws (V as f16).
   const bool mix = p->precision == RF_PRECISION_MIX;
+  const bool mx = p->precision == RF_PRECISION_MXFP4;
   char* w = static_cast<char*>(ws);
-  const void* qsrc = mix ? static_cast<const void*>(w + p->off_q8) : q_r;
-  const void* ksrc = mix ? static_cast<const void*>(w + p->off_k8) : k_r;
-  if ((s = make_map(&mq, p, qsrc, g.n1, mix)) != RF_OK) return s;
-  if ((s = make_map(&mk, p, ksrc, g.n2, mix)) != RF_OK) return s;
-  if ((s = make_map(&mv, p, v_r, g.n2, false)) != RF_OK) return s;
+  const void* qsrc = mix ? static_cast<const void*>(w + p->off_q8) : mx ? static_cast<const void*>(w + p->off_qx) : q_r;
+  const void* ksrc = mix ? static_cast<const void*>(w + p->off_k8) : mx ? static_cast<const void*>(w + p->off_kx) : k_r;
+  const void* vsrc = mx ? static_cast<const void*>(w + p->off_vx) : v_r;
+  const MapElem qk_elem = mix ? kElemByte : kElemPlan;
+  if ((s = make_map(&mq, p, qsrc, g.n1, qk_elem)) != RF_OK) return s;
+  if ((s = make_map(&mk, p, ksrc, g.n2, qk_elem)) != RF_OK) return s;
+  if ((s = make_map(&mv, p, vsrc, g.n2, mx ? kElemF16 : kElemPlan)) != RF_OK) return s;
   AttnArgs args;
   args.g = g;
   args.sel_idx = sel_idx;
@@ -675,9 +783,15 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
     if (mix)
       return bf ? launch_t<128, true, true>(mq, mk, mv, args, (unsigned)grid, st)
                 : launch_t<128, false, true>(mq, mk, mv, args, (unsigned)grid, st);
+    if (mx)
+      return bf ? launch_t<128, true, false, true>(mq, mk, mv, args, (unsigned)grid, st)
+                : launch_t<128, false, false, true>(mq, mk, mv, args, (unsigned)grid, st);
     return bf ? launch_t<128, true, false>(mq, mk, mv, args, (unsigned)grid, st)
               : launch_t<128, false, false>(mq, mk, mv, args, (unsigned)grid, st);
   }
+  if (mx)
+    return bf ? launch_t<64, true, false, true>(mq, mk, mv, args, (unsigned)grid, st)
+              : launch_t<64, false, false, true>(mq, mk, mv, args, (unsigned)grid, st);
   return bf ? launch_t<64, true, false>(mq, mk, mv, args, (unsigned)grid, st)
             : launch_t<64, false, false>(mq, mk, mv, args, (unsigned)grid, st);
 }

@@ -397,6 +397,52 @@ __device__ __forceinline__ uint32_t rf_pack2(float a, float b) {
 }
 
 // ---------------------------------------------------------------------------
+// MXFP4: E2M1 elements (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) sharing one
+// power-of-two scale per group of 32 (MXAttention abstract: MXFP4 attention
+// with Universal Optimal Scaling, boundary Qmax = 7.25).
+// ---------------------------------------------------------------------------
+constexpr float kMxQmax = 7.25f;
+constexpr float kMxLog2Qmax = 2.857980995127572f;  // log2(7.25)
+
+// Two floats rounded to E2M1 (nearest, ties to the even code, saturating at
+// +-6), returned as the exact f16 values of the two codes: a in the low half.
+__device__ __forceinline__ uint32_t rf_e2m1x2_round(float a, float b) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 c;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 c, %1, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+      : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// ceil(log2(t)) for finite t > 0, from the bits (subnormals scaled up first).
+__device__ __forceinline__ int rf_ceil_log2(float t) {
+  int off = 0;
+  if (t < 1.17549435e-38f) {
+    t *= 18446744073709551616.0f;  // 2^64, exact
+    off = 64;
+  }
+  const uint32_t b = __float_as_uint(t);
+  return (int)(b >> 23) - 127 + ((b & 0x7FFFFFu) != 0u ? 1 : 0) - off;
+}
+
+// 2^k as a float, -126 <= k <= 127.
+__device__ __forceinline__ float rf_pow2(int k) { return __int_as_float((127 + k) << 23); }
+
+// x * 2^k for |k| <= 252, as two exact power-of-two products.
+__device__ __forceinline__ float rf_scale_pow2(float x, int k) {
+  const int k1 = k / 2;
+  return x * rf_pow2(k1) * rf_pow2(k - k1);
+}
+
+// UOS shared exponent of a group whose largest magnitude is amax: the
+// smallest e with amax <= 7.25 * 2^e (0 for an all-zero group).  amax / 7.25
+// is a correctly rounded division, so a boundary value 7.25 * 2^k gives k.
+__device__ __forceinline__ int rf_uos_exponent(float amax) {
+  return amax > 0.f ? rf_ceil_log2(__fdiv_rn(amax, kMxQmax)) : 0;
+}
+
+// ---------------------------------------------------------------------------
 // UMMA (tcgen05) descriptors
 // ---------------------------------------------------------------------------
 

@@ -56,6 +56,8 @@ struct rf_plan {
   rf_precision_t precision;
   rf_token_order_t token_order;
   int64_t off_q8, off_k8, off_qs, off_ks;  // RF_PRECISION_MIX workspace regions, else -1
+  int64_t off_qx, off_kx, off_vx;          // RF_PRECISION_MXFP4 workspace regions, else -1
+  int64_t off_quant;                       // first precision-specific region (ws_bytes if none)
   int64_t kept_flops_upper;
 };
 
@@ -73,8 +75,8 @@ rf_status_t rf_launch_rearrange(const rf_plan* p, const void* q, const void* k, 
 rf_status_t rf_launch_pool(const rf_plan* p, const void* q_r, const void* k_r, void* ws,
                            cudaStream_t st);
 rf_status_t rf_launch_inverse(const rf_plan* p, const void* o_r, void* o, cudaStream_t st);
-rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_r, void* ws,
-                               cudaStream_t st);
+rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_r, const void* v_r,
+                               void* ws, cudaStream_t st);
 rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_num, void* ws,
                              cudaStream_t st);
 rf_status_t rf_launch_expired_wait_selftest(const rf_plan* p, void* ws, cudaStream_t st);

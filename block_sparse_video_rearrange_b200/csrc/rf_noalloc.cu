@@ -65,9 +65,9 @@ extern "C" rf_status_t rf_pool_select_noalloc(const rf_plan_t* p, const void* q_
     return rf_fail(RF_ERR_INVALID_ARG, "null tensor");
   if ((reinterpret_cast<uintptr_t>(q_r) & 15) || (reinterpret_cast<uintptr_t>(k_r) & 15))
     return rf_fail(RF_ERR_INVALID_ARG, "q_r and k_r must be 16-byte aligned");
-  // The selection part of the workspace layout (a mix-precision plan puts its
-  // E4M3 copies after it; selection never touches them).
-  const int64_t sel_bytes = p->off_q8 >= 0 ? p->off_q8 : p->ws_bytes;
+  // The selection part of the workspace layout (mix and mxfp4 plans put their
+  // quantized copies after it; selection never touches them).
+  const int64_t sel_bytes = p->off_quant;
   if ((uint64_t)sel_bytes > RF_NOALLOC_SCRATCH_BYTES)
     return rf_fail(RF_ERR_INVALID_ARG,
                    "this problem needs " + std::to_string(sel_bytes) +

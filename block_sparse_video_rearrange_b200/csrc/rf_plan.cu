@@ -126,7 +126,7 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   if (opt.token_order != RF_ORDER_TILE && opt.token_order != RF_ORDER_FRAME_PAIR)
     return rf_fail(RF_ERR_INVALID_ARG, "token order must be RF_ORDER_TILE or RF_ORDER_FRAME_PAIR");
   if (opt.precision != RF_PRECISION_NATIVE && opt.precision != RF_PRECISION_MIX &&
-      opt.precision != RF_PRECISION_FP8)
+      opt.precision != RF_PRECISION_FP8 && opt.precision != RF_PRECISION_MXFP4)
     return rf_fail(RF_ERR_INVALID_ARG, "unknown precision");
   if (opt.precision == RF_PRECISION_FP8)
     return rf_fail(RF_ERR_UNSUPPORTED, "precision fp8 (FP8 P V) is not built; use mix");
@@ -246,6 +246,8 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   p->precision = (rf_precision_t)opt.precision;
   p->token_order = order;
   p->off_q8 = p->off_k8 = p->off_qs = p->off_ks = -1;
+  p->off_qx = p->off_kx = p->off_vx = -1;
+  p->off_quant = off;
   if (p->precision == RF_PRECISION_MIX) {
     p->off_q8 = off;
     off = align_up(off + p->rows_total * n1 * d, 256);
@@ -255,6 +257,16 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
     off = align_up(off + (int64_t)n1 * qblk * 4, 256);
     p->off_ks = off;
     off = align_up(off + (int64_t)n2 * qblk * 4, 256);
+  }
+  // RF_PRECISION_MXFP4: MXFP4-rounded 16-bit copies of Q', K', V' (layouts of
+  // q_r / k_r / v_r).
+  if (p->precision == RF_PRECISION_MXFP4) {
+    p->off_qx = off;
+    off = align_up(off + p->rows_total * n1 * d * 2, 256);
+    p->off_kx = off;
+    off = align_up(off + p->rows_total * n2 * d * 2, 256);
+    p->off_vx = off;
+    off = align_up(off + p->rows_total * n2 * d * 2, 256);
   }
   p->ws_bytes = off;
   *out = p;
@@ -281,6 +293,9 @@ rf_status_t rf_plan_info(const rf_plan_t* p, rf_plan_info_t* out) {
   out->ws_k8 = p->off_k8;
   out->ws_q_scale = p->off_qs;
   out->ws_k_scale = p->off_ks;
+  out->ws_q_mx = p->off_qx;
+  out->ws_k_mx = p->off_kx;
+  out->ws_v_mx = p->off_vx;
   return RF_OK;
 }
 
@@ -341,7 +356,21 @@ rf_status_t rf_quantize_qk(const rf_plan_t* p, const void* q_r, const void* k_r,
   rf_status_t st = check_ws(p, ws, ws_bytes);
   if (st != RF_OK) return st;
   if ((st = rf_require_device()) != RF_OK) return st;
-  return rf_launch_quantize(p, q_r, k_r, ws, (cudaStream_t)stream);
+  return rf_launch_quantize(p, q_r, k_r, nullptr, ws, (cudaStream_t)stream);
+}
+
+rf_status_t rf_quantize_mx(const rf_plan_t* p, const void* q_r, const void* k_r, const void* v_r,
+                           void* ws, size_t ws_bytes, rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (p->precision != RF_PRECISION_MXFP4)
+    return rf_fail(RF_ERR_INVALID_ARG, "rf_quantize_mx needs a plan with precision mxfp4");
+  if (!q_r || !k_r || !v_r || !aligned16(q_r) || !aligned16(k_r) || !aligned16(v_r))
+    return rf_fail(RF_ERR_INVALID_ARG, "q_r, k_r and v_r must be non-null and 16-byte aligned");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  return rf_launch_quantize(p, q_r, k_r, v_r, ws, (cudaStream_t)stream);
 }
 
 rf_status_t rf_pool_select(const rf_plan_t* p, const void* q_r, const void* k_r,

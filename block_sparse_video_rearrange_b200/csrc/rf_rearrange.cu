@@ -12,6 +12,9 @@
 //
 // With precision "mix" the rearrange also writes an E4M3 copy of each Q and K
 // block with its fp32 scale (amax / 448) while the block is in registers.
+// With precision "mxfp4" it writes MXFP4-rounded copies instead: Q and K rows
+// in groups of 32 columns, V columns in groups of 32 rows of each block, each
+// group on its UOS power-of-two scale, stored as the exact 16-bit values.
 //
 // One CTA moves one 128-row block of one head of one tensor: 16-byte vector
 // loads and stores, whole rows per group of D/8 threads, every load of a
@@ -25,15 +28,43 @@
 namespace {
 
 enum Mode { kRearrange = 0, kInverse = 1, kPoolOnly = 2, kQuantOnly = 3 };
+enum Quant { kQuantNone = 0, kQuantE4M3 = 1, kQuantMx = 2 };
 
-// Outputs of the fused E4M3 quantization (precision "mix"): one-byte copies of
-// Q' and K' in their layouts, and one fp32 scale per (head, global block).
+// Outputs of the fused quantization.  Precision "mix": one-byte E4M3 copies of
+// Q' and K' in their layouts and one fp32 scale per (head, global block).
+// Precision "mxfp4": MXFP4-rounded copies of Q' and K' (input dtype) and of V'
+// (always f16, the type of the P V product), in the layouts of q_r, k_r, v_r.
 struct QuantOut {
   uint8_t* q8;
   uint8_t* k8;
   float* q_scale;
   float* k_scale;
+  uint4* qx;
+  uint4* kx;
+  uint4* vx;
 };
+
+// Eight 16-bit values (one 16-byte chunk) rounded to MXFP4, element i on
+// shared exponent e[i]: E2M1(x / 2^e) * 2^e, packed as kOutBf16 ? bf16 : f16.
+// f16 results saturate at +-65504 (a V group whose rounding would go beyond).
+template <class Dec, bool kOutBf16>
+__device__ __forceinline__ uint4 rf_mx_round8(const uint4 v, const int* e) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int e0 = e[2 * c], e1 = e[2 * c + 1];
+    const uint32_t h = rf_e2m1x2_round(rf_scale_pow2(Dec::lo(w[c]), -e0), rf_scale_pow2(Dec::hi(w[c]), -e1));
+    float y0 = rf_scale_pow2(__half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu))), e0);
+    float y1 = rf_scale_pow2(__half2float(__ushort_as_half((unsigned short)(h >> 16))), e1);
+    if (!kOutBf16) {
+      y0 = fminf(fmaxf(y0, -65504.f), 65504.f);
+      y1 = fminf(fmaxf(y1, -65504.f), 65504.f);
+    }
+    o[c] = rf_pack2<kOutBf16>(y0, y1);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
 
 // Four floats to four E4M3 codes (round to nearest even, saturating at
 // +-448), the first in the lowest byte.
@@ -48,10 +79,12 @@ constexpr int kThreads = 256;
 
 // How the fused pooling reads the two 16-bit values packed in a 32-bit word.
 struct DecodeBf16 {
+  static constexpr bool kBf16 = true;
   __device__ static float lo(uint32_t w) { return __uint_as_float(w << 16); }
   __device__ static float hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 };
 struct DecodeF16 {
+  static constexpr bool kBf16 = false;
   __device__ static float lo(uint32_t w) {
     return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
   }
@@ -60,7 +93,7 @@ struct DecodeF16 {
   }
 };
 
-template <int D, int MODE, class Dec, bool kQuant>
+template <int D, int MODE, class Dec, int kQuant>
 __global__ void __launch_bounds__(kThreads)
     rf_permute_kernel(const RfGeomDev g, const uint4* __restrict__ q, const uint4* __restrict__ k,
                       const uint4* __restrict__ v, uint4* __restrict__ q_out,
@@ -120,7 +153,76 @@ __global__ void __launch_bounds__(kThreads)
       if (rr < nrows) dst[dst_off[rr] + ch] = val[i];
     }
   }
-  if constexpr (kQuant && (MODE == kRearrange || MODE == kQuantOnly)) {
+  if constexpr (kQuant == kQuantMx && (MODE == kRearrange || MODE == kQuantOnly)) {
+    constexpr bool kInBf16 = Dec::kBf16;
+    if (tensor < 2) {
+      // Q and K: every row in groups of 32 columns.  A group is four 16-byte
+      // chunks, held by four consecutive lanes (kChunks is a multiple of 4).
+      uint4* dstx = tensor == 0 ? qo.qx : qo.kx;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int rr = rl + i * kRowLanes;
+        uint32_t mb = __vmaxu2(__vmaxu2(val[i].x & 0x7FFF7FFFu, val[i].y & 0x7FFF7FFFu),
+                               __vmaxu2(val[i].z & 0x7FFF7FFFu, val[i].w & 0x7FFF7FFFu));
+        mb = max(mb & 0xFFFFu, mb >> 16);
+        mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+        mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+        const int e1 = rf_uos_exponent(Dec::lo(mb));
+        const int e[8] = {e1, e1, e1, e1, e1, e1, e1, e1};
+        if (rr < nrows) dstx[dst_off[rr] + ch] = rf_mx_round8<Dec, kInBf16>(val[i], e);
+      }
+    } else {
+      // V: every column in groups of 32 rows counted from the block's first
+      // row (rows past nrows hold zeros and do not raise a group's maximum).
+      // A thread holds kRowsPerGroup rows of each group; the other rows of the
+      // group sit with the other row lanes of the same chunk.
+      constexpr int kRowsPerGroup = 32 / kRowLanes;
+      constexpr int kGroups = RF_BLOCK / 32;
+      constexpr int kWords = D / 2;  // packed 16-bit pairs per row
+      __shared__ uint32_t part[kGroups][kRowLanes][kWords];
+      __shared__ uint32_t gmax[kGroups][kWords];
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
+        uint32_t m4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int j = 0; j < kRowsPerGroup; ++j) {
+          const uint4 x = val[gi * kRowsPerGroup + j];
+          m4[0] = __vmaxu2(m4[0], x.x & 0x7FFF7FFFu);
+          m4[1] = __vmaxu2(m4[1], x.y & 0x7FFF7FFFu);
+          m4[2] = __vmaxu2(m4[2], x.z & 0x7FFF7FFFu);
+          m4[3] = __vmaxu2(m4[3], x.w & 0x7FFF7FFFu);
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) part[gi][rl][ch * 4 + c] = m4[c];
+      }
+      __syncthreads();
+      if (threadIdx.x < kGroups * kWords) {
+        const int gi = threadIdx.x / kWords, wd = threadIdx.x % kWords;
+        uint32_t m = 0u;
+#pragma unroll 4
+        for (int l = 0; l < kRowLanes; ++l) m = __vmaxu2(m, part[gi][l][wd]);
+        gmax[gi][wd] = m;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int gi = 0; gi < kGroups; ++gi) {
+        int e[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t m = gmax[gi][ch * 4 + c];
+          e[2 * c] = rf_uos_exponent(Dec::lo(m));
+          e[2 * c + 1] = rf_uos_exponent(Dec::hi(m));
+        }
+#pragma unroll
+        for (int j = 0; j < kRowsPerGroup; ++j) {
+          const int i = gi * kRowsPerGroup + j;
+          const int rr = rl + i * kRowLanes;
+          if (rr < nrows) qo.vx[dst_off[rr] + ch] = rf_mx_round8<Dec, false>(val[i], e);
+        }
+      }
+    }
+  }
+  if constexpr (kQuant == kQuantE4M3 && (MODE == kRearrange || MODE == kQuantOnly)) {
     if (tensor < 2) {  // uniform over the CTA: Q and K blocks get an E4M3 copy
       // amax over the block's valid rows (rows past nrows hold zeros).  For
       // finite bf16 and fp16 alike |x| orders as the 15-bit magnitude field,
@@ -209,13 +311,20 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
   char* w = static_cast<char*>(ws);
   float* pq = ws ? reinterpret_cast<float*>(w + p->off_pq) : nullptr;
   float* pk = ws ? reinterpret_cast<float*>(w + p->off_pk) : nullptr;
-  const bool quant = (MODE == kRearrange || MODE == kQuantOnly) && p->precision == RF_PRECISION_MIX;
-  QuantOut qout{nullptr, nullptr, nullptr, nullptr};
+  const bool quant_stage = MODE == kRearrange || MODE == kQuantOnly;
+  const bool quant = quant_stage && p->precision == RF_PRECISION_MIX;
+  const bool mx = quant_stage && p->precision == RF_PRECISION_MXFP4;
+  QuantOut qout{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
   if (quant) {
     qout.q8 = reinterpret_cast<uint8_t*>(w + p->off_q8);
     qout.k8 = reinterpret_cast<uint8_t*>(w + p->off_k8);
     qout.q_scale = reinterpret_cast<float*>(w + p->off_qs);
     qout.k_scale = reinterpret_cast<float*>(w + p->off_ks);
+  }
+  if (mx) {
+    qout.qx = reinterpret_cast<uint4*>(w + p->off_qx);
+    qout.kx = reinterpret_cast<uint4*>(w + p->off_kx);
+    qout.vx = reinterpret_cast<uint4*>(w + p->off_vx);
   }
   const uint4* a = static_cast<const uint4*>(q);
   const uint4* b = static_cast<const uint4*>(k);
@@ -228,15 +337,21 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
   if (g.d == 128) {
     if (quant) {
       // precision mix is built for D = 128 only (checked when the plan is made)
-      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, true><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
-      else    rf_permute_kernel<128, MODE, DecodeF16, true><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, kQuantE4M3><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      else    rf_permute_kernel<128, MODE, DecodeF16, kQuantE4M3><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    } else if (mx) {
+      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, kQuantMx><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      else    rf_permute_kernel<128, MODE, DecodeF16, kQuantMx><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
     } else {
-      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
-      else    rf_permute_kernel<128, MODE, DecodeF16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, kQuantNone><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      else    rf_permute_kernel<128, MODE, DecodeF16, kQuantNone><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
     }
+  } else if (mx) {
+    if (bf) rf_permute_kernel<64, MODE, DecodeBf16, kQuantMx><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    else    rf_permute_kernel<64, MODE, DecodeF16, kQuantMx><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
   } else {
-    if (bf) rf_permute_kernel<64, MODE, DecodeBf16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
-    else    rf_permute_kernel<64, MODE, DecodeF16, false><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    if (bf) rf_permute_kernel<64, MODE, DecodeBf16, kQuantNone><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    else    rf_permute_kernel<64, MODE, DecodeF16, kQuantNone><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
   }
   return rf_check_launch("rf_permute_kernel");
 }
@@ -254,10 +369,11 @@ rf_status_t rf_launch_pool(const rf_plan* p, const void* q_r, const void* k_r, v
                            p->g.n1 + p->g.n2);
 }
 
-rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_r, void* ws,
-                               cudaStream_t st) {
-  return launch<kQuantOnly>(p, q_r, k_r, nullptr, nullptr, nullptr, nullptr, ws, st,
-                            p->g.n1 + p->g.n2);
+rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_r, const void* v_r,
+                               void* ws, cudaStream_t st) {
+  // mix quantizes Q and K; mxfp4 also V (the third tensor's heads)
+  const int heads = p->g.n1 + p->g.n2 + (p->precision == RF_PRECISION_MXFP4 ? p->g.n2 : 0);
+  return launch<kQuantOnly>(p, q_r, k_r, v_r, nullptr, nullptr, nullptr, ws, st, heads);
 }
 
 rf_status_t rf_launch_inverse(const rf_plan* p, const void* o_r, void* o, cudaStream_t st) {

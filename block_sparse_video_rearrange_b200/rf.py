@@ -28,7 +28,7 @@ STATUS_NAMES = {0: "RF_OK", 1: "RF_ERR_INVALID_ARG", 2: "RF_ERR_UNSUPPORTED_DEVI
 LAYOUTS = {"BNSD": 0, "TND": 1}
 DTYPES = {"bf16": 0, "fp16": 1}
 ORDERS = {"tile": 0, "frame_pair": 1}   # rf_token_order_t
-PRECISIONS = {"native": 0, "mix": 1, "fp8": 2}   # rf_precision_t
+PRECISIONS = {"native": 0, "mix": 1, "fp8": 2, "mxfp4": 3}   # rf_precision_t
 TORCH_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16}
 POOL_MODES = {"from_ws": 0, "recompute": 1}
 
@@ -36,7 +36,7 @@ EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange"
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
             "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
             "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex", "rf_quantize_qk",
-            "rf_selftest_expired_wait")
+            "rf_selftest_expired_wait", "rf_quantize_mx")
 
 
 class RfError(RuntimeError):
@@ -58,7 +58,8 @@ class PlanInfo(ctypes.Structure):
                 ("n_seqs", ctypes.c_int32), ("n1", ctypes.c_int32), ("n2", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("precision", ctypes.c_int32), ("token_order", ctypes.c_int32),
                 ("ws_q8", ctypes.c_int64), ("ws_k8", ctypes.c_int64),
-                ("ws_q_scale", ctypes.c_int64), ("ws_k_scale", ctypes.c_int64)]
+                ("ws_q_scale", ctypes.c_int64), ("ws_k_scale", ctypes.c_int64),
+                ("ws_q_mx", ctypes.c_int64), ("ws_k_mx", ctypes.c_int64), ("ws_v_mx", ctypes.c_int64)]
 
 
 class PlanOptions(ctypes.Structure):
@@ -84,6 +85,7 @@ def _load() -> ctypes.CDLL:
         "rf_plan_create_ex": [ctypes.POINTER(SeqGeom), i32, i32, i32, i32, i32, i32, i32, ctypes.c_double,
                               i32, i32, ctypes.POINTER(PlanOptions), ctypes.POINTER(vp)],
         "rf_quantize_qk": [vp, vp, vp, vp, sz, vp],
+        "rf_quantize_mx": [vp, vp, vp, vp, vp, sz, vp],
         "rf_selftest_expired_wait": [vp, vp, sz, vp],
         "rf_plan_info": [vp, ctypes.POINTER(PlanInfo)],
         "rf_plan_seq_info": [vp, i32, ctypes.POINTER(SeqInfo)],
@@ -286,6 +288,15 @@ def quantize_qk(plan: Plan, q_r, k_r, ws, stream=None) -> None:
                                _stream(stream)), "rf_quantize_qk")
 
 
+def quantize_mx(plan: Plan, q_r, k_r, v_r, ws, stream=None) -> None:
+    """Precision "mxfp4": MXFP4-rounded copies of rearranged q_r / k_r / v_r into ws."""
+    _expect(q_r, plan.tensor_shape(plan.n1), plan.torch_dtype, "q_r")
+    _expect(k_r, plan.tensor_shape(plan.n2), plan.torch_dtype, "k_r")
+    _expect(v_r, plan.tensor_shape(plan.n2), plan.torch_dtype, "v_r")
+    _check(_lib.rf_quantize_mx(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(v_r), _ptr(ws),
+                               ws.numel() * ws.element_size(), _stream(stream)), "rf_quantize_mx")
+
+
 def inverse_rearrange(plan: Plan, o_r, o, stream=None) -> None:
     """Scatter the output back to the original token order."""
     _expect(o, plan.tensor_shape(plan.n1), plan.torch_dtype, "o")
@@ -362,7 +373,8 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     (prefix_len, t, h, w) per sequence (BNSD: one for the whole batch).
     `order` is the token order of the aligned video ("tile", or "frame_pair"
     for 2x8x8 blocks over frame pairs) and `precision` the kernel precision
-    ("native", or "mix" for E4M3 Q K^T); both are ignored when `plan` is given.
+    ("native", "mix" for E4M3 Q K^T, or "mxfp4" for MXFP4 attention with UOS
+    scaling and PNQ); both are ignored when `plan` is given.
 
     Host inputs run through `pipeline.HostPipeline` (made once per problem
     shape and kept): head chunks whose copies to and from the GPU overlap

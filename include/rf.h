@@ -23,6 +23,9 @@
  *         call (workspace size, then execute), and the constraints list.
  *   [ABS] RainFusion2.0 abstract: block means as representative tokens,
  *         spatiotemporal token permutation, first-frame sink.
+ *   [MX]  "MXAttention: Data-Free Optimal Scaling and Pre-Normalization
+ *         Quantization for MXFP4 Attention", abstract: MXFP4 attention, UOS
+ *         scaling boundary Qmax = 7.25, PNQ.
  *
  * Conventions (all entry points):
  *   - Every pointer named q, k, v, *_r, o, select_idx, select_num or ws is a
@@ -130,6 +133,10 @@ typedef struct {
    * element) and of their scales (fp32 [n1][t_qblk] and [n2][t_qblk], indexed
    * by global query-block number). */
   int64_t ws_q8, ws_k8, ws_q_scale, ws_k_scale;
+  /* RF_PRECISION_MXFP4 only (else -1): byte offsets in ws of the MXFP4-rounded
+   * copies of Q', K' (the inputs' 16-bit type) and V' (always f16), each with
+   * the layout and strides of q_r / k_r / v_r. */
+  int64_t ws_q_mx, ws_k_mx, ws_v_mx;
 } rf_plan_info_t;
 
 /* Per-sequence geometry under suffix promotion ([UG] "Geometry handling"). */
@@ -180,8 +187,33 @@ RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int
  *                        scale_q * scale_k.  Head dim 128 only.
  *   RF_PRECISION_FP8     FP8 for P V as well: not built (RF_ERR_UNSUPPORTED).
  * The pages name the three modes and nothing more; the E4M3 format, the block
- * granularity and the scale rule above are this library's reading. */
-typedef enum { RF_PRECISION_NATIVE = 0, RF_PRECISION_MIX = 1, RF_PRECISION_FP8 = 2 } rf_precision_t;
+ * granularity and the scale rule above are this library's reading.
+ *   RF_PRECISION_MXFP4   MXFP4 attention with Universal Optimal Scaling and
+ *                        Pre-Normalization Quantization ([MX] "MXAttention",
+ *                        abstract).  Every operand of both products is MXFP4:
+ *                        E2M1 elements (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;
+ *                        nearest, ties to the even code, saturating) sharing a
+ *                        power-of-two scale 2^e per group of 32, e the smallest
+ *                        integer with amax <= 7.25 * 2^e (UOS, Qmax = 7.25).
+ *                        Groups run along each product's reduction axis: Q and K
+ *                        rows in groups of 32 columns; V columns and P rows in
+ *                        groups of 32 keys counted from the first row of each
+ *                        key block.  rf_rearrange (or rf_quantize_mx) writes the
+ *                        rounded Q', K', V' into the workspace as exact 16-bit
+ *                        values (V' as f16; values that would round past 65504
+ *                        saturate there).  The softmax takes the exponentials
+ *                        against an integer running maximum (log2 units), rounds
+ *                        each group of 32 of them to MXFP4 the same way, and sums
+ *                        the rounded values into the row sum, so the weights that
+ *                        multiply V' sum to one exactly; P V runs in f16.  The
+ *                        products use the 16-bit tensor cores, on which every
+ *                        MXFP4 value is exact.  Head dim 64 or 128. */
+typedef enum {
+  RF_PRECISION_NATIVE = 0,
+  RF_PRECISION_MIX = 1,
+  RF_PRECISION_FP8 = 2,
+  RF_PRECISION_MXFP4 = 3
+} rf_precision_t;
 /* Options of rf_plan_create_ex; zero-initialised means the defaults. */
 typedef struct {
   int32_t token_order;  /* rf_token_order_t, default RF_ORDER_TILE */
@@ -192,7 +224,7 @@ typedef struct {
  * options == NULL, i.e. tile order and native precision).  Every other
  * argument and error as rf_plan_create; an unknown option value or a non-zero
  * reserved field is RF_ERR_INVALID_ARG; RF_PRECISION_FP8, or RF_PRECISION_MIX
- * with d != 128, is RF_ERR_UNSUPPORTED.  Every later call on the plan
+ * with d != 128, is RF_ERR_UNSUPPORTED.  RF_PRECISION_MXFP4 takes d 64 or 128.  Every later call on the plan
  * (rearrange, pooling, selection, attention, inverse, rf_plan_permutation)
  * follows the plan's options. */
 RF_API rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
@@ -214,7 +246,8 @@ RF_API rf_status_t rf_plan_seq_info(const rf_plan_t* plan, int32_t seq, rf_seq_i
  * ws          : workspace of at least workspace_bytes; receives the fp32
  *               block means of the sparse blocks of Q and K (the fused
  *               pooling of [UG] opening paragraph / [ABS] insight 1) and, with
- *               precision "mix", the E4M3 copies of Q' and K' and their scales.
+ *               precision "mix", the E4M3 copies of Q' and K' and their scales;
+ *               with precision "mxfp4", the MXFP4 copies of Q', K' and V'.
  * Bit-exact copy; deterministic. */
 RF_API rf_status_t rf_rearrange(const rf_plan_t* plan, const void* q, const void* k, const void* v,
                          void* q_r, void* k_r, void* v_r, void* ws, size_t ws_bytes,
@@ -227,6 +260,14 @@ RF_API rf_status_t rf_rearrange(const rf_plan_t* plan, const void* q, const void
  * plan with another precision. */
 RF_API rf_status_t rf_quantize_qk(const rf_plan_t* plan, const void* q_r, const void* k_r, void* ws,
                                   size_t ws_bytes, rf_stream_t stream);
+/* Precision "mxfp4": write the MXFP4-rounded copies of q_r, k_r and v_r into
+ * ws (offsets ws_q_mx, ws_k_mx, ws_v_mx of rf_plan_info_t; the rounding rule
+ * is stated at RF_PRECISION_MXFP4).  rf_rearrange already does this in the same
+ * pass; this call is for callers that produce q_r / k_r / v_r themselves.
+ * Inputs 16-byte aligned, non-null.  RF_ERR_INVALID_ARG for a plan with another
+ * precision. */
+RF_API rf_status_t rf_quantize_mx(const rf_plan_t* plan, const void* q_r, const void* k_r,
+                                  const void* v_r, void* ws, size_t ws_bytes, rf_stream_t stream);
 /* Steps 2-3 ([UG] opening paragraphs and "Configuration"; [API] selectIdx and
  * selectNum constraints).
  * q_r, k_r    : rearranged Q and K (read only when pool_mode == RF_POOL_RECOMPUTE;
@@ -279,6 +320,8 @@ RF_API rf_status_t rf_pool_select_noalloc(const rf_plan_t* plan, const void* q_r
  * Precision "mix": Q K^T reads the E4M3 copies of Q' and K' and their scales in
  *               ws (written by rf_rearrange or rf_quantize_qk on this ws), not
  *               q_r / k_r; P V reads v_r as usual.
+ * Precision "mxfp4": both products read the MXFP4 copies in ws (written by
+ *               rf_rearrange or rf_quantize_mx on this ws), not q_r / k_r / v_r.
  * Deterministic: no split-K, no atomics. */
 RF_API rf_status_t rf_block_sparse_attn(const rf_plan_t* plan, const void* q_r, const void* k_r,
                                  const void* v_r, const int32_t* select_idx,

@@ -116,23 +116,46 @@ def ocp_exponent(amax: float) -> int:
     return e - 2
 
 
+def uos_exponents(amax: np.ndarray) -> np.ndarray:
+    """uos_exponent of every element of amax (int64), with the same exact fix-ups."""
+    a = np.asarray(amax, dtype=np.float64)
+    e = np.zeros(a.shape, dtype=np.int64)
+    nz = a > 0
+    e[nz] = np.ceil(np.log2(a[nz] / QMAX_UOS)).astype(np.int64)
+    up = nz & (a / np.exp2(e) > QMAX_UOS)
+    e[up] += 1
+    down = nz & (a / np.exp2(e - 1) <= QMAX_UOS)
+    e[down] -= 1
+    return e
+
+
+def quantize_groups(x: np.ndarray) -> np.ndarray:
+    """Every row of x is one MX group (at most 32 values): E2M1(x / 2^e) * 2^e with
+    e the row's UOS exponent."""
+    x = np.asarray(x, dtype=np.float64)
+    if x.size == 0:
+        return x.copy()
+    s = np.exp2(uos_exponents(np.max(np.abs(x), axis=-1, keepdims=True)))
+    return e2m1_decode(e2m1_round_codes(x / s)) * s
+
+
 def quantize_group(x: np.ndarray, rule: str = "uos") -> np.ndarray:
     """One MX group (<= 32 values) quantized and dequantized: E2M1(x / 2^e) * 2^e."""
     x = np.asarray(x, dtype=np.float64)
     if x.size == 0:
         return x.copy()
-    amax = float(np.max(np.abs(x)))
-    e = uos_exponent(amax) if rule == "uos" else ocp_exponent(amax)
+    if rule == "uos":
+        return quantize_groups(x[None])[0]
+    e = ocp_exponent(float(np.max(np.abs(x))))
     return e2m1_decode(e2m1_round_codes(x / 2.0 ** e)) * 2.0 ** e
 
 
-def quantize_rows(x: np.ndarray, rule: str = "uos") -> np.ndarray:
+def quantize_rows(x: np.ndarray) -> np.ndarray:
     """R21 for Q and K: every row in groups of 32 along its last axis."""
     x = np.asarray(x, dtype=np.float64)
     out = np.empty_like(x)
-    for r in range(x.shape[0]):
-        for c0 in range(0, x.shape[1], MX_BLOCK):
-            out[r, c0:c0 + MX_BLOCK] = quantize_group(x[r, c0:c0 + MX_BLOCK], rule)
+    for c0 in range(0, x.shape[1], MX_BLOCK):
+        out[:, c0:c0 + MX_BLOCK] = quantize_groups(x[:, c0:c0 + MX_BLOCK])
     return out
 
 
@@ -149,8 +172,7 @@ def quantize_v(v_r: np.ndarray, g: rfo.SeqGeometry) -> np.ndarray:
     out = np.zeros_like(v)
     for b in range(g.n_blocks):
         for grp in key_groups(g, b):
-            for d in range(v.shape[1]):
-                out[grp.start:grp.stop, d] = quantize_group(v[grp.start:grp.stop, d])
+            out[grp.start:grp.stop] = quantize_groups(v[grp.start:grp.stop].T).T
     return out
 
 
@@ -191,8 +213,7 @@ def attend_query_block_mx(qq: np.ndarray, kq: np.ndarray, vq: np.ndarray, g: rfo
         c = 0
         for grp in groups:
             n = len(grp)
-            for i in range(pm.shape[0]):
-                pm[i, c:c + n] = quantize_group(pm[i, c:c + n])
+            pm[:, c:c + n] = quantize_groups(pm[:, c:c + n])
             c += n
     l = pm.sum(axis=1, keepdims=True)
     return (pm @ vq[rows]) / l

@@ -14,6 +14,7 @@ import numpy as np
 import torch
 
 from block_sparse_video_rearrange_b200 import rf, synth
+from oracle import mxattention as mxo
 from oracle import rainfusion as orc
 
 MAX_ABS = 2e-2
@@ -64,7 +65,39 @@ def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "fro
                pooled_q=pq, pooled_k=pk, scale=scale)
     if precision == "mix":
         out.update(mix_buffers(plan, b.ws))
+    if precision == "mxfp4":
+        out.update(mx_buffers(plan, b.ws))
     return out
+
+
+def mx_buffers(plan: rf.Plan, ws: torch.Tensor) -> Dict[str, np.ndarray]:
+    """Host copies (16-bit patterns) of the MXFP4 copies of Q', K' (plan dtype) and V' (f16)."""
+    info = plan.info
+    ws8 = ws.view(torch.uint8)
+    rows, d = int(info.rows_total), plan.d
+
+    def region(off, heads):
+        n = rows * heads * d * 2
+        return ws8[int(off):int(off) + n].cpu().numpy().view(np.uint16).reshape(plan.tensor_shape(heads))
+    return dict(qx=region(info.ws_q_mx, plan.n1), kx=region(info.ws_k_mx, plan.n2),
+                vx=region(info.ws_v_mx, plan.n2))
+
+
+def oracle_mx_inputs(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray]):
+    """float64 Q', K', V' rounded to MXFP4 by the oracle (UOS, groups along each product's
+    reduction axis) from the exact 16-bit rearranged values."""
+    q, k, v = (synth.bits_to_float64(x, w.dtype) for x in rbits)
+    return (mxo.quantize_head(p, q, w.n1, "rows"), mxo.quantize_head(p, k, w.n2, "rows"),
+            mxo.quantize_head(p, v, w.n2, "keys"))
+
+
+def check_mx_quantization(p: orc.Problem, w: synth.Workload, ref, gpu) -> None:
+    """The MXFP4 copies equal the oracle's rounding value for value (Q', K' in the input
+    type, V' in f16; every MXFP4 value of these inputs is exact in either)."""
+    for name, x, dt in (("qx", ref[0], w.dtype), ("kx", ref[1], w.dtype), ("vx", ref[2], "fp16")):
+        got = synth.bits_to_float64(gpu[name], dt)
+        diff = got != x
+        assert not diff.any(), f"{name}: {int(diff.sum())} values differ, e.g. {got[diff][:4]} vs {x[diff][:4]}"
 
 
 def mix_buffers(plan: rf.Plan, ws: torch.Tensor) -> Dict[str, np.ndarray]:
@@ -167,12 +200,14 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
 
 def check_attention(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu,
                     items: Sequence[Tuple[int, int]] | None = None, values=None,
-                    check: bool = True) -> Dict[str, float]:
+                    check: bool = True, oracle_fn=None) -> Dict[str, float]:
     """GPU o_r against the oracle run on the GPU's selectIdx, for (q-block, head) items.
-    `values` replaces the float64 (Q', K', V') decoded from rbits (mix precision);
+    `values` replaces the float64 (Q', K', V') decoded from rbits (mix and mxfp4
+    precisions); `oracle_fn` replaces the oracle attention (mxfp4: the PNQ one);
     with check=False the errors are returned without asserting the bars."""
     qf, kf, vf = values if values is not None else (synth.bits_to_float64(x, w.dtype) for x in rbits)
-    ref = orc.attention(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items)
+    fn = oracle_fn if oracle_fn is not None else orc.attention
+    ref = fn(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items)
     o_r = synth.bits_to_float64(gpu["o_r"], w.dtype)
     table = orc.qblock_table(p)
     num = den = 0.0

@@ -201,3 +201,39 @@ def test_quantize_needs_a_mix_plan():
     fake = ctypes.c_void_p(1 << 20)
     st = rf.lib().rf_quantize_qk(plan.handle, fake, fake, fake, plan.workspace_bytes, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("layout,seqs,n1,n2,d", [("BNSD", [(512, 21, 30, 52)], 40, 40, 128),
+                                                 ("TND", [(256, 13, 32, 48), (384, 21, 24, 40)], 32, 8, 128),
+                                                 ("BNSD", [(128, 9, 16, 32)], 2, 2, 64)])
+def test_mxfp4_precision_workspace_layout(layout, seqs, n1, n2, d):
+    """The MXFP4 copies of Q', K', V' sit after the native workspace, 256-byte aligned,
+    two bytes per element each; the other mix fields stay -1."""
+    nat = rf.Plan(seqs, n1, n2, d, layout, "bf16", 0.8)
+    mx = rf.Plan(seqs, n1, n2, d, layout, "bf16", 0.8, precision="mxfp4")
+    a, b = nat.info, mx.info
+    assert b.precision == 3
+    assert a.ws_q_mx == a.ws_k_mx == a.ws_v_mx == -1
+    assert b.ws_q8 == b.ws_k8 == b.ws_q_scale == b.ws_k_scale == -1
+    rows = int(b.rows_total)
+    assert b.ws_q_mx >= a.workspace_bytes and b.ws_q_mx % 256 == 0
+    assert b.ws_k_mx >= b.ws_q_mx + rows * n1 * d * 2 and b.ws_k_mx % 256 == 0
+    assert b.ws_v_mx >= b.ws_k_mx + rows * n2 * d * 2 and b.ws_v_mx % 256 == 0
+    assert b.workspace_bytes >= b.ws_v_mx + rows * n2 * d * 2
+    for f in ("rows_total", "t_qblk", "max_kv_blocks", "pooled_blocks", "ws_pooled_q", "ws_pooled_k"):
+        assert getattr(a, f) == getattr(b, f), f
+
+
+def test_mxfp4_options_and_quantize_entry_point():
+    assert _create_ex(rf.PlanOptions(0, 3), d=64) == (0, True)
+    assert _create_ex(rf.PlanOptions(1, 3), d=128) == (0, True)
+    fake = ctypes.c_void_p(1 << 20)
+    native = rf.Plan([(128, 9, 16, 32)], 2, 2, 128)
+    mix = rf.Plan([(128, 9, 16, 32)], 2, 2, 128, precision="mix")
+    for plan in (native, mix):   # another precision: rejected before any device work
+        assert rf.lib().rf_quantize_mx(plan.handle, fake, fake, fake, fake, plan.workspace_bytes, None) == 1
+    mx = rf.Plan([(128, 9, 16, 32)], 2, 2, 128, precision="mxfp4")
+    assert rf.lib().rf_quantize_qk(mx.handle, fake, fake, fake, mx.workspace_bytes, None) == 1
+    assert rf.lib().rf_quantize_mx(mx.handle, fake, fake, None, fake, mx.workspace_bytes, None) == 1
+    unaligned = ctypes.c_void_p((1 << 20) + 8)
+    assert rf.lib().rf_quantize_mx(mx.handle, fake, fake, unaligned, fake, mx.workspace_bytes, None) == 1

@@ -6,6 +6,7 @@ import pytest
 import torch
 
 from block_sparse_video_rearrange_b200 import rf, synth
+from oracle import mxattention as mxo
 from oracle import rainfusion as orc
 from tests import parity
 
@@ -284,6 +285,63 @@ def test_mix_quantize_entry_point_equals_fused_quantization():
     torch.cuda.synchronize()
     alone = parity.mix_buffers(plan, b.ws)
     for key in ("q8", "k8", "q_scale", "k_scale"):
+        assert np.array_equal(alone[key], fused[key]), key
+
+
+# ------------------------------------------------------------------------------------------
+# Precision "mxfp4" (MXAttention abstract: MXFP4 attention, UOS scaling with Qmax = 7.25,
+# Pre-Normalization Quantization): the MXFP4 copies of Q', K', V' equal the oracle's rounding
+# value for value; the output against the oracle's PNQ attention on those values within the
+# same bars as the native path.
+# ------------------------------------------------------------------------------------------
+
+MX_SMALL = ["tiny", "ragged_d128", "tnd_gqa_small", "dense", "s_one", "no_prefix", "text_only",
+            "all_promoted"]
+
+
+@pytest.mark.parametrize("name", MX_SMALL)
+def test_mxfp4_small_parity(name):
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision="mxfp4")
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    ref = parity.oracle_mx_inputs(p, w, rbits)
+    parity.check_mx_quantization(p, w, ref, gpu)
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)             # pooling reads the unrounded values
+    parity.check_selection(p, qbars, kbars, gpu)
+    parity.check_attention(p, w, rbits, gpu, values=ref, oracle_fn=mxo.attention_mx)
+
+
+@pytest.mark.parametrize("name,s", [("wan", None), ("tnd_gqa", None), ("minimax", 0.8)])
+def test_mxfp4_full_size_parity(name, s):
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision="mxfp4")
+    rbits = [orc.rearrange(p, x) for x in bits]
+    ref = parity.oracle_mx_inputs(p, w, rbits)
+    parity.check_mx_quantization(p, w, ref, gpu)
+    items = parity.sample_items(p, np.random.default_rng(10), per_kind=3)
+    parity.check_attention(p, w, rbits, gpu, items, values=ref, oracle_fn=mxo.attention_mx)
+    # the quantization error itself, against the unquantized oracle: reported, bounded loosely
+    err = parity.check_attention(p, w, rbits, gpu, items, check=False)
+    assert err["rel_l2"] <= 0.25, err
+
+
+def test_mxfp4_quantize_entry_point_equals_fused_quantization():
+    w = SMALL["ragged_d128"]
+    bits = synth.generate_qkv(w)
+    fused = parity.run_gpu(w, bits, precision="mxfp4")
+    plan = fused["plan"]
+    b = rf.Buffers(plan)
+    q_r, k_r, v_r = (parity.to_device(fused[n], w.dtype) for n in ("q_r", "k_r", "v_r"))
+    rf.quantize_mx(plan, q_r, k_r, v_r, b.ws)
+    torch.cuda.synchronize()
+    alone = parity.mx_buffers(plan, b.ws)
+    for key in ("qx", "kx", "vx"):
         assert np.array_equal(alone[key], fused[key]), key
 
 
