@@ -66,13 +66,15 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     assert b"scratch" in rf.lib().rf_last_error()
 
 
-def test_noalloc_accepts_a_mix_plan_whose_selection_part_fits():
-    """A mix-precision plan's workspace also holds the E4M3 copies of Q' and K';
-    selection needs only the part before them, which is what must fit."""
+@pytest.mark.parametrize("precision", ["mix", "mxfp4"])
+def test_noalloc_accepts_a_quantized_plan_whose_selection_part_fits(precision):
+    """A mix or mxfp4 plan's workspace also holds quantized copies of Q' and K'
+    (and V'); selection needs only the part before them, which is what must fit."""
     w = CASES["wan"]
     bits = synth.generate_qkv(w)
-    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, precision="mix")
-    assert plan.workspace_bytes > 32 << 20 and plan.info.ws_q8 <= 32 << 20
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, precision=precision)
+    first = plan.info.ws_q8 if precision == "mix" else plan.info.ws_q_mx
+    assert plan.workspace_bytes > 32 << 20 and first <= 32 << 20
     q, k, v = (parity.to_device(x, w.dtype) for x in bits)
     b = rf.Buffers(plan)
     rf.rearrange(plan, q, k, v, b.q_r, b.k_r, b.v_r, b.ws)
