@@ -331,6 +331,18 @@ def test_mxfp4_full_size_parity(name, s):
     assert err["rel_l2"] <= 0.25, err
 
 
+def test_mxfp4_with_frame_pair_order():
+    w = SMALL["tnd_gqa_small"]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w, order="frame_pair")
+    gpu = parity.run_gpu(w, bits, order="frame_pair", precision="mxfp4")
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    ref = parity.oracle_mx_inputs(p, w, rbits)
+    parity.check_mx_quantization(p, w, ref, gpu)
+    parity.check_attention(p, w, rbits, gpu, values=ref, oracle_fn=mxo.attention_mx)
+
+
 def test_mxfp4_quantize_entry_point_equals_fused_quantization():
     w = SMALL["ragged_d128"]
     bits = synth.generate_qkv(w)

@@ -53,3 +53,16 @@ def test_pipeline_status_and_default_chunks():
     out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
     pipe(q, k, v, out)
     assert pipe.check_status() == (0, (0, 0))
+
+
+@pytest.mark.parametrize("precision", ["mix", "mxfp4"])
+def test_chunked_host_call_with_a_reduced_precision_equals_one_pass(precision):
+    """Quantization groups never cross heads, so chunking by heads leaves the
+    reduced-precision result unchanged too."""
+    w = CASES["tnd"]
+    bits = synth.generate_qkv(w)
+    ref = parity.run_gpu(w, bits, precision=precision)["o"]
+    q, k, v = _host(bits, w.dtype)
+    out = rf.rainfusion_attention(q, k, v, parity.seqs_of(w), w.sparsity, w.layout, precision=precision,
+                                  chunks=2)
+    assert np.array_equal(out.view(torch.int16).numpy().view(np.uint16), ref)
