@@ -453,7 +453,8 @@ def main():
             line["clocks"] = clocks
         if world == 1 and not args.no_cpu_baseline:
             del q, k, v
-            step_s, oflops, desc, spent = oracle_step_sample(wr, bits)
+            # about 10 s of CPU work: the front steps in full, 300 attention items
+            step_s, oflops, desc, spent = oracle_step_sample(wr, bits, budget_items=300)
             line["cpu_baseline"] = {"value": round(oflops / step_s / 1e12, 6), "unit": "TFLOP/s",
                                     "cores": oracle_threads(), "kind": "oracle",
                                     "sample": desc, "ms_per_step_extrapolated": round(step_s * 1e3, 1),

@@ -4,8 +4,8 @@ TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
 CPU-baseline leg import this module.  It shares no code with the CUDA path.
 
 Source: [MX] "MXAttention: Data-Free Optimal Scaling and Pre-Normalization
-Quantization for MXFP4 Attention", abstract (author page listing, page 5 of
-the pages this path is described on).  The abstract fixes three facts:
+Quantization for MXFP4 Attention", abstract (as listed on an author page).
+The abstract fixes three facts:
   * the attention runs in MXFP4: elements are FP4 values that share a
     power-of-two scale per small block (the OCP microscaling format);
   * Universal Optimal Scaling (UOS) picks each block's power-of-two scale
