@@ -201,6 +201,24 @@ def block_rows(g: SeqGeometry, b: int) -> range:
     return range(g.lp + BLOCK * i, g.lp + BLOCK * (i + 1))
 
 
+def kv_block_rows(g: SeqGeometry, b: int, block_kv: int = BLOCK) -> range:
+    """Rows of key/value block b when key blocks hold block_kv rows ([API] "Formula":
+    blocks of blockShapeX x blockShapeY, reading R23: query blocks of blockShapeX =
+    128 rows as everywhere else, key/value blocks of blockShapeY rows).  The key
+    blocks tile the dense prefix from row 0 (ceiling division, the last may be
+    partial) and the sparse region from row Lp, like block_rows."""
+    n_pb = -(-g.lp // block_kv)
+    if b < n_pb:
+        return range(block_kv * b, min(block_kv * (b + 1), g.lp))
+    i = b - n_pb
+    return range(g.lp + block_kv * i, g.lp + block_kv * (i + 1))
+
+
+def kv_block_count(g: SeqGeometry, block_kv: int = BLOCK) -> int:
+    """Key/value blocks of one sequence: ceil(Lp / block_kv) + S / block_kv."""
+    return -(-g.lp // block_kv) + g.sparse // block_kv
+
+
 def block_means(x_r: np.ndarray, g: SeqGeometry) -> np.ndarray:
     """[nb, D] float64 means of each sparse-region block of one head's rows x_r [L, D]."""
     out = np.zeros((g.nb, x_r.shape[-1]), dtype=np.float64)
@@ -266,7 +284,8 @@ def select_sequence(qbar: np.ndarray, kbar: np.ndarray, g: SeqGeometry) -> Tuple
 # --------------------------------------------------------------------------------------
 
 def attend_query_block(q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray, g: SeqGeometry,
-                       qb: int, key_blocks: Sequence[int], scale: float) -> np.ndarray:
+                       qb: int, key_blocks: Sequence[int], scale: float,
+                       block_kv: int = BLOCK) -> np.ndarray:
     """float64 output rows of query block qb of one head.
 
     The keys are the union of the rows of the listed blocks (-1 entries are
@@ -280,7 +299,7 @@ def attend_query_block(q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray, g: Seq
     for b in key_blocks:
         if b < 0:
             continue
-        krows.extend(block_rows(g, int(b)))
+        krows.extend(kv_block_rows(g, int(b), block_kv))
     q = np.asarray(q_r[qrows.start:qrows.stop], dtype=np.float64)
     k = np.asarray(k_r[krows], dtype=np.float64)
     v = np.asarray(v_r[krows], dtype=np.float64)
@@ -400,7 +419,8 @@ def qblock_table(p: Problem) -> List[Tuple[int, SeqGeometry, int]]:
 
 def attention(p: Problem, q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray,
               idx: np.ndarray, num: np.ndarray, scale: float,
-              items: Sequence[Tuple[int, int]] | None = None) -> Dict[Tuple[int, int], np.ndarray]:
+              items: Sequence[Tuple[int, int]] | None = None,
+              block_kv: int = BLOCK) -> Dict[Tuple[int, int], np.ndarray]:
     """float64 output rows for (global q-block, q-head) items (default: all).
 
     Inputs are float64 arrays in the rearranged layout.  Head n reads key/value
@@ -415,7 +435,7 @@ def attention(p: Problem, q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray,
         s, g, b = table[t]
         row = idx[t, n, :num[t, n]]
         out[(t, n)] = attend_query_block(p.head_rows(q_r, s, n), p.head_rows(k_r, s, n // G),
-                                         p.head_rows(v_r, s, n // G), g, b, row, scale)
+                                         p.head_rows(v_r, s, n // G), g, b, row, scale, block_kv)
     return out
 
 

@@ -134,3 +134,43 @@ def test_kept_flops_dense_closed_form():
     q, k, v = _inputs(p)
     out = rf.run_path(p, q, k, v, 0.25)
     assert rf.kept_flops(p, out["idx"], out["num"]) == 4 * p.d * g.length * g.length * p.n1
+
+
+# --------------------------------------------------------------------------------------
+# Key/value blocks of 64 rows under 128-row query blocks ([API] blockShape X x Y)
+# --------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("geom", [(100, 1, 16, 16), (40, 1, 16, 16), (64, 2, 16, 16), (0, 2, 16, 24),
+                                  (300, 0, 0, 0), (77, 9, 17, 33)])
+def test_kv64_blocks_partition_the_sequence_and_nest_in_128_blocks(geom):
+    g = rf.geometry(*geom, 0.8)
+    n64 = rf.kv_block_count(g, 64)
+    rows = [r for b in range(n64) for r in rf.kv_block_rows(g, b, 64)]
+    assert rows == list(range(g.length))                  # a partition, in order
+    assert n64 == -(-g.lp // 64) + 2 * g.nb
+    assert rf.kv_block_count(g, 128) == g.n_blocks
+    for b in range(g.n_blocks):                           # block_kv = 128 is block_rows itself
+        assert rf.kv_block_rows(g, b, 128) == rf.block_rows(g, b)
+    # every 128-row block is the union of the 64-row blocks inside it
+    for b in range(g.n_blocks):
+        r = rf.block_rows(g, b)
+        inside = [c for c in range(n64) if rf.kv_block_rows(g, c, 64).start in r]
+        assert [x for c in inside for x in rf.kv_block_rows(g, c, 64)] == list(r)
+        assert 1 <= len(inside) <= 2
+
+
+def test_kv64_attention_equals_128_attention_on_the_same_rows():
+    g = rf.geometry(100, 1, 16, 16, 0.5)                 # partial 100-row prefix block
+    rng = np.random.default_rng(21)
+    q, k, v = (rng.standard_normal((g.length, 32)) for _ in range(3))
+    # blocks 0 (prefix, rows 0..99) and 2 (rows 228..355) at 128 rows are 64-row blocks
+    # 0, 1 (rows 0..63, 64..99) and 4, 5 (rows 228..291, 292..355)
+    a = rf.attend_query_block(q, k, v, g, 1, [0, 2], 0.2)
+    b = rf.attend_query_block(q, k, v, g, 1, [0, 1, 4, 5], 0.2, block_kv=64)
+    assert np.max(np.abs(a - b)) < 1e-13
+    # a single 64-row block: exactly the softmax over those rows
+    c = rf.attend_query_block(q, k, v, g, 2, [3], 0.2, block_kv=64)
+    rows = list(range(164, 228))
+    x = 0.2 * q[228:356] @ k[rows].T
+    w = np.exp(x - x.max(axis=1, keepdims=True))
+    assert np.max(np.abs(c - (w / w.sum(axis=1, keepdims=True)) @ v[rows])) < 1e-13
