@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--order", default="tile", choices=["tile", "frame_pair"],
                     help="token order of the aligned video (frame_pair: frames paired into 2x8x8 blocks)")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--block-kv", type=int, default=128, choices=[128, 64],
+                    help="64: time the attention with blockShape 128 x 64 on the 64-row halves of the "
+                         "step's 128-row selection (expanded once on the host after warm-up; same kept FLOPs)")
     ap.add_argument("--chunks", type=int, default=None,
                     help="head chunks of the host pipeline in the e2e measurement (default: the library's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -122,6 +125,40 @@ def kept_flops_from_selection(plan, idx, num):
         q_rows = rows[:nblk][:, None]
         total += int((4 * plan.d * q_rows * kv_rows).sum())
     return total
+
+
+def expand_selection_kv64(plan, idx, num, width):
+    """The 128-row key-block selection rewritten over 64-row key blocks (every
+    selected block becomes the one or two 64-row blocks inside it, in order)."""
+    infos = plan.seq_info_all()
+    T, N, _ = idx.shape
+    out = np.full((T, N, width), -1, dtype=np.int32)
+    cnt = np.zeros((T, N), dtype=np.int32)
+    owner = []                                  # sequence of every global query block
+    for si in infos:
+        owner += [si] * (int(si.n_pb) + int(si.nb))
+    if plan.layout == "BNSD":
+        owner *= plan.batch                     # one geometry for every batch element
+    for t in range(T):
+        si = owner[t]
+        lp, n_pb = int(si.lp), int(si.n_pb)
+        n_pb64 = -(-lp // 64)
+        for n in range(N):
+            row = []
+            for bb in idx[t, n, :num[t, n]]:
+                bb = int(bb)
+                if bb < 0:
+                    continue
+                if bb < n_pb:
+                    row.append(2 * bb)
+                    if 128 * bb + 64 < lp:
+                        row.append(2 * bb + 1)
+                else:
+                    i = bb - n_pb
+                    row += [n_pb64 + 2 * i, n_pb64 + 2 * i + 1]
+            out[t, n, :len(row)] = row
+            cnt[t, n] = len(row)
+    return out, cnt
 
 
 def algorithmic_bytes(plan, elem=2):
@@ -298,6 +335,8 @@ def main():
     scale = 1.0 / math.sqrt(w.d)
     stream = torch.cuda.current_stream(dev)
 
+    kv64 = None   # --block-kv 64: (plan, selectIdx, selectNum, workspace) over 64-row key blocks
+
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
@@ -307,7 +346,10 @@ def main():
         rf.pool_select(plan, None, None, b.select_idx, b.select_num, b.ws)
         if ev is not None:
             ev[2].record(stream)
-        rf.block_sparse_attn(plan, b.q_r, b.k_r, b.v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
+        if kv64 is None:
+            rf.block_sparse_attn(plan, b.q_r, b.k_r, b.v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
+        else:
+            rf.block_sparse_attn(kv64[0], b.q_r, b.k_r, b.v_r, kv64[1], kv64[2], scale, b.o_r, kv64[3])
         if ev is not None:
             ev[3].record(stream)
         rf.inverse_rearrange(plan, b.o_r, b.o)
@@ -317,6 +359,18 @@ def main():
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
+    if args.block_kv == 64:
+        if args.precision != "native":
+            raise SystemExit("--block-kv 64 runs native precision only")
+        p64 = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=args.order,
+                      block_kv=64)
+        i64, n64 = expand_selection_kv64(plan, b.select_idx.cpu().numpy(), b.select_num.cpu().numpy(),
+                                         int(p64.info.max_kv_blocks))
+        kv64 = (p64, torch.from_numpy(i64).to(dev), torch.from_numpy(n64).to(dev),
+                torch.zeros(p64.workspace_bytes, dtype=torch.uint8, device=dev))
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize(dev)
     st, flags = rf.check_device_status(plan, b.ws)
     if st != 0:
         raise RuntimeError(f"device status after warm-up: {st} {flags}")
@@ -344,6 +398,8 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])  # [steps, 4]
     st, flags = rf.check_device_status(plan, b.ws)
+    if st == 0 and kv64 is not None:
+        st, flags = rf.check_device_status(kv64[0], kv64[3])
     if st != 0:
         raise RuntimeError(f"device status after timing: {st} {flags}")
 
@@ -402,7 +458,8 @@ def main():
         inv_ms = float(np.mean(per[:, 3]))
         value = flops_all / (ms_step * 1e-3) / 1e12
         traffic = (profiled_traffic(w.name.split("@")[0], sparsity,
-                                    "" if args.precision == "native" else "/" + args.precision)
+                                    ("" if args.precision == "native" else "/" + args.precision)
+                                    + ("/kv64" if args.block_kv == 64 else ""))
                    if args.order == "tile" and not args.heads else None)
         line = {
             "metric": METRIC,
@@ -421,6 +478,8 @@ def main():
                        "sparsity": sparsity,
                        **({"token_order": args.order} if args.order != "tile" else {}),
                        **({"precision": "mix (E4M3 QK^T, 16-bit PV)"} if args.precision == "mix" else {}),
+                       **({"block_shape": "128 x 64 (attention on the 64-row halves of the step's 128-row "
+                                          "selection, expanded once after warm-up)"} if args.block_kv == 64 else {}),
                        **({"precision": "mxfp4 (UOS Qmax 7.25, PNQ; MXFP4 values on the 16-bit tensor cores)"}
                           if args.precision == "mxfp4" else {}),
                        "global_batch": w.batch * world, "seq_len": int(plan.info.rows_total),

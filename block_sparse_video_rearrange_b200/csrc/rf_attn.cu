@@ -108,7 +108,9 @@ struct __align__(1024) AttnSmem {
   int n_valid;
   float row_m[2][RF_BLOCK];
   float row_l[2][RF_BLOCK];
-  int list[RF_MAX_KV_LIST];
+  // compacted selectIdx row; with 64-row key blocks, pairs (a, b) of one
+  // 128-key tile each (b = -1: none), hence two spare entries
+  int list[RF_MAX_KV_LIST + 2];
   float kscale[kQk8 ? RF_MAX_KV_LIST : 1];  // dequantization scale of K block list[j]
 };
 
@@ -289,6 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const RfSeqDev& s = g.seq[rf_seq_of_qblk(g, tb)];
   const int qb = tb - s.qblk_off;
   const int nblk = s.n_pb + s.nb;
+  const bool kv64 = g.block_kv == 64;                       // blockShape 128 x 64
+  const int nkv = kv64 ? rf_n_pb64(s) + 2 * s.nb : nblk;   // key/value blocks of this sequence
   const int gk = n / (g.n1 / g.n2);  // key/value head
   int q_r0, q_rows;
   rf_block_span(s, qb, q_r0, q_rows);
@@ -342,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int v = row[c];
     sm.list[c] = v;
     if constexpr (kQk8)
-      if (v >= 0 && v < nblk) sm.kscale[c] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
+      if (v >= 0 && v < nkv) sm.kscale[c] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
   }
   __syncthreads();
   if (warp == 0) {
@@ -357,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int v = c < num ? sm.list[c] : -1;
       float ks = 0.f;
       if constexpr (kQk8) ks = c < num ? sm.kscale[c] : 0.f;
-      const bool ok = c < num && v >= 0 && v < nblk;
+      const bool ok = c < num && v >= 0 && v < nkv;
       if (c < num && v != -1 && !ok) ++bad;
       const uint32_t ball = __ballot_sync(0xffffffffu, ok);
       if (ok) {
@@ -367,11 +371,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       cnt += __popc(ball);
     }
     bad = __reduce_add_sync(0xffffffffu, bad);
+    int units = cnt;  // tiles of 128 keys
+    if (kv64) {
+      // Pair the 64-row blocks into 128-key tiles: list[2t], list[2t + 1].
+      // Valid key rows must run from the tile's first row, so the partial
+      // prefix block may be the second of a pair but not the first: if it
+      // falls on an even position it stays alone (the entries after it move
+      // up by one) -- it can occur at most once.  An odd count leaves the
+      // last tile's second half empty.
+      const int part_blk = (s.Lp & 63) ? rf_n_pb64(s) - 1 : -1;
+      int qpos = -1;
+      for (int c0 = 0; c0 < cnt; c0 += 32) {
+        const int c = c0 + lane;
+        const uint32_t hit = __ballot_sync(0xffffffffu, c < cnt && sm.list[c] == part_blk);
+        if (hit && qpos < 0) qpos = c0 + __ffs(hit) - 1;
+      }
+      const int shift = (qpos >= 0 && (qpos & 1) == 0) ? 1 : 0;
+      if (shift) {
+        // entries qpos + 1 .. cnt - 1 move to +1, 32 at a time from the end:
+        // a chunk reads everything before it writes
+        for (int hi = cnt; hi > qpos + 1; hi -= 32) {
+          const int c = hi - 1 - lane;
+          const bool act = c > qpos;
+          const int v = act ? sm.list[c] : 0;
+          __syncwarp();
+          if (act) sm.list[c + 1] = v;
+          __syncwarp();
+        }
+        if (lane == 0) sm.list[qpos + 1] = -1;
+      }
+      const int tot = cnt + shift;
+      if (lane == 0 && (tot & 1)) sm.list[tot] = -1;
+      units = (tot + 1) >> 1;
+    }
     if (lane == 0) {
       // A wait that already expired in this workspace (this launch or an
       // earlier one not yet cleared by rf_check_device_status) stops all work.
       const bool stopped = *reinterpret_cast<volatile uint32_t*>(a.status + RF_STATUS_TIMEOUT) != 0;
-      sm.n_valid = stopped ? 0 : cnt;
+      sm.n_valid = stopped ? 0 : units;
       if (bad) atomicAdd(a.status + RF_STATUS_BAD_INDEX, (uint32_t)bad);
     }
   }
@@ -408,13 +445,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         record_timeout(abort, a.status, is_k ? 0 : 1);
         break;
       }
-      int r0, nr;
-      rf_block_span(s, sm.list[j], r0, nr);
-      coords(g.n2, gk, r0, c1, c2);
       const uint32_t bar = rf_smem_u32(&full[st]);
       mbar_arrive_expect_tx(bar, tile_bytes);
-      for (int x = 0; x < boxes; ++x)
-        tma_load_3d(rf_smem_u32(tiles + st * tile_bytes + x * kBoxBytes), map, bar, x * 64, c1, c2);
+      if (!kv64) {
+        int r0, nr;
+        rf_block_span(s, sm.list[j], r0, nr);
+        coords(g.n2, gk, r0, c1, c2);
+        for (int x = 0; x < boxes; ++x)
+          tma_load_3d(rf_smem_u32(tiles + st * tile_bytes + x * kBoxBytes), map, bar, x * 64, c1, c2);
+      } else {
+        // two 64-row boxes per column box (the maps have 64-row boxes): block a
+        // into tile rows 0..63, block b into rows 64..127; an empty second
+        // half loads block a again, so that its (masked) keys stay finite
+        const int blk_a = sm.list[2 * j];
+        const int blk_b = sm.list[2 * j + 1] >= 0 ? sm.list[2 * j + 1] : blk_a;
+        int ra, rb, na, nb2, c1b, c2b;
+        rf_kv64_span(s, blk_a, ra, na);
+        rf_kv64_span(s, blk_b, rb, nb2);
+        coords(g.n2, gk, ra, c1, c2);
+        coords(g.n2, gk, rb, c1b, c2b);
+        for (int x = 0; x < boxes; ++x) {
+          const uint32_t dst = rf_smem_u32(tiles + st * tile_bytes + x * kBoxBytes);
+          tma_load_3d(dst, map, bar, x * 64, c1, c2);
+          tma_load_3d(dst + 64 * 128, map, bar, x * 64, c1b, c2b);
+        }
+      }
       issued = j + 1;
     }
     if (*abort) {
@@ -526,7 +581,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int j = 2 * i + wg;
       if (!warp_wait(rf_smem_u32(&sm.bar_s_full[wg]), i & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      const int vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;  // uniform over the CTA
+      int vr;  // valid key rows of the tile, from its first row; uniform over the CTA
+      if (kv64) {
+        int r0, na, nb2 = 0;
+        rf_kv64_span(s, sm.list[2 * j], r0, na);
+        if (sm.list[2 * j + 1] >= 0) rf_kv64_span(s, sm.list[2 * j + 1], r0, nb2);
+        vr = na + nb2;
+      } else {
+        vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;
+      }
       const float sl2 = kQk8 ? sl2_q * sm.kscale[j] : sl2_q;
       const uint32_t scol = lane_base + s_col;
       uint32_t sr[128];
@@ -688,9 +751,11 @@ EncodeTiledFn encode_fn() {
 enum MapElem { kElemPlan = 0, kElemByte = 1, kElemF16 = 2 };
 
 // Tensor map over [rows, heads, D] (TND) or [B*heads, rows, D] (BNSD) with a
-// 128-row x 128-byte box and 128-byte swizzle: 64 columns of a 16-bit tensor,
-// or 128 columns of a one-byte (E4M3) tensor.
-rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int heads, MapElem elem) {
+// box_rows x 128-byte box and 128-byte swizzle: 64 columns of a 16-bit tensor,
+// or 128 columns of a one-byte (E4M3) tensor.  box_rows is 128, or 64 for the
+// key/value maps of blockShape 128 x 64.
+rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int heads, MapElem elem,
+                     int box_rows = RF_BLOCK) {
   const bool one_byte = elem == kElemByte;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return rf_fail(RF_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
@@ -704,11 +769,11 @@ rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int hea
     const cuuint64_t L = (cuuint64_t)g.seq[0].L;
     dims[0] = d; dims[1] = L; dims[2] = (cuuint64_t)p->batch * heads;
     strides[0] = d * esz; strides[1] = L * d * esz;
-    box[0] = box_cols; box[1] = RF_BLOCK; box[2] = 1;
+    box[0] = box_cols; box[1] = (cuuint32_t)box_rows; box[2] = 1;
   } else {
     dims[0] = d; dims[1] = (cuuint64_t)heads; dims[2] = (cuuint64_t)p->rows_total;
     strides[0] = d * esz; strides[1] = (cuuint64_t)heads * d * esz;
-    box[0] = box_cols; box[1] = 1; box[2] = RF_BLOCK;
+    box[0] = box_cols; box[1] = 1; box[2] = (cuuint32_t)box_rows;
   }
   const CUtensorMapDataType dt = one_byte ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : (p->dtype == RF_BF16 && elem == kElemPlan) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -767,8 +832,9 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   const void* vsrc = mx ? static_cast<const void*>(w + p->off_vx) : v_r;
   const MapElem qk_elem = mix ? kElemByte : kElemPlan;
   if ((s = make_map(&mq, p, qsrc, g.n1, qk_elem)) != RF_OK) return s;
-  if ((s = make_map(&mk, p, ksrc, g.n2, qk_elem)) != RF_OK) return s;
-  if ((s = make_map(&mv, p, vsrc, g.n2, mx ? kElemF16 : kElemPlan)) != RF_OK) return s;
+  const int kv_box = g.block_kv == 64 ? 64 : RF_BLOCK;
+  if ((s = make_map(&mk, p, ksrc, g.n2, qk_elem, kv_box)) != RF_OK) return s;
+  if ((s = make_map(&mv, p, vsrc, g.n2, mx ? kElemF16 : kElemPlan, kv_box)) != RF_OK) return s;
   AttnArgs args;
   args.g = g;
   args.sel_idx = sel_idx;

@@ -42,6 +42,20 @@ __host__ __device__ __forceinline__ void rf_block_span(const RfSeqDev& s, int b,
   }
 }
 
+// Key/value blocks of 64 rows (blockShape 128 x 64): ceil(Lp / 64) prefix
+// blocks from row 0 (the last may be partial), then 2 * nb blocks from row Lp.
+__host__ __device__ __forceinline__ int rf_n_pb64(const RfSeqDev& s) { return (s.Lp + 63) >> 6; }
+__host__ __device__ __forceinline__ void rf_kv64_span(const RfSeqDev& s, int b, int& r0, int& nrows) {
+  const int n_pb = rf_n_pb64(s);
+  if (b < n_pb) {
+    r0 = 64 * b;
+    nrows = s.Lp - r0 < 64 ? s.Lp - r0 : 64;
+  } else {
+    r0 = s.Lp + 64 * (b - n_pb);
+    nrows = 64;
+  }
+}
+
 // Original (input-order) row of rearranged row r of one sequence.
 //   rearranged = [text | promoted | sparse]; the video part follows V', the
 //   video tokens in tile order: aligned tokens by (frame, tile row, tile col,

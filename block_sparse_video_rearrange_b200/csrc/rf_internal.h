@@ -37,6 +37,7 @@ struct RfGeomDev {
   int n1, n2, d;
   int t_qblk;
   int max_kv;
+  int block_kv;         // key/value block rows: 128, or 64 ([API] blockShape 128 x 64)
   int pooled_total;     // sum of nb over instances
   int max_nb;
   RfSeqDev seq[RF_MAX_SEQS];

@@ -141,8 +141,10 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
     return rf_fail(RF_ERR_INVALID_ARG, "sparsity must be finite and in [0, 1]");
   if (block_q <= 0 || block_kv <= 0)
     return rf_fail(RF_ERR_INVALID_ARG, "blockShape entries must be > 0");
-  if (block_q != RF_BLOCK || block_kv != RF_BLOCK)
-    return rf_fail(RF_ERR_UNSUPPORTED, "only 128 x 128 blocks are built");
+  if (block_q != RF_BLOCK || (block_kv != RF_BLOCK && block_kv != 64))
+    return rf_fail(RF_ERR_UNSUPPORTED, "blockShape must be 128 x 128 or 128 x 64");
+  if (block_kv != RF_BLOCK && opt.precision != RF_PRECISION_NATIVE)
+    return rf_fail(RF_ERR_UNSUPPORTED, "blockShape 128 x 64 is built for native precision only");
   if (n1 <= 0 || n2 <= 0 || n1 % n2 != 0)
     return rf_fail(RF_ERR_INVALID_ARG, "heads: need n1 > 0, n2 > 0 and n1 % n2 == 0");
   if (d <= 0) return rf_fail(RF_ERR_INVALID_ARG, "head dim must be > 0");
@@ -192,7 +194,9 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
     s.score_off = scores;
     g.seq[i] = s;
     int nblk = s.n_pb + s.nb;
-    if (nblk > max_kv) max_kv = nblk;
+    // selectIdx rows count key/value blocks of block_kv rows
+    const int nkv = block_kv == RF_BLOCK ? nblk : rf_n_pb64(s) + 2 * s.nb;
+    if (nkv > max_kv) max_kv = nkv;
     if (s.nb > max_nb) max_nb = s.nb;
     rows += s.L;
     qblk += nblk;
@@ -217,7 +221,7 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   }
   if (max_kv > RF_MAX_KV_LIST || max_nb > RF_MAX_NB) {
     delete p;
-    return rf_fail(RF_ERR_UNSUPPORTED, "a sequence has more than 2048 blocks");
+    return rf_fail(RF_ERR_UNSUPPORTED, "a sequence has more than 2048 blocks (query or key/value)");
   }
   if (qblk * n1 > (1ll << 31) - 1) {
     delete p;
@@ -225,6 +229,7 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   }
   g.t_qblk = (int)qblk;
   g.max_kv = max_kv;
+  g.block_kv = block_kv;
   g.pooled_total = (int)pooled;
   g.max_nb = max_nb;
   p->rows_total = layout == RF_LAYOUT_BNSD ? (int64_t)batch * g.seq[0].L : rows;
@@ -381,6 +386,9 @@ rf_status_t rf_pool_select(const rf_plan_t* p, const void* q_r, const void* k_r,
   if (!select_idx || !select_num) return rf_fail(RF_ERR_INVALID_ARG, "null selectIdx/selectNum");
   if (pool_mode != RF_POOL_FROM_WS && pool_mode != RF_POOL_RECOMPUTE)
     return rf_fail(RF_ERR_INVALID_ARG, "bad pool mode");
+  if (p->g.block_kv != RF_BLOCK)
+    return rf_fail(RF_ERR_UNSUPPORTED, "selection ranks 128-row key blocks only; with blockShape 128 x 64 "
+                                       "the caller supplies selectIdx");
   if (pool_mode == RF_POOL_RECOMPUTE &&
       (!q_r || !k_r || !aligned16(q_r) || !aligned16(k_r)))
     return rf_fail(RF_ERR_INVALID_ARG, "recompute needs 16-byte aligned q_r and k_r");
@@ -433,6 +441,9 @@ rf_status_t rf_inverse_rearrange(const rf_plan_t* p, const void* o_r, void* o, r
 rf_status_t rf_forward(const rf_plan_t* p, const void* q, const void* k, const void* v, void* q_r,
                        void* k_r, void* v_r, int32_t* select_idx, int32_t* select_num, float scale,
                        void* o_r, void* o, void* ws, size_t ws_bytes, rf_stream_t stream) {
+  // Refuse before enqueuing anything when a later step would refuse.
+  if (p && p->g.block_kv != RF_BLOCK)
+    return rf_fail(RF_ERR_UNSUPPORTED, "rf_forward needs 128 x 128 blocks (selection ranks 128-row key blocks)");
   rf_status_t st = rf_rearrange(p, q, k, v, q_r, k_r, v_r, ws, ws_bytes, stream);
   if (st != RF_OK) return st;
   st = rf_pool_select(p, nullptr, nullptr, select_idx, select_num, ws, ws_bytes, RF_POOL_FROM_WS,

@@ -164,8 +164,15 @@ typedef struct rf_plan rf_plan_t;
  *   n1, n2      : query and key/value heads, n1 % n2 == 0 ([API] GQA constraint).
  *   d           : head dim, 64 or 128 (others: RF_ERR_UNSUPPORTED).
  *   sparsity    : finite, in [0, 1] ([UG] "Configuration"); 0 keeps every block.
- *   block_q, block_kv : [API] blockShape; must be > 0; only 128 x 128 is built
- *                 (others: RF_ERR_UNSUPPORTED).
+ *   block_q, block_kv : [API] blockShape; must be > 0.  Built: 128 x 128, and
+ *                 128 x 64 (query blocks of 128 rows, key/value blocks of 64
+ *                 rows: ceil(lp / 64) prefix key blocks from row 0, the last
+ *                 possibly partial, then 2 * nb from row lp; native precision
+ *                 only).  With 128 x 64, selectIdx entries and max_kv_blocks
+ *                 count 64-row key blocks, the selection step (which ranks
+ *                 128-row blocks) and rf_forward return RF_ERR_UNSUPPORTED, and
+ *                 rf_block_sparse_attn takes a caller-made selectIdx.  Others:
+ *                 RF_ERR_UNSUPPORTED.
  *   out         : receives the plan; free with rf_plan_destroy.
  * Errors: RF_ERR_INVALID_ARG for a broken constraint (out untouched). */
 RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
@@ -313,7 +320,11 @@ RF_API rf_status_t rf_pool_select_noalloc(const rf_plan_t* plan, const void* q_r
  * select_idx, select_num : as written by rf_pool_select (any valid selection is
  *               accepted: entries in [0, n_pb + nb) of the row's sequence; the
  *               first select_num entries are used; out-of-range entries are
- *               skipped and flagged in ws).
+ *               skipped and flagged in ws).  With blockShape 128 x 64 the
+ *               entries are 64-row key blocks in [0, ceil(lp / 64) + 2 * nb);
+ *               the kernel pairs consecutive entries into 128-key tiles (the
+ *               partial last prefix block never opens a pair), so listing both
+ *               halves of a 128-row block gives that block's tile.
  * scale       : > 0 and finite (typically 1/sqrt(D)).
  * inner_precise : 0 = fp32 softmax ([API]: 1 = fp16 softmax is not allowed with
  *               bf16 and is not built here: RF_ERR_UNSUPPORTED).

@@ -133,6 +133,27 @@ def mix_reference_inputs(p: orc.Problem, w: synth.Workload, gpu, rbits: Sequence
     return qf, kf, synth.bits_to_float64(rbits[2], w.dtype)
 
 
+def expand_to_kv64(p: orc.Problem, idx: np.ndarray, num: np.ndarray, width: int):
+    """A 128-row key-block selection rewritten over 64-row key blocks: every
+    selected block becomes the one or two 64-row blocks inside it (in order)."""
+    table = orc.qblock_table(p)
+    T, N, _ = idx.shape
+    out = np.full((T, N, width), -1, dtype=np.int32)
+    cnt = np.zeros((T, N), dtype=np.int32)
+    inside = {}
+    for t in range(T):
+        s, g, _ = table[t]
+        if g not in inside:
+            n64 = orc.kv_block_count(g, 64)
+            starts = {orc.kv_block_rows(g, c, 64).start: c for c in range(n64)}
+            inside[g] = [[starts[r] for r in orc.block_rows(g, b) if r in starts] for b in range(g.n_blocks)]
+        for n in range(N):
+            row = [c for b in idx[t, n, :num[t, n]] if b >= 0 for c in inside[g][int(b)]]
+            out[t, n, :len(row)] = row
+            cnt[t, n] = len(row)
+    return out, cnt
+
+
 def oracle_rearranged_bits(p: orc.Problem, bits: np.ndarray) -> np.ndarray:
     """The oracle's permutation applied to raw 16-bit patterns (exact)."""
     return orc.rearrange(p, bits)
@@ -200,14 +221,15 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
 
 def check_attention(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu,
                     items: Sequence[Tuple[int, int]] | None = None, values=None,
-                    check: bool = True, oracle_fn=None) -> Dict[str, float]:
+                    check: bool = True, oracle_fn=None, block_kv: int = 128) -> Dict[str, float]:
     """GPU o_r against the oracle run on the GPU's selectIdx, for (q-block, head) items.
     `values` replaces the float64 (Q', K', V') decoded from rbits (mix and mxfp4
     precisions); `oracle_fn` replaces the oracle attention (mxfp4: the PNQ one);
     with check=False the errors are returned without asserting the bars."""
     qf, kf, vf = values if values is not None else (synth.bits_to_float64(x, w.dtype) for x in rbits)
     fn = oracle_fn if oracle_fn is not None else orc.attention
-    ref = fn(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items)
+    extra = {} if block_kv == 128 else {"block_kv": block_kv}
+    ref = fn(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items, **extra)
     o_r = synth.bits_to_float64(gpu["o_r"], w.dtype)
     table = orc.qblock_table(p)
     num = den = 0.0

@@ -237,3 +237,29 @@ def test_mxfp4_options_and_quantize_entry_point():
     assert rf.lib().rf_quantize_mx(mx.handle, fake, fake, None, fake, mx.workspace_bytes, None) == 1
     unaligned = ctypes.c_void_p((1 << 20) + 8)
     assert rf.lib().rf_quantize_mx(mx.handle, fake, fake, unaligned, fake, mx.workspace_bytes, None) == 1
+
+
+def test_block_shape_128_by_64_plan():
+    """blockShape 128 x 64: key blocks of 64 rows (native precision only); the
+    selectIdx width counts them; selection and the whole-path call refuse."""
+    seqs = [(100, 9, 16, 32)]        # Lp = 100: two 64-row prefix blocks, the second partial
+    p128 = rf.Plan(seqs, 2, 2, 128)
+    p64 = rf.Plan(seqs, 2, 2, 128, block_kv=64)
+    g = orc.geometry(100, 9, 16, 32, 0.8)
+    assert int(p128.info.max_kv_blocks) == g.n_blocks
+    assert int(p64.info.max_kv_blocks) == orc.kv_block_count(g, 64) == 2 + 2 * g.nb
+    assert int(p64.info.t_qblk) == int(p128.info.t_qblk)          # query blocks stay 128 rows
+    assert p64.select_shapes()[0][2] == int(p64.info.max_kv_blocks)
+    for bq, bkv in ((64, 128), (128, 32), (64, 64), (256, 128)):
+        with pytest.raises(rf.RfError) as e:
+            rf.Plan(seqs, 2, 2, 128, block_q=bq, block_kv=bkv)
+        assert e.value.status == 6
+    for precision in ("mix", "mxfp4"):
+        with pytest.raises(rf.RfError) as e:
+            rf.Plan(seqs, 2, 2, 128, block_kv=64, precision=precision)
+        assert e.value.status == 6
+    fake = ctypes.c_void_p(1 << 20)
+    lib = rf.lib()
+    assert lib.rf_pool_select(p64.handle, fake, fake, fake, fake, fake, p64.workspace_bytes, 0, None) == 6
+    assert lib.rf_forward(p64.handle, fake, fake, fake, fake, fake, fake, fake, fake, ctypes.c_float(0.1),
+                          fake, fake, fake, p64.workspace_bytes, None) == 6

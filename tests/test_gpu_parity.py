@@ -394,3 +394,93 @@ def test_exp2_polynomial_against_mufu_and_exact():
     xi = torch.arange(-120, 9, dtype=torch.float32).cuda()
     yi, _ = rf.selftest_exp2(xi)
     assert torch.equal(yi.double(), torch.exp2(xi.double()))
+
+
+# ------------------------------------------------------------------------------------------
+# blockShape 128 x 64 (aclnnRainFusionAttention "Formula": blocks of blockShapeX x
+# blockShapeY): key/value blocks of 64 rows, paired by the kernel into 128-key tiles.
+# ------------------------------------------------------------------------------------------
+
+KV64 = ["ragged_d128", "tnd_gqa_small", "tiny", "text_only", "all_promoted", "no_prefix"]
+
+
+def _kv64_run(w, q_r, k_r, v_r, idx, num, scale):
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch,
+                   block_kv=64)
+    b = rf.Buffers(plan)
+    assert tuple(b.select_idx.shape) == idx.shape
+    b.select_idx.copy_(torch.from_numpy(idx))
+    b.select_num.copy_(torch.from_numpy(num))
+    rf.block_sparse_attn(plan, q_r, k_r, v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
+    st, flags = rf.check_device_status(plan, b.ws)
+    assert st == 0, (st, flags)
+    return parity.to_bits(b.o_r)
+
+
+@pytest.mark.parametrize("name", KV64)
+def test_kv64_halves_of_a_128_selection_give_the_128_result_bit_for_bit(name):
+    """Listing both 64-row halves of every selected 128-row block rebuilds the same
+    128-key tiles (the partial prefix block alone when it is one half), so the
+    output equals the 128 x 128 path's bit for bit -- except in a sequence whose
+    dense prefix ends 64 rows into a 128-row block: there the last prefix block
+    is a whole 64-row block, pairs with the next selected block, and the tiles
+    (hence the summation order) differ; those rows are held to the parity bar."""
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits)
+    plan64 = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch,
+                     block_kv=64)
+    idx64, num64 = parity.expand_to_kv64(p, gpu["idx"], gpu["num"], int(plan64.info.max_kv_blocks))
+    q_r, k_r, v_r = (parity.to_device(gpu[n], w.dtype) for n in ("q_r", "k_r", "v_r"))
+    o64 = _kv64_run(w, q_r, k_r, v_r, idx64, num64, gpu["scale"])
+    a64 = synth.bits_to_float64(o64, w.dtype)
+    a128 = synth.bits_to_float64(gpu["o_r"], w.dtype)
+    regrouped = 0
+    for s_id, g in p.sequences():
+        for n in range(w.n1):
+            x, y = p.head_rows(a64, s_id, n), p.head_rows(a128, s_id, n)
+            if g.lp % 128 == 64:
+                regrouped += 1
+                assert np.max(np.abs(x - y)) <= parity.MAX_ABS
+            else:
+                assert np.array_equal(x, y), (s_id, n)
+    assert regrouped < len(p.sequences()) * w.n1      # most rows are checked bit for bit
+
+
+@pytest.mark.parametrize("name", KV64)
+def test_kv64_random_selection_against_the_oracle(name):
+    """Arbitrary ascending 64-row selections (odd counts, gaps, the partial prefix
+    block at even and odd positions, -1 slots) against the oracle with 64-row key blocks."""
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits)
+    table = orc.qblock_table(p)
+    plan64 = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch,
+                     block_kv=64)
+    T, N = gpu["num"].shape
+    M = int(plan64.info.max_kv_blocks)
+    rng = np.random.default_rng(5)
+    idx = np.full((T, N, M), -1, dtype=np.int32)
+    num = np.zeros((T, N), dtype=np.int32)
+    clean = np.full((T, N, M), -1, dtype=np.int32)
+    clean_num = np.zeros((T, N), dtype=np.int32)
+    for t in range(T):
+        s, g, _ = table[t]
+        n64 = orc.kv_block_count(g, 64)
+        for n in range(N):
+            size = int(rng.integers(1, n64 + 1))
+            chosen = sorted(rng.choice(n64, size=size, replace=False).tolist())
+            row = list(chosen)
+            if (t + n) % 4 == 1 and len(row) < M:
+                row.insert(int(rng.integers(0, len(row) + 1)), -1)   # an unused slot
+            idx[t, n, :len(row)] = row
+            num[t, n] = len(row)
+            clean[t, n, :len(chosen)] = chosen
+            clean_num[t, n] = len(chosen)
+    q_r, k_r, v_r = (parity.to_device(gpu[n], w.dtype) for n in ("q_r", "k_r", "v_r"))
+    o64 = _kv64_run(w, q_r, k_r, v_r, idx, num, gpu["scale"])
+    rbits = [orc.rearrange(p, x) for x in bits]
+    got = dict(idx=clean, num=clean_num, scale=gpu["scale"], o_r=o64)
+    parity.check_attention(p, w, rbits, got, block_kv=64)
