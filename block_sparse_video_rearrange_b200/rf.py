@@ -143,6 +143,7 @@ class Plan:
                "rf_plan_create_ex")
         self.order = order
         self.precision = precision
+        self.block_q, self.block_kv = int(block_q), int(block_kv)
         self._h = handle
         self._lib = _lib  # kept so that destruction at interpreter exit still finds it
         self.layout, self.dtype, self.sparsity, self.batch = layout, dtype, float(sparsity), batch
