@@ -226,3 +226,18 @@ def test_vectorized_exponents_equal_the_scalar_rule():
     a = np.concatenate([np.exp(rng.uniform(-80, 80, 3000)), 7.25 * 2.0 ** np.arange(-40, 40),
                         np.nextafter(7.25 * 2.0 ** np.arange(-40, 40), np.inf), [0.0]])
     assert list(mx.uos_exponents(a)) == [mx.uos_exponent(float(x)) for x in a]
+
+
+def test_vectorized_rows_and_columns_equal_group_by_group_rounding():
+    g = rfo.geometry(77, 2, 17, 33, 0.8)          # partial prefix block, ragged grid
+    rng = np.random.default_rng(14)
+    x = rng.standard_normal((g.length, 64)) * np.exp(rng.uniform(-3, 3, (g.length, 1)))
+    rows = mx.quantize_rows(x)
+    for r in range(0, g.length, 37):
+        for c0 in (0, 32):
+            assert np.array_equal(rows[r, c0:c0 + 32], mx.quantize_group(x[r, c0:c0 + 32]))
+    cols = mx.quantize_v(x, g)
+    for b in range(g.n_blocks):
+        for grp in mx.key_groups(g, b):
+            for d in (0, 5, 63):
+                assert np.array_equal(cols[grp.start:grp.stop, d], mx.quantize_group(x[grp.start:grp.stop, d]))
