@@ -407,7 +407,8 @@ def main():
     # runs head chunks whose copies overlap the compute); copies inside the timed region,
     # the result back on the host at the end of every step.
     e2e = None
-    if args.e2e_steps > 0:
+    # the public call has no 128 x 64 selection, so --block-kv 64 times the kernels only
+    if args.e2e_steps > 0 and kv64 is None:
         out_host = None
 
         def e2e_step():
