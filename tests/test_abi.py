@@ -263,3 +263,26 @@ def test_block_shape_128_by_64_plan():
     assert lib.rf_pool_select(p64.handle, fake, fake, fake, fake, fake, p64.workspace_bytes, 0, None) == 6
     assert lib.rf_forward(p64.handle, fake, fake, fake, fake, fake, fake, fake, fake, ctypes.c_float(0.1),
                           fake, fake, fake, p64.workspace_bytes, None) == 6
+
+
+# ---------------- randomized geometry sweep (host-side index math) ----------------
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=60, deadline=None)
+@given(p=st.integers(0, 400), t=st.integers(0, 7), h=st.integers(0, 40), w=st.integers(0, 40),
+       order=st.sampled_from(["tile", "frame_pair"]))
+def test_random_geometries_match_the_oracle(p, t, h, w, order):
+    """For random (prefix, t, h, w) and both token orders: the plan's sizes, the 64-row
+    key-block count and the row mapping the kernels execute all equal the oracle's."""
+    if p + t * h * w == 0:
+        return
+    g = orc.geometry(p, t, h, w, 0.8, order)
+    plan = rf.Plan([(p, t, h, w)], 1, 1, 64, order=order)
+    si = plan.seq_info[0]
+    assert (int(si.length), int(si.lp), int(si.sparse), int(si.n_pb), int(si.nb), int(si.ns), int(si.k),
+            bool(si.dense)) == (g.length, g.lp, g.sparse, g.n_pb, g.nb, g.ns, g.k, g.dense)
+    assert np.array_equal(plan.permutation(0), orc.permutation(g))
+    p64 = rf.Plan([(p, t, h, w)], 1, 1, 64, order=order, block_kv=64)
+    assert int(p64.info.max_kv_blocks) == orc.kv_block_count(g, 64)
