@@ -263,6 +263,7 @@ def test_block_shape_128_by_64_plan():
     assert lib.rf_pool_select(p64.handle, fake, fake, fake, fake, fake, p64.workspace_bytes, 0, None) == 6
     assert lib.rf_forward(p64.handle, fake, fake, fake, fake, fake, fake, fake, fake, ctypes.c_float(0.1),
                           fake, fake, fake, p64.workspace_bytes, None) == 6
+    assert lib.rf_pool_select_noalloc(p64.handle, fake, fake, fake, fake, None) == 6
 
 
 # ---------------- randomized geometry sweep (host-side index math) ----------------
