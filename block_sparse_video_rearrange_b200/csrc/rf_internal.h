@@ -67,6 +67,7 @@ enum { RF_STATUS_BAD_INDEX = 0, RF_STATUS_TIMEOUT = 1, RF_STATUS_WORDS = 64 };
 
 // Error reporting (thread-local detail string).
 rf_status_t rf_fail(rf_status_t st, const std::string& msg);
+void rf_clear_error();  // every entry point starts with an empty detail string
 rf_status_t rf_check_launch(const char* what);
 rf_status_t rf_require_device();  // current device must be sm_100
 

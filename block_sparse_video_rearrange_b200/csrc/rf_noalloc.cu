@@ -32,7 +32,9 @@ void* g_scratch[RF_NOALLOC_MAX_DEVICES] = {};
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached for the life of the
+// process; a cudaDeviceReset on that device invalidates it, and the header
+// tells callers not to use this entry point after one.
 rf_status_t scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -60,6 +62,7 @@ rf_status_t scratch_for_current_device(void** out) {
 extern "C" rf_status_t rf_pool_select_noalloc(const rf_plan_t* p, const void* q_r, const void* k_r,
                                               int32_t* select_idx, int32_t* select_num,
                                               rf_stream_t stream) {
+  rf_clear_error();
   if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
   if (!q_r || !k_r || !select_idx || !select_num)
     return rf_fail(RF_ERR_INVALID_ARG, "null tensor");

@@ -60,6 +60,8 @@ rf_status_t rf_fail(rf_status_t st, const std::string& msg) {
   return st;
 }
 
+void rf_clear_error() { g_last_error.clear(); }
+
 rf_status_t rf_check_launch(const char* what) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)

@@ -144,11 +144,25 @@ class HostPipeline:
             if ev is not None:
                 caller.wait_event(ev)
 
+    def workspaces(self):
+        """The device workspace of every buffer set (status words at their start)."""
+        return [st["bufs"].ws for st in self.sets]
+
     def check_status(self) -> Tuple[int, Tuple[int, int]]:
-        """Device status words of every buffer set (synchronises); the first non-zero one."""
+        """Device status words of every buffer set (synchronises, reads and clears
+        them all); the first non-zero one."""
         torch.cuda.synchronize(self.device)
+        first = (0, (0, 0))
         for st in self.sets:
             s, flags = rf.check_device_status(self.plan, st["bufs"].ws)
-            if s != 0:
-                return s, flags
-        return 0, (0, 0)
+            if s != 0 and first[0] == 0:
+                first = (s, flags)
+        return first
+
+    def raise_on_device_fault(self) -> None:
+        """check_status, raising RfError(RF_ERR_DEVICE_FAULT) if any word was set."""
+        s, flags = self.check_status()
+        if s != rf.RF_OK:
+            raise rf.RfError(s, "rainfusion_attention (host pipeline)",
+                             f"device status words: {flags[0]} bad selectIdx entries, "
+                             f"expired-wait bits {flags[1]:#x}")

@@ -326,6 +326,15 @@ def check_device_status(plan: Plan, ws, stream=None) -> Tuple[int, Tuple[int, in
     return st, (int(flags[0]), int(flags[1]))
 
 
+def raise_on_device_fault(plan: Plan, ws, where: str, stream=None) -> None:
+    """Synchronise, read and clear the status words in ws; raise RfError(RF_ERR_DEVICE_FAULT)
+    if a kernel recorded an out-of-range selectIdx entry or an expired bounded wait."""
+    st, flags = check_device_status(plan, ws, stream)
+    if st != RF_OK:
+        raise RfError(st, where, f"device status words: {flags[0]} bad selectIdx entries, "
+                                 f"expired-wait bits {flags[1]:#x}")
+
+
 class Buffers:
     """Device intermediates and outputs of one path invocation (owned by torch)."""
 
@@ -365,7 +374,7 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          layout: str = "BNSD", scale: Optional[float] = None,
                          plan: Optional[Plan] = None, bufs: Optional[Buffers] = None,
                          order: str = "tile", precision: str = "native",
-                         chunks: Optional[int] = None) -> torch.Tensor:
+                         chunks: Optional[int] = None, check: bool = True) -> torch.Tensor:
     """User-level call: RainFusion v2 block-sparse attention of q, k, v (original token order).
 
     q, k, v may live on the host (pinned or not) or on the GPU; the result is
@@ -381,6 +390,14 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     shape and kept): head chunks whose copies to and from the GPU overlap
     the compute of other chunks; `chunks` overrides its default.  The result
     is the same, bit for bit, as one pass over all heads.
+
+    With check=True (the default) the call then synchronises and reads the
+    kernels' status words (aclnnRainFusionAttention returns a status code; a
+    CUDA kernel can only record one): an out-of-range selectIdx entry or an
+    expired bounded wait raises RfError with status RF_ERR_DEVICE_FAULT, and
+    the words are cleared, so the next call starts clean.  check=False skips
+    the synchronisation (timing loops); a later call with check=True, or
+    check_device_status, still sees what was recorded.
     """
     dtype = {torch.bfloat16: "bf16", torch.float16: "fp16"}[q.dtype]
     if not q.is_cuda and plan is None and bufs is None:
@@ -401,6 +418,8 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
         pipe(q, k, v, out, scale)
         torch.cuda.current_stream(dev).synchronize()
+        if check:
+            pipe.raise_on_device_fault()
         return out
     if plan is None:
         if layout == "BNSD":
@@ -415,6 +434,8 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         bufs = Buffers(plan, dev)
     qd, kd, vd = (x.to(dev, non_blocking=True) for x in (q, k, v))
     out = forward(plan, qd.contiguous(), kd.contiguous(), vd.contiguous(), bufs, scale)
+    if check:
+        raise_on_device_fault(plan, bufs.ws, "rainfusion_attention")
     if host:
         res = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
         res.copy_(out, non_blocking=True)

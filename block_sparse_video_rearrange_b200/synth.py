@@ -137,7 +137,13 @@ def generate_qkv(w: Workload) -> List[np.ndarray]:
     The seed depends only on the workload's base name, so a sparsity sweep
     reuses identical inputs.
     """
-    conv = float32_to_bf16_bits if w.dtype == "bf16" else float32_to_fp16_bits
+    conv1 = float32_to_bf16_bits if w.dtype == "bf16" else float32_to_fp16_bits
+
+    def conv(x):          # head by head: small temporaries, same bits as one call
+        out = np.empty(x.shape, dtype=np.uint16)
+        for n in range(x.shape[0]):
+            out[n] = conv1(x[n])
+        return out
     rng = np.random.Generator(np.random.PCG64(w.seed))
     result = []
     for tensor_idx, heads in enumerate((w.n1, w.n2, w.n2)):

@@ -26,7 +26,7 @@ through `rf` exactly as on one GPU.
 from __future__ import annotations
 
 import math
-from typing import Optional, Sequence, Tuple
+from typing import Callable, Optional, Sequence, Tuple
 
 import torch
 import torch.distributed as dist
@@ -103,22 +103,61 @@ class UlyssesAttention:
     [B, N1, L/P, D] and [B, N2, L/P, D], or TND [T/P, N1, D] and [T/P, N2, D]
     on this rank's GPU); returns this rank's row slice of the output.  The plan
     and the device buffers (for N1/P and N2/P heads) are made once.
+
+    `path`, when given, replaces the CUDA path on the rank's heads: a callable
+    (plan, qh, kh, vh, scale) -> output heads in the layout of qh.  It exists
+    so that the exchange and the reassembly can be tested on CPU ranks with a
+    stand-in computation; without it every step runs in librf.
     """
 
     def __init__(self, seqs: Sequence[Tuple[int, int, int, int]], n1: int, n2: int, d: int,
                  layout: str = "BNSD", dtype: str = "bf16", sparsity: float = 0.8, batch: int = 1,
-                 group=None, order: str = "tile", precision: str = "native", device=None):
+                 group=None, order: str = "tile", precision: str = "native", device=None,
+                 path: Optional[Callable] = None):
         world, _ = _world(group)
         check_shardable(seqs, n1, n2, layout, batch, world)
         self.group, self.layout, self.world = group, layout, world
         self.plan = rf.Plan(seqs, n1 // world, n2 // world, d, layout, dtype, sparsity, batch=batch,
                             order=order, precision=precision)
-        self.bufs = rf.Buffers(self.plan, device if device is not None else "cuda")
+        self.path = path
+        self.bufs = rf.Buffers(self.plan, device if device is not None else "cuda") if path is None else None
 
     def __call__(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
-                 scale: Optional[float] = None) -> torch.Tensor:
+                 scale: Optional[float] = None, events: Optional[Sequence] = None,
+                 check: bool = True) -> torch.Tensor:
+        """One layer.  `events`, if given, are 7 CUDA events recorded on the current
+        stream around the phases: exchange in, rearrange, pool_select, attention,
+        inverse, exchange out.  check=True synchronises after the call and raises
+        RfError(RF_ERR_DEVICE_FAULT) if a kernel recorded a fault (check=False
+        leaves the status words for a later check)."""
+        if scale is None:
+            scale = 1.0 / math.sqrt(self.plan.d)
+
+        def mark(i):
+            if events is not None:
+                events[i].record()
+        mark(0)
         qh = seq_to_head(q, self.layout, self.group)
         kh = seq_to_head(k, self.layout, self.group)
         vh = seq_to_head(v, self.layout, self.group)
-        o = rf.forward(self.plan, qh, kh, vh, self.bufs, scale if scale is not None else 1.0 / math.sqrt(self.plan.d))
-        return head_to_seq(o, self.layout, self.group)
+        mark(1)
+        if self.path is not None:
+            o = self.path(self.plan, qh, kh, vh, scale)
+            for i in range(2, 6):
+                mark(i)
+        else:
+            b, p = self.bufs, self.plan
+            rf.rearrange(p, qh, kh, vh, b.q_r, b.k_r, b.v_r, b.ws)
+            mark(2)
+            rf.pool_select(p, None, None, b.select_idx, b.select_num, b.ws)
+            mark(3)
+            rf.block_sparse_attn(p, b.q_r, b.k_r, b.v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
+            mark(4)
+            rf.inverse_rearrange(p, b.o_r, b.o)
+            mark(5)
+            o = b.o
+        out = head_to_seq(o, self.layout, self.group)
+        mark(6)
+        if check and self.path is None:
+            rf.raise_on_device_fault(self.plan, self.bufs.ws, "UlyssesAttention")
+        return out

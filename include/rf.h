@@ -303,12 +303,17 @@ RF_API rf_status_t rf_pool_select(const rf_plan_t* plan, const void* q_r, const 
  * Scratch: one static device array of 32 MiB inside librf.  It is set up on
  * the first call on each device (with that device current), which loads it
  * onto that GPU, where it stays until the process exits; make that first call
- * before any stream capture.  Problems whose selection scratch
- * (rf_plan_info().workspace_bytes; for a precision "mix" plan the part before
- * ws_q8) exceeds 32 MiB are rejected with RF_ERR_INVALID_ARG.  Every call on a device shares the array: calls that
- * overlap on the GPU (other streams, other threads) race and must be
- * serialised by the caller.  Calls no cudaMalloc, cudaFree or other
- * allocating routine. */
+ * before any stream capture.  The device address found at that set-up is
+ * kept for the life of the process: after cudaDeviceReset (or anything else
+ * that replaces the device's primary context) this entry point must not be
+ * called again on that device.  Size limit: the selection part of the plan's
+ * workspace layout must fit in 32 MiB -- that is the offset of the first
+ * quantized region (rf_plan_info().ws_q8 for a precision "mix" plan,
+ * ws_q_mx for a precision "mxfp4" plan), otherwise workspace_bytes; larger
+ * problems are rejected with RF_ERR_INVALID_ARG before any device work.
+ * Every call on a device shares the array: calls that overlap on the GPU
+ * (other streams, other threads) race and must be serialised by the caller.
+ * Calls no cudaMalloc, cudaFree or other allocating routine. */
 RF_API rf_status_t rf_pool_select_noalloc(const rf_plan_t* plan, const void* q_r, const void* k_r,
                                           int32_t* select_idx, int32_t* select_num,
                                           rf_stream_t stream);
@@ -360,9 +365,15 @@ RF_API rf_status_t rf_forward(const rf_plan_t* plan, const void* q, const void* 
 RF_API rf_status_t rf_plan_permutation(const rf_plan_t* plan, int32_t seq, int64_t* src_rows, int64_t n);
 
 /* Reads and clears the device status words in ws.  Synchronises `stream`.
+ * [API] constraints: selectIdx entries must be valid block indices or -1, and
+ * the call returns a status code; a CUDA kernel cannot return one, so the
+ * kernels record what they skipped and this call reports it.  It also stands
+ * in for a memory checker on the kernels' own bounds (they check every
+ * selectIdx entry themselves and record, rather than fault).
  * flags_out (may be NULL) receives the raw words: [0] out-of-range selectIdx
  * entries seen, [1] expired bounded waits.  Returns RF_ERR_DEVICE_FAULT if
- * either is non-zero. */
+ * either is non-zero.  ws is the caller's device workspace; nothing else is
+ * read or written. */
 RF_API rf_status_t rf_check_device_status(const rf_plan_t* plan, void* ws, uint32_t* flags_out,
                                    rf_stream_t stream);
 
@@ -382,13 +393,20 @@ RF_API rf_status_t rf_selftest_exp2(const float* x, float* y_poly, float* y_mufu
  * Takes about one second of device time; asynchronous on `stream`. */
 RF_API rf_status_t rf_selftest_expired_wait(const rf_plan_t* plan, void* ws, size_t ws_bytes,
                                             rf_stream_t stream);
-/* Frees a plan (NULL is a no-op). */
+/* Frees a plan (NULL is a no-op).  [API]: the second phase of the two-phase
+ * call releases what the first made; here the plan is the only thing the
+ * library owns (host memory), so this is all that is freed. */
 RF_API void rf_plan_destroy(rf_plan_t* plan);
 
-/* Static description of a status code. */
+/* Static description of a status code (the [API] page's return codes are
+ * named aclnnStatus values; these are this library's).  The string is owned by
+ * the library and never freed. */
 RF_API const char* rf_status_string(rf_status_t status);
 
-/* Detail of the last error returned on the calling thread ("" if none). */
+/* Detail of the last error returned on the calling thread ("" if none; every
+ * entry point clears it first).  The pages have no counterpart: aclnn reports
+ * its detail through the CANN log instead.  The string is owned by the
+ * library and valid until the next call on the same thread. */
 RF_API const char* rf_last_error(void);
 
 #ifdef __cplusplus

@@ -1,8 +1,9 @@
 """Shared parity checks: the CUDA path (through the C ABI) against the CPU oracle.
 
-Bars (stated for this path): permutation and selectNum bit-exact; selectIdx
-bit-exact except where two candidate block scores are within 1e-4 relative
-(then the swap must be such a near tie); attention output, with the oracle run
+Bars (stated for this path): permutation and selectNum bit-exact on every
+row; selectIdx bit-exact except where two candidate block scores are within
+1e-4 relative (then the GPU's row must still be a valid top-k up to such near
+ties); attention output, with the oracle run
 on the GPU's own selectIdx, max-abs <= 2e-2 and relative L2 <= 1e-2.
 """
 from __future__ import annotations
@@ -187,7 +188,13 @@ def check_pooled(p: orc.Problem, qbars, kbars, gpu) -> None:
 
 
 def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int, int]] | None = None) -> Dict[str, int]:
-    """selectIdx / selectNum against the oracle's selection.  Returns counters."""
+    """selectIdx / selectNum against the oracle's selection.  Returns counters.
+
+    selectNum must equal the oracle's on every row (bit-exact).  A selectIdx row
+    may differ from the oracle's only by near ties: the GPU's top-k set T (its
+    non-sink video blocks, completed with the best-scoring sinks) must be a
+    valid top-k of the oracle's float64 scores, in that every block in T scores
+    at least as high as every video block outside T, up to TIE_REL relative."""
     idx_o, num_o = orc.select(p, qbars, kbars)
     idx_g, num_g = gpu["idx"], gpu["num"]
     assert idx_g.shape == idx_o.shape and num_g.shape == num_o.shape
@@ -198,6 +205,7 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
     todo = rows if rows is not None else [(t, n) for t in range(len(table)) for n in range(p.n1)]
     for t, n in todo:
         stats["rows"] += 1
+        assert num_g[t, n] == num_o[t, n], f"selectNum differs at (t={t}, n={n}): {num_g[t, n]} vs {num_o[t, n]}"
         a = idx_g[t, n, :num_g[t, n]].tolist()
         b = idx_o[t, n, :num_o[t, n]].tolist()
         # padding is -1 everywhere past selectNum
@@ -207,14 +215,22 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
             stats["exact"] += 1
             continue
         s, g, qb = table[t]
+        assert not g.dense and qb >= g.n_pb + g.ns, f"dense row (t={t}, n={n}) differs"
+        assert a[:g.n_pb] == list(range(g.n_pb)), (t, n, a[:g.n_pb])
         si = seq_pos[s]
         sc = qbars[si][n, qb - g.n_pb] @ kbars[si][n // G].T
-        extra = [j - g.n_pb for j in set(a) - set(b)]
-        missing = [j - g.n_pb for j in set(b) - set(a)]
-        assert extra and missing, (t, n, a, b)
-        for x in extra:
-            for m in missing:
-                assert abs(sc[x] - sc[m]) <= TIE_REL * max(abs(sc[x]), abs(sc[m])), (t, n, x, m, sc[x], sc[m])
+        video = [j - g.n_pb for j in a[g.n_pb:]]
+        sinks = set(range(g.ns))
+        assert sinks <= set(video), (t, n)
+        chosen = [j for j in video if j not in sinks]
+        assert len(chosen) <= g.k, (t, n, len(chosen), g.k)
+        best_sinks = sorted(sinks, key=lambda j: (-sc[j], j))[:g.k - len(chosen)]
+        top = set(chosen) | set(best_sinks)
+        rest = [j for j in range(g.nb) if j not in top]
+        if top and rest:
+            lo = min(top, key=lambda j: sc[j])
+            hi = max(rest, key=lambda j: sc[j])
+            assert sc[lo] >= sc[hi] - TIE_REL * max(abs(sc[lo]), abs(sc[hi])), (t, n, lo, hi, sc[lo], sc[hi])
         stats["near_tie"] += 1
     return stats
 

@@ -87,6 +87,14 @@ def test_keep_count_matches_oracle(s):
         assert plan.seq_info[0].k == orc.keep_count(nb, s)
 
 
+def test_keep_count_of_the_plan_equals_the_pinned_values():
+    """The host plan's k against the hand-worked values of reading R4 (not the oracle)."""
+    from tests.test_oracle_geometry import PINNED_K
+    for (p, t, h, w, s, nb, k) in PINNED_K:
+        plan = rf.Plan([(p, t, h, w)], 1, 1, 128, sparsity=s)
+        assert (plan.seq_info[0].nb, plan.seq_info[0].k) == (nb, k), (p, t, h, w, s)
+
+
 def test_host_validation_runs_before_any_device_call():
     plan = rf.Plan([(128, 9, 16, 32)], 2, 2, 64)
     fake = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: validation fails first

@@ -61,3 +61,36 @@ def test_attention_after_a_recorded_expiry_skips_its_work():
                o_r=parity.to_bits(b.o_r))
     p = parity.problem(w)
     parity.check_attention(p, w, parity_rearranged(p, bits), gpu)
+
+
+def test_public_call_raises_on_a_recorded_fault_and_the_next_call_succeeds():
+    """rainfusion_attention reads the status words after every call (check=True): an
+    expiry recorded in its workspace raises RfError(RF_ERR_DEVICE_FAULT), the words are
+    cleared, and the next call computes the right result."""
+    w = SMALL["ragged_d128"]
+    bits = synth.generate_qkv(w)
+    ref = parity.run_gpu(w, bits)
+    seqs = parity.seqs_of(w)
+    plan = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity)
+    b = rf.Buffers(plan)
+    q, k, v = (parity.to_device(x, w.dtype) for x in bits)
+    rf.selftest_expired_wait(plan, b.ws)
+    with pytest.raises(rf.RfError) as e:
+        rf.rainfusion_attention(q, k, v, seqs, w.sparsity, plan=plan, bufs=b)
+    assert e.value.status == 5
+    out = rf.rainfusion_attention(q, k, v, seqs, w.sparsity, plan=plan, bufs=b)
+    torch.cuda.synchronize()
+    assert np.array_equal(parity.to_bits(out), ref["o"])
+
+    # the same through the host pipeline (host tensors): the fault is recorded in one of
+    # the pipeline's workspaces, the next call raises, the call after it succeeds
+    hq, hk, hv = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in bits)
+    first = rf.rainfusion_attention(hq, hk, hv, seqs, w.sparsity)
+    assert np.array_equal(first.view(torch.int16).numpy().view(np.uint16), ref["o"])
+    pipe = next(pp for key, pp in rf._PIPELINES.items() if key[0] == tuple(map(tuple, seqs)))
+    rf.selftest_expired_wait(pipe.plan, pipe.workspaces()[-1])
+    with pytest.raises(rf.RfError) as e:
+        rf.rainfusion_attention(hq, hk, hv, seqs, w.sparsity)
+    assert e.value.status == 5
+    again = rf.rainfusion_attention(hq, hk, hv, seqs, w.sparsity)
+    assert np.array_equal(again.view(torch.int16).numpy().view(np.uint16), ref["o"])

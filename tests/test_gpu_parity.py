@@ -171,7 +171,7 @@ def test_user_call_with_host_tensors():
 # ------------------------------------------------------------------------------------------
 
 FULL = [("wan", None), ("minimax", 0.8), ("minimax", 0.5), ("minimax", 0.9), ("tnd_gqa", None),
-        ("aligned", 0.8), ("aligned", 0.0)]
+        ("aligned", 0.8), ("aligned", 0.0), ("aligned", 0.5), ("aligned", 0.9)]
 
 
 @pytest.mark.parametrize("name,s", FULL)
@@ -188,6 +188,33 @@ def test_full_size_parity(name, s):
     assert stats["near_tie"] <= max(1, stats["rows"] // 1000), stats
     items = parity.sample_items(p, np.random.default_rng(7), per_kind=3)
     parity.check_attention(p, w, rbits, gpu, items)
+
+
+# Whole heads at full size: every query block of the first and the last query head
+# against the oracle, one full-size configuration per precision.
+WHOLE_HEADS = [("aligned", 0.8, "native"), ("wan", None, "mix"), ("wan", None, "mxfp4")]
+
+
+@pytest.mark.parametrize("name,s,precision", WHOLE_HEADS)
+def test_full_size_whole_heads(name, s, precision):
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision=precision)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    items = [(t, n) for t in range(p.t_qblk) for n in (0, w.n1 - 1)]
+    if precision == "native":
+        err = parity.check_attention(p, w, rbits, gpu, items)
+    elif precision == "mix":
+        parity.check_mix_quantization(p, w, rbits, gpu)
+        err = parity.check_attention(p, w, rbits, gpu, items, values=parity.mix_reference_inputs(p, w, gpu, rbits))
+    else:
+        ref = parity.oracle_mx_inputs(p, w, rbits)
+        parity.check_mx_quantization(p, w, ref, gpu)
+        err = parity.check_attention(p, w, rbits, gpu, items, values=ref, oracle_fn=mxo.attention_mx)
+    print(f"{name}@{w.sparsity:g} {precision}: {err['items']} items (two whole heads), "
+          f"max abs {err['max_abs']:.3e}, rel L2 {err['rel_l2']:.3e}")
+    assert err["items"] == 2 * p.t_qblk
 
 
 # ------------------------------------------------------------------------------------------

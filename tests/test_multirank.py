@@ -89,3 +89,78 @@ def test_ulysses_shardability_rules():
         ulysses.check_shardable([(512, 21, 30, 52)], 40, 40, "BNSD", 1, 16)     # rows do not divide
     with pytest.raises(ValueError):
         ulysses.check_shardable([(256, 13, 32, 48)], 32, 8, "TND", 1, 16)       # 8 kv heads over 16 ranks
+
+
+# ---------------- UlyssesAttention composition (gloo, world size 2 and 4) ----------------
+#
+# Each rank runs the layer on its row slices; the per-rank path is replaced by the CPU
+# oracle (injected by the test: the product never imports it).  The reassembled output
+# must equal the oracle's whole path over all heads, because every step of the path is
+# independent per (sequence, head) and a query head stays with its key/value head.
+
+ULYSSES_CASES = {
+    # BNSD, G = 2, 32 sparse blocks (not dense), L = 4,160 rows
+    "bnsd": dict(layout="BNSD", dtype="bf16", seqs=[(64, 8, 16, 32)], n1=8, n2=4, d=64, sparsity=0.8),
+    # TND varlen, G = 2: a sparse sequence next to a short dense one, T = 6,676 rows
+    "tnd": dict(layout="TND", dtype="fp16", seqs=[(32, 8, 16, 32), (100, 9, 16, 17)], n1=8, n2=4, d=64,
+                sparsity=0.7),
+}
+
+
+def _oracle_path(plan, qh, kh, vh, scale):
+    import numpy as np
+    from block_sparse_video_rearrange_b200 import synth
+    from oracle import rainfusion as orc
+    p = orc.make_problem(plan.layout, plan.batch, plan.seqs, plan.n1, plan.n2, plan.d, plan.sparsity)
+    f = [synth.bits_to_float64(x.contiguous().view(torch.int16).numpy().view(np.uint16), plan.dtype)
+         for x in (qh, kh, vh)]
+    return torch.from_numpy(orc.run_path(p, *f, scale)["o"])
+
+
+def _case_inputs(c):
+    import numpy as np
+    from block_sparse_video_rearrange_b200 import synth
+    specs = tuple(synth.SeqSpec(*s) for s in c["seqs"])
+    w = synth.Workload("ulysses", c["layout"], c["dtype"], 1, specs, c["n1"], c["n2"], c["d"], c["sparsity"], 77)
+    bits = synth.generate_qkv(w)
+    tdt = torch.bfloat16 if c["dtype"] == "bf16" else torch.float16
+    return [torch.from_numpy(b.view(np.int16)).view(tdt) for b in bits]
+
+
+def _ulysses_layer_worker(rank, world, port, name, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    from block_sparse_video_rearrange_b200 import ulysses
+    c = ULYSSES_CASES[name]
+    q, k, v = _case_inputs(c)
+    axis = 2 if c["layout"] == "BNSD" else 0
+    rows = q.shape[axis] // world
+    mine = [x.narrow(axis, rank * rows, rows).contiguous() for x in (q, k, v)]
+    layer = ulysses.UlyssesAttention(c["seqs"], c["n1"], c["n2"], c["d"], c["layout"], c["dtype"], c["sparsity"],
+                                     path=_oracle_path)
+    o = layer(*mine, scale=0.125)
+    out[rank] = o.numpy()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", sorted(ULYSSES_CASES))
+@pytest.mark.parametrize("world", [2, 4])
+def test_ulysses_layer_equals_the_oracle_over_all_heads(name, world):
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    from block_sparse_video_rearrange_b200 import rf
+    mgr = mp.Manager()
+    out = mgr.dict()
+    port = 27500 + (os.getpid() + 31 * world + 7 * len(name)) % 1000
+    mp.spawn(_ulysses_layer_worker, args=(world, port, name, out), nprocs=world, join=True)
+    c = ULYSSES_CASES[name]
+    q, k, v = _case_inputs(c)
+    plan = rf.Plan(c["seqs"], c["n1"], c["n2"], c["d"], c["layout"], c["dtype"], c["sparsity"])
+    full = _oracle_path(plan, q, k, v, 0.125).numpy()
+    axis = 2 if c["layout"] == "BNSD" else 0
+    got = np.concatenate([out[r] for r in range(world)], axis=axis)
+    assert got.shape == full.shape
+    assert np.max(np.abs(got - full)) <= 1e-12

@@ -253,3 +253,45 @@ def test_unknown_order_is_rejected():
         rf.geometry(0, 2, 8, 8, 0.8, "zigzag")
     with pytest.raises(ValueError):
         rf.video_order(2, 8, 8, "zigzag")
+
+
+# ---------------- k per configuration (reading R4: k = ceil((1 - s) * nb)) ----------------
+#
+# "RainFusion Attention" user guide, "Configuration": sparsity is the nominal
+# fraction of ranked key blocks dropped.  Reading R4 keeps ceil((1 - s) * nb)
+# blocks.  The values below are that rule worked out by hand for every
+# configuration of the benchmark, and they are written here as numbers, not
+# recomputed: a floor (or round-half-down) implementation fails on Tiny
+# (7.2 -> 8), Wan (37.8 -> 38), MiniMax at 0.5 and 0.9 (232.5 -> 233,
+# 46.5 -> 47) and both TND sequences (31.2, 31.4 -> 32); the guard against
+# float noise is exercised by MiniMax at 0.8 ((1 - 0.8) * 465 = 92.99999...).
+PINNED_K = [
+    # (prefix, t, h, w, sparsity, nb, k)
+    (128, 9, 16, 32, 0.8, 36, 8),          # Tiny
+    (512, 21, 30, 52, 0.8, 189, 38),       # Wan2.2-shaped
+    (256, 62, 24, 42, 0.5, 465, 233),      # MiniMax-H3-shaped sweep
+    (256, 62, 24, 42, 0.8, 465, 93),
+    (256, 62, 24, 42, 0.9, 465, 47),
+    (512, 21, 48, 80, 0.0, 630, 630),      # Aligned sweep
+    (512, 21, 48, 80, 0.5, 630, 315),
+    (512, 21, 48, 80, 0.8, 630, 126),
+    (512, 21, 48, 80, 0.9, 630, 63),
+    (256, 13, 32, 48, 0.8, 156, 32),       # TND sequence 0
+    (384, 21, 24, 40, 0.8, 157, 32),       # TND sequence 1
+]
+
+
+@pytest.mark.parametrize("p,t,h,w,s,nb,k", PINNED_K)
+def test_keep_count_pinned_per_configuration(p, t, h, w, s, nb, k):
+    g = rf.geometry(p, t, h, w, s)
+    assert (g.nb, g.k) == (nb, k)
+    assert rf.keep_count(nb, s) == k
+
+
+def test_keep_count_pins_reject_a_floor(monkeypatch):
+    """Plant the likeliest mistake (floor instead of ceiling) in the oracle and check
+    that the pinned table catches it."""
+    import math as _math
+    monkeypatch.setattr(rf.math, "ceil", _math.floor)
+    wrong = [(p, t, h, w, s) for (p, t, h, w, s, nb, k) in PINNED_K if rf.geometry(p, t, h, w, s).k != k]
+    assert len(wrong) >= 6, wrong

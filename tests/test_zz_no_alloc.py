@@ -64,6 +64,18 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     st = rf.lib().rf_pool_select_noalloc(plan.handle, p, p, p, p, None)
     assert st == 1                            # RF_ERR_INVALID_ARG
     assert b"scratch" in rf.lib().rf_last_error()
+    # a successful call right after the rejection leaves no stale error text
+    w = CASES["ragged_d128"]
+    bits = synth.generate_qkv(w)
+    small = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch)
+    q, k, v = (parity.to_device(x, w.dtype) for x in bits)
+    b = rf.Buffers(small)
+    rf.rearrange(small, q, k, v, b.q_r, b.k_r, b.v_r, b.ws)
+    st = rf.lib().rf_pool_select_noalloc(plan.handle, p, p, p, p, None)
+    assert st == 1
+    rf.pool_select_noalloc(small, b.q_r, b.k_r, b.select_idx, b.select_num)
+    assert rf.lib().rf_last_error() == b""
+    torch.cuda.synchronize()
 
 
 @pytest.mark.parametrize("precision", ["mix", "mxfp4"])
