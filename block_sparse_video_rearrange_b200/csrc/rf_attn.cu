@@ -19,33 +19,37 @@
 //   warps 4-7  softmax warpgroup 1: the odd-numbered selected blocks
 //              (thread = query row = TMEM lane in both groups)
 //   warp 8     TMA producer of Q (once) and K_j through a 3-stage ring
-//   warp 9     TMEM allocation and the single-thread tcgen05.mma issue
+//   warp 9     TMEM allocation and the tcgen05.mma issue of S_j = Q K_j^T
 //   warp 10    TMA producer of V_j through a 2-stage ring (K and V have
 //              separate producers so that a K load never queues behind a V
 //              load that waits for an earlier P V product)
-//   warp 11    idle (it completes the third warpgroup)
+//   warp 11    the tcgen05.mma issue of O += P_j V_j
+// One elected thread per issuing warp issues that warp's MMAs.  A single
+// issuing thread cannot keep the tensor pipe busy at M = N = 128: every
+// barrier check costs it about as much as an MMA's worth of pipe time.
 // The kernel launches with 168 registers per thread; the third warpgroup
 // gives registers back (72 each) and the softmax groups take them (216 each),
 // so that a thread holds its whole 128-column score row: 2*128*216 + 128*72
 // = 384*168.
 // TMEM columns: S_w at [128 w, 128 w + 128) and O_w at [256 + 128 w, +D) for
-// warpgroup w.  P is written back over its own S buffer as packed 16-bit pairs
-// and is the A operand (from TMEM) of O_w += P V.
-// Each warpgroup keeps its own running max / sum and accumulator over its
-// half of the blocks; the epilogue merges the two halves (a fixed split, so
-// the result is deterministic).  MMA issue order: S_0, S_1, then for every j:
-// O_{j%2} += P_j V_j followed by S_{j+2}, so one group's softmax overlaps the
-// other group's matrix products.  P_j V_j goes in two halves of the key rows:
-// the softmax releases the first 64 columns of P_j before computing the rest.
-// The softmax works in the exp2 domain; O_w is rescaled only when a row max
-// grows by more than 2^8 (a warp-uniform decision), right after the row max,
-// before any of P_j is released (O_w is at rest then: S_j completes after the
-// group's previous P V).  Column pairs selected by
+// softmax group w.  P_j is written back over its own score buffer as packed
+// 16-bit pairs and is the A operand (from TMEM) of O_w += P_j V_j.
+// S_j goes into buffer j % 2 once P_{j-2} V_{j-2} (which reads P_{j-2} from
+// it) is complete, so a group's chain is S_j -> softmax -> P_j V_j -> S_{j+2};
+// the two groups alternate, and one group's softmax overlaps the other
+// group's products.  P_j V_j goes in two halves of the key rows: the softmax
+// releases the first 64 columns of P_j before computing the rest.
+// Each group keeps its own running max, sum and accumulator over its half of
+// the blocks, so the groups never wait for each other; the epilogue merges
+// the two halves (a fixed split, so the result is deterministic).  O_w is
+// rescaled only when a row max grows by more than 2^8 (a warp-uniform
+// decision), right after the row max and before any of P_j is released (O_w
+// is at rest then: S_j was issued after the group's previous P V was complete).
+// The softmax works in the exp2 domain.  Column pairs selected by
 // RF_EMU_PAIR_MASK take their exponentials from a polynomial on the FMA pipe
-// (rf_exp2_poly) instead of the MUFU unit.  Measured on the Wan2.2-shaped
-// layer, offloading 12.5% or 25% of them was slower than none (the extra
-// instructions cost more than the MUFU time they save at this schedule), so
-// the default mask is 0.
+// (rf_exp2_poly2, two values per paired instruction) instead of the MUFU unit,
+// whose 16 results per clock per SM are otherwise as busy as the tensor pipe
+// at D = 128.
 // Every wait is bounded: on expiry the CTA records it in the status words and
 // unwinds (waiting, again bounded, for its own copies and MMAs in flight).
 //
@@ -72,6 +76,7 @@ constexpr int kThreads = 384;
 constexpr int kProducerWarp = 8;   // Q and K loads
 constexpr int kMmaWarp = 9;
 constexpr int kVProducerWarp = 10; // V loads
+constexpr int kPvWarp = 11;        // P V issue
 constexpr int kLaunchRegs = 168;   // 65536 / 384, rounded down to a multiple of 8
 constexpr uint32_t kSoftmaxRegs = 216;
 constexpr uint32_t kOtherRegs = 72;
@@ -80,8 +85,10 @@ static_assert(2 * 128 * kSoftmaxRegs + 128 * kOtherRegs <= kThreads * kLaunchReg
 #ifndef RF_EMU_PAIR_MASK
 #define RF_EMU_PAIR_MASK 0x0u
 #endif
-constexpr uint32_t kEmuPairMask = RF_EMU_PAIR_MASK;  // bit i: pair i of every 16 column pairs uses rf_exp2_poly
+constexpr uint32_t kEmuPairMask = RF_EMU_PAIR_MASK;  // bit i: pair i of every 16 column pairs uses rf_exp2_poly2
 constexpr int kStagesK = 3;  // K ring: K_{j+3} is requested as soon as S_j is done
+constexpr uint32_t kPCol = 128;  // P of group w at kPCol + 64 w (128 keys as 16-bit pairs)
+constexpr uint32_t kOCol = 256;  // O_w, the accumulator of softmax group w, at kOCol + 128 w
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy rescale while growth <= 256x
@@ -100,7 +107,11 @@ struct __align__(1024) AttnSmem {
   uint64_t bar_q;
   uint64_t bar_k_full[kStagesK], bar_k_empty[kStagesK];
   uint64_t bar_v_full[kStagesV], bar_v_empty[kStagesV];
-  uint64_t bar_s_full[2], bar_p_half[2], bar_p_full[2];
+  uint64_t bar_s_full[2];    // S_j computed (j % 2: one barrier per softmax group, so that
+                             // a group never mistakes the other group's S for its own)
+  uint64_t bar_s_free;       // S_j read into registers: the score buffer may take S_{j+1}
+  uint64_t bar_p_half[2], bar_p_full[2];  // P_j stored, first half / all (j % 2)
+  uint64_t bar_pv_done[2];   // O_{j%2} += P_j V_j complete: P buffer j % 2 may take P_{j+2}
   uint64_t bar_final;
   uint64_t bar_drain;
   uint32_t tmem_base;
@@ -163,25 +174,31 @@ __device__ __forceinline__ float row_max(const uint32_t* sr, int vr) {
   return rf_max3(rf_max3(m[0], m[1], m[2]), rf_max3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// p = 2^(s * sl2 - m) for the 64 scores c0 .. c0 + 63 of a row (the first vr
-// of the row valid), packed pairwise to 16-bit into pk[32]; the fp32 sums go
-// to the four paired accumulators acc (a column pair's accumulator does not
-// depend on c0, so two halves sum in the same order as one pass would).  The
-// scale-and-subtract and the sums run as paired fp32 instructions (two columns
-// per instruction).  Pairs selected by kEmuPairMask use the FMA-pipe
-// polynomial, the others ex2.approx.
+// p = 2^(s * sl2 - m) for the 32 scores c0 .. c0 + 31 of a row (the first vr
+// of the row valid), packed pairwise to 16-bit and stored to the 16 TMEM
+// columns at p_addr; the fp32 sums go to the four paired accumulators acc (a
+// column pair's accumulator does not depend on c0, so the quarters sum in the
+// same order as one pass would).  The scale-and-subtract and the sums run as
+// paired fp32 instructions (two columns per instruction).  Pairs selected by
+// kEmuPairMask use the FMA-pipe polynomial (both values of the pair at once),
+// the others ex2.approx.
 template <bool kBf16, bool kFull>
-__device__ __forceinline__ void half_row_exp(const uint32_t* sr, int c0, int vr, float sl2, float neg_m,
-                                             uint32_t* pk, uint64_t* acc) {
+__device__ __forceinline__ void quarter_row_exp(const uint32_t* sr, int c0, int vr, float sl2, float neg_m,
+                                                uint32_t p_addr, uint64_t* acc) {
   const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
   const uint64_t negm2 = rf_f2(__float_as_uint(neg_m), __float_as_uint(neg_m));
+  uint32_t pk[16];
 #pragma unroll
-  for (int c = 0; c < 64; c += 2) {
+  for (int c = 0; c < 32; c += 2) {
     const bool emu = (kEmuPairMask >> ((c >> 1) & 15)) & 1u;
-    float x0, x1;
+    float x0, x1, p0, p1;
     rf_f2_split(rf_fma2(rf_f2(sr[c0 + c], sr[c0 + c + 1]), sl2x2, negm2), x0, x1);
-    float p0 = emu ? rf_exp2_poly(x0) : rf_ex2(x0);
-    float p1 = emu ? rf_exp2_poly(x1) : rf_ex2(x1);
+    if (emu) {
+      rf_exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = rf_ex2(x0);
+      p1 = rf_ex2(x1);
+    }
     if (!kFull) {
       p0 = c0 + c < vr ? p0 : 0.f;
       p1 = c0 + c + 1 < vr ? p1 : 0.f;
@@ -189,6 +206,7 @@ __device__ __forceinline__ void half_row_exp(const uint32_t* sr, int c0, int vr,
     acc[(c >> 1) & 3] = rf_add2(acc[(c >> 1) & 3], rf_f2(__float_as_uint(p0), __float_as_uint(p1)));
     pk[c >> 1] = rf_pack2<kBf16>(p0, p1);
   }
+  tmem_st16(p_addr, pk);
 }
 
 // Maxima of the four 32-column groups of a row of raw scores (the first vr
@@ -211,50 +229,48 @@ __device__ __forceinline__ void group_max4(const uint32_t* sr, int vr, float* gm
   }
 }
 
-// Precision "mxfp4": P over the 64 scores c0 .. c0 + 63 of a row (two groups
-// of 32 keys), rounded to MXFP4 per group and packed as f16 pairs into
-// pk[32]; the rounded values are summed into lsum.  m is the integer running
-// max; gm2 the two groups' raw score maxima.  Group exponent (UOS):
+// Precision "mxfp4": P over the 32 scores cb .. cb + 31 of a row (one group of
+// 32 keys), rounded to MXFP4 and packed as f16 pairs into the 16 TMEM columns
+// at p_addr; the rounded values are summed into lsum.  m is the integer
+// running max; gmax the group's raw score maximum.  Group exponent (UOS):
 // e = ceil(log2(amax / 7.25)) with log2(amax) = gmax * sl2 - m; the
 // exponentials are taken as 2^(s * sl2 - (m + e)), rounded to E2M1 (the
 // hardware conversion saturates at 6), summed exactly in f16 (at most 32
 // values of at most 6 on a 0.5 grid) and scaled by 2^e.
 template <bool kFull>
-__device__ __forceinline__ void half_row_exp_mx(const uint32_t* sr, int c0, int vr, float sl2, float m,
-                                                const float* gm2, uint32_t* pk, float& lsum) {
+__device__ __forceinline__ void group_exp_mx(const uint32_t* sr, int cb, int vr, float sl2, float m,
+                                             float gmax, uint32_t p_addr, float& lsum) {
   const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
+  const bool live = kFull || cb < vr;
+  const int e = live ? (int)ceilf(fmaf(gmax, sl2, -m) - kMxLog2Qmax) : 0;
+  const float neg_me = -(m + (float)e);
+  const uint64_t negme2 = rf_f2(__float_as_uint(neg_me), __float_as_uint(neg_me));
+  // 2^e as f16 (normal from 2^-14, subnormal down to 2^-24; a group whose
+  // scale is below that rounds to zero in f16, as its P V terms would)
+  const unsigned short hb = e >= -14 ? (unsigned short)((15 + e) << 10)
+                                     : (e >= -24 ? (unsigned short)(1u << (e + 24)) : (unsigned short)0);
+  const __half2 up2 = __half2half2(__ushort_as_half(hb));
+  __half2 acc0 = __float2half2_rn(0.f), acc1 = acc0;
+  uint32_t pk[16];
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int cb = c0 + 32 * h;
-    const bool live = kFull || cb < vr;
-    const int e = live ? (int)ceilf(fmaf(gm2[h], sl2, -m) - kMxLog2Qmax) : 0;
-    const float neg_me = -(m + (float)e);
-    const uint64_t negme2 = rf_f2(__float_as_uint(neg_me), __float_as_uint(neg_me));
-    // 2^e as f16 (normal from 2^-14, subnormal down to 2^-24; a group whose
-    // scale is below that rounds to zero in f16, as its P V terms would)
-    const unsigned short hb = e >= -14 ? (unsigned short)((15 + e) << 10)
-                                       : (e >= -24 ? (unsigned short)(1u << (e + 24)) : (unsigned short)0);
-    const __half2 up2 = __half2half2(__ushort_as_half(hb));
-    __half2 acc0 = __float2half2_rn(0.f), acc1 = acc0;
-#pragma unroll
-    for (int c = 0; c < 32; c += 2) {
-      float x0, x1;
-      rf_f2_split(rf_fma2(rf_f2(sr[cb + c], sr[cb + c + 1]), sl2x2, negme2), x0, x1);
-      float y0 = rf_ex2(x0), y1 = rf_ex2(x1);
-      if (!kFull) {
-        y0 = cb + c < vr ? y0 : 0.f;
-        y1 = cb + c + 1 < vr ? y1 : 0.f;
-      }
-      const uint32_t r = rf_e2m1x2_round(y0, y1);
-      const __half2 rh = *reinterpret_cast<const __half2*>(&r);
-      if (c & 2) acc1 = __hadd2(acc1, rh);
-      else       acc0 = __hadd2(acc0, rh);
-      const __half2 ph = __hmul2(rh, up2);
-      pk[(cb - c0 + c) >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
+  for (int c = 0; c < 32; c += 2) {
+    float x0, x1;
+    rf_f2_split(rf_fma2(rf_f2(sr[cb + c], sr[cb + c + 1]), sl2x2, negme2), x0, x1);
+    float y0 = rf_ex2(x0), y1 = rf_ex2(x1);
+    if (!kFull) {
+      y0 = cb + c < vr ? y0 : 0.f;
+      y1 = cb + c + 1 < vr ? y1 : 0.f;
     }
-    const float2 sum = __half22float2(__hadd2(acc0, acc1));
-    if (live && e >= -126) lsum = fmaf(sum.x + sum.y, rf_pow2(e), lsum);
+    const uint32_t r = rf_e2m1x2_round(y0, y1);
+    const __half2 rh = *reinterpret_cast<const __half2*>(&r);
+    if (c & 2) acc1 = __hadd2(acc1, rh);
+    else       acc0 = __hadd2(acc0, rh);
+    const __half2 ph = __hmul2(rh, up2);
+    pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
   }
+  const float2 sum = __half22float2(__hadd2(acc0, acc1));
+  if (live && e >= -126) lsum = fmaf(sum.x + sum.y, rf_pow2(e), lsum);
+  tmem_st16(p_addr, pk);
 }
 
 __device__ __forceinline__ float acc_sum(const uint64_t* acc) {
@@ -308,12 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(rf_smem_u32(&sm.bar_v_empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(rf_smem_u32(&sm.bar_s_full[i]), 1);
       mbar_init(rf_smem_u32(&sm.bar_p_half[i]), 128);
       mbar_init(rf_smem_u32(&sm.bar_p_full[i]), 128);
+      mbar_init(rf_smem_u32(&sm.bar_pv_done[i]), 1);
     }
-    mbar_init(rf_smem_u32(&sm.bar_final), 1);
-    mbar_init(rf_smem_u32(&sm.bar_drain), 1);
+    mbar_init(rf_smem_u32(&sm.bar_s_full[0]), 1);
+    mbar_init(rf_smem_u32(&sm.bar_s_full[1]), 1);
+    mbar_init(rf_smem_u32(&sm.bar_s_free), 128);
+    mbar_init(rf_smem_u32(&sm.bar_final), 2);   // one commit from each issuing warp
+    mbar_init(rf_smem_u32(&sm.bar_drain), 2);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -480,77 +499,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
         mbar_wait(rf_smem_u32(&full[j % stages]), (j / stages) & 1, &no_abort);
     }
-  } else if (warp == kMmaWarp && nv > 0) {
-    // ---------------- tcgen05.mma issue ----------------
-    // The whole warp runs this loop (warp-uniform control flow keeps the
-    // descriptors in uniform registers); one elected lane issues every MMA
-    // and every commit, so the commits track all of them.
+  } else if ((warp == kMmaWarp || warp == kPvWarp) && nv > 0) {
+    // ---------------- tcgen05.mma issue: S products (warp 9), P V products (warp 11) ----------------
+    // Two issuing warps: a single thread cannot keep the tensor pipe fed with
+    // 128 x 128 x 16 instructions once its barrier checks sit between them.
+    // Each warp runs its whole loop (warp-uniform control flow keeps the
+    // descriptors in uniform registers); one elected lane issues every MMA and
+    // every commit of that warp, so its commits track all of its MMAs.
     const uint32_t fmt = kBf16 ? 1u : 0u;
-    // kind::f8f6f4 takes E4M3 as format 0 in the same descriptor fields.
-    const uint32_t idesc_qk = umma_idesc_f16(kQk8 ? 0u : fmt, 128, 128, 0);
-    // precision "mxfp4": P and V are f16 whatever the input type
-    const uint32_t idesc_pv = umma_idesc_f16(kMx ? 0u : fmt, 128, D, 1);
-    // Adding (bytes >> 4) to a descriptor moves its 14-bit start-address field.
-    const uint64_t dq = umma_desc_sw128(rf_smem_u32(sm.q), 16, 1024);
-    const uint64_t dk0 = umma_desc_sw128(rf_smem_u32(sm.k[0]), 16, 1024);
-    const uint64_t dv0 = umma_desc_sw128(rf_smem_u32(sm.v[0]), kBoxBytes, 1024);
-    // S_j = Q K_j^T into the S buffer of warpgroup j % 2.  Every MMA takes a
-    // 32-byte slice of the reduction (16 bf16/fp16 or 32 E4M3 elements).
-    auto issue_qk = [&](int j) -> bool {
-      const int st = j % kStagesK;
-      if (!warp_wait<true>(rf_smem_u32(&sm.bar_k_full[st]), (j / kStagesK) & 1, abort)) return false;
-      tc_fence_after();
-      if (elect_one()) {
-        const uint64_t dk = dk0 + (uint64_t)(st * (kQkTileBytes >> 4));
-#pragma unroll
-        for (int kk = 0; kk < (int)(kQkTileBytes / RF_BLOCK / 32); ++kk) {
-          const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
-          if constexpr (kQk8)
-            mma_ss_f8(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
-          else
-            mma_ss(tmem + (j & 1) * 128, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+    bool ok = true;
+    if (warp == kMmaWarp) {
+      // kind::f8f6f4 takes E4M3 as format 0 in the same descriptor fields.
+      const uint32_t idesc_qk = umma_idesc_f16(kQk8 ? 0u : fmt, 128, 128, 0);
+      // Adding (bytes >> 4) to a descriptor moves its 14-bit start-address field.
+      const uint64_t dq = umma_desc_sw128(rf_smem_u32(sm.q), 16, 1024);
+      const uint64_t dk0 = umma_desc_sw128(rf_smem_u32(sm.k[0]), 16, 1024);
+      ok = warp_wait<true>(rf_smem_u32(&sm.bar_q), 0, abort);
+      for (int j = 0; ok && j < nv; ++j) {
+        const int st = j % kStagesK;
+        // S_j goes into the score buffer once the softmax has read S_{j-1}.
+        if (j > 0 && !warp_wait<true>(rf_smem_u32(&sm.bar_s_free), (j - 1) & 1, abort)) {
+          ok = false;
+          break;
         }
-        tc_commit(rf_smem_u32(&sm.bar_s_full[j & 1]));
-        tc_commit(rf_smem_u32(&sm.bar_k_empty[st]));
-      }
-      __syncwarp();
-      return true;
-    };
-    bool ok = warp_wait<true>(rf_smem_u32(&sm.bar_q), 0, abort);
-    if (ok) ok = issue_qk(0);
-    if (ok && nv > 1) ok = issue_qk(1);
-    for (int j = 0; ok && j < nv; ++j) {
-      const int w = j & 1, i = j >> 1, st = j % kStagesV;
-      const uint64_t dv = dv0 + (uint64_t)(st * (kVTileBytes >> 4));
-      // O_w += P_j V_j in two halves of the key rows: the first as soon as the
-      // softmax has stored the first 64 columns of P_j, the second when all of
-      // P_j is in.
-      if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_half[w]), i & 1, abort)) { ok = false; break; }
-      if (!warp_wait<true>(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
-      tc_fence_after();
-      if (elect_one()) {
+        if (!warp_wait<true>(rf_smem_u32(&sm.bar_k_full[st]), (j / kStagesK) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
+          // S_j = Q K_j^T: every MMA takes a 32-byte slice of the reduction
+          // (16 bf16/fp16 or 32 E4M3 elements).
+          const uint64_t dk = dk0 + (uint64_t)(st * (kQkTileBytes >> 4));
+          const uint32_t d_s = tmem;
 #pragma unroll
-        for (int kk = 0; kk < RF_BLOCK / 32; ++kk)
-          mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)),
-                 idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < (int)(kQkTileBytes / RF_BLOCK / 32); ++kk) {
+            const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+            if constexpr (kQk8)
+              mma_ss_f8(d_s, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(d_s, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(rf_smem_u32(&sm.bar_s_full[j & 1]));
+          tc_commit(rf_smem_u32(&sm.bar_k_empty[st]));
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_full[w]), i & 1, abort)) { ok = false; break; }
-      tc_fence_after();
-      if (elect_one()) {
+    } else {
+      // precision "mxfp4": P and V are f16 whatever the input type
+      const uint32_t idesc_pv = umma_idesc_f16(kMx ? 0u : fmt, 128, D, 1);
+      const uint64_t dv0 = umma_desc_sw128(rf_smem_u32(sm.v[0]), kBoxBytes, 1024);
+      for (int j = 0; ok && j < nv; ++j) {
+        const int b = j & 1, st = j % kStagesV;
+        const uint32_t ph = (j >> 1) & 1;
+        const uint64_t dv = dv0 + (uint64_t)(st * (kVTileBytes >> 4));
+        const uint32_t a_p = tmem + kPCol + (uint32_t)(b * 64);  // P_j
+        const uint32_t d_o = tmem + kOCol + (uint32_t)(b * 128);  // O_b
+        // O += P_j V_j in two halves of the key rows: the first as soon as the
+        // softmax has stored the first 64 columns of P_j, the second when all
+        // of P_j is in.
+        if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_half[b]), ph, abort)) { ok = false; break; }
+        if (!warp_wait<true>(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = RF_BLOCK / 32; kk < RF_BLOCK / 16; ++kk)
-          mma_ts(tmem + 256 + w * 128, tmem + w * 128 + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)),
-                 idesc_pv, 1u);
-        tc_commit(rf_smem_u32(&sm.bar_v_empty[st]));
+          for (int kk = 0; kk < RF_BLOCK / 32; ++kk)
+            mma_ts(d_o, a_p + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), idesc_pv,
+                   (j >= 2 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+        if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_full[b]), ph, abort)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = RF_BLOCK / 32; kk < RF_BLOCK / 16; ++kk)
+            mma_ts(d_o, a_p + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), idesc_pv, 1u);
+          tc_commit(rf_smem_u32(&sm.bar_v_empty[st]));
+          tc_commit(rf_smem_u32(&sm.bar_pv_done[b]));
+        }
+        __syncwarp();
       }
-      __syncwarp();
-      if (j + 2 < nv && !issue_qk(j + 2)) { ok = false; break; }
     }
     if (!ok && lane == 0) record_timeout(abort, a.status, 2);
-    // Every MMA issued so far (all of them, on the normal path) completes
-    // before bar_final, which gates the epilogue, and before bar_drain,
-    // which gates freeing TMEM.
+    // Every MMA this warp issued (all of them, on the normal path) completes
+    // before bar_final, which gates the epilogue, and before bar_drain, which
+    // gates freeing TMEM; both barriers count the two issuing warps.
     if (elect_one()) {
       tc_commit(rf_smem_u32(&sm.bar_final));
       tc_commit(rf_smem_u32(&sm.bar_drain));
@@ -571,10 +601,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = warp >> 2;                 // this warpgroup's block parity
     const int row = (warp & 3) * 32 + lane;   // query row = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    const uint32_t s_col = wg * 128, o_col = 256 + wg * 128;
     // precision "mix": S_j carries the E4M3 scales of the Q block and of K block j
     const float sl2_q = kQk8 ? a.sl2 * a.q_scale[(size_t)n * g.t_qblk + tb] : a.sl2;
     const int my_blocks = (nv + 1 - wg) >> 1;  // blocks j < nv with j % 2 == wg
+    const uint32_t scol = lane_base;                          // S_j (both groups in turn)
+    const uint32_t pcol = lane_base + kPCol + (uint32_t)(wg * 64);
+    const uint32_t ocol = lane_base + kOCol + (uint32_t)(wg * 128);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int i = 0; i < my_blocks; ++i) {
@@ -591,13 +623,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;
       }
       const float sl2 = kQk8 ? sl2_q * sm.kscale[j] : sl2_q;
-      const uint32_t scol = lane_base + s_col;
       uint32_t sr[128];
       tmem_ld32(scol, sr);
       tmem_ld32(scol + 32, sr + 32);
       tmem_ld32(scol + 64, sr + 64);
       tmem_ld32(scol + 96, sr + 96);
       tmem_wait_ld();
+      // S_j is in registers: the score buffer may take S_{j+1}.
+      tc_fence_before();
+      mbar_arrive(rf_smem_u32(&sm.bar_s_free));
       float gm[4];
       float mx_t;
       if constexpr (kMx) {
@@ -607,6 +641,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         mx_t = (vr == RF_BLOCK ? row_max<true>(sr, vr) : row_max<false>(sr, vr)) * sl2;
       }
+      // P buffer wg and O_wg still serve P_{j-2} V_{j-2} until that product is
+      // complete (issued long ago; normally done).
+      if (i > 0) {
+        if (!warp_wait(rf_smem_u32(&sm.bar_pv_done[wg]), (i - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+      }
       const bool rescale = __any_sync(0xffffffffu, mx_t > m_run + kRescaleThreshold);
       if (rescale) {
         // mxfp4: the running max stays an integer
@@ -615,47 +655,64 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_run *= alpha;
         m_run = m_new;
         if (i > 0) {
-          // O_w holds this group's earlier P V products and is at rest: S_j
-          // was issued after the last of them, and S_j is complete.  Rescale
-          // it before any of P_j is released to the MMA warp.
+          // O_wg holds this group's earlier P V products and is at rest (its
+          // last one is complete, see above).  Rescale it before any of P_j is
+          // released.
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(lane_base + o_col + c0, o);
+            tmem_ld32(ocol + c0, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(lane_base + o_col + c0, o);
+            tmem_st32(ocol + c0, o);
           }
         }
       }
-      // P_j over the first 64 columns of S_j (already in registers), one half
-      // at a time: the first half is released to the MMA warp while the second
-      // is being computed.
+      // P_j in four quarters of 32 columns (16 TMEM columns each): the first
+      // two are released to the MMA warp while the other two are being
+      // computed.
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       float lsum = 0.f;
-      uint32_t pk[32];
       if constexpr (kMx) {
-        if (vr == RF_BLOCK) half_row_exp_mx<true>(sr, 0, vr, sl2, m_run, gm, pk, lsum);
-        else                half_row_exp_mx<false>(sr, 0, vr, sl2, m_run, gm, pk, lsum);
+        if (vr == RF_BLOCK) {
+          group_exp_mx<true>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
+          group_exp_mx<true>(sr, 32, vr, sl2, m_run, gm[1], pcol + 16, lsum);
+        } else {
+          group_exp_mx<false>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
+          group_exp_mx<false>(sr, 32, vr, sl2, m_run, gm[1], pcol + 16, lsum);
+        }
       } else {
-        if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 0, vr, sl2, -m_run, pk, acc);
-        else                half_row_exp<kBf16, false>(sr, 0, vr, sl2, -m_run, pk, acc);
+        if (vr == RF_BLOCK) {
+          quarter_row_exp<kBf16, true>(sr, 0, vr, sl2, -m_run, pcol, acc);
+          quarter_row_exp<kBf16, true>(sr, 32, vr, sl2, -m_run, pcol + 16, acc);
+        } else {
+          quarter_row_exp<kBf16, false>(sr, 0, vr, sl2, -m_run, pcol, acc);
+          quarter_row_exp<kBf16, false>(sr, 32, vr, sl2, -m_run, pcol + 16, acc);
+        }
       }
-      tmem_st32(scol, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(rf_smem_u32(&sm.bar_p_half[wg]));
       if constexpr (kMx) {
-        if (vr == RF_BLOCK) half_row_exp_mx<true>(sr, 64, vr, sl2, m_run, gm + 2, pk, lsum);
-        else                half_row_exp_mx<false>(sr, 64, vr, sl2, m_run, gm + 2, pk, lsum);
+        if (vr == RF_BLOCK) {
+          group_exp_mx<true>(sr, 64, vr, sl2, m_run, gm[2], pcol + 32, lsum);
+          group_exp_mx<true>(sr, 96, vr, sl2, m_run, gm[3], pcol + 48, lsum);
+        } else {
+          group_exp_mx<false>(sr, 64, vr, sl2, m_run, gm[2], pcol + 32, lsum);
+          group_exp_mx<false>(sr, 96, vr, sl2, m_run, gm[3], pcol + 48, lsum);
+        }
         l_run += lsum;
       } else {
-        if (vr == RF_BLOCK) half_row_exp<kBf16, true>(sr, 64, vr, sl2, -m_run, pk, acc);
-        else                half_row_exp<kBf16, false>(sr, 64, vr, sl2, -m_run, pk, acc);
+        if (vr == RF_BLOCK) {
+          quarter_row_exp<kBf16, true>(sr, 64, vr, sl2, -m_run, pcol + 32, acc);
+          quarter_row_exp<kBf16, true>(sr, 96, vr, sl2, -m_run, pcol + 48, acc);
+        } else {
+          quarter_row_exp<kBf16, false>(sr, 64, vr, sl2, -m_run, pcol + 32, acc);
+          quarter_row_exp<kBf16, false>(sr, 96, vr, sl2, -m_run, pcol + 48, acc);
+        }
         l_run += acc_sum(acc);
       }
-      tmem_st32(scol + 32, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(rf_smem_u32(&sm.bar_p_full[wg]));
@@ -667,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.row_m[wg][row] = m_run;
     sm.row_l[wg][row] = l_run;
     softmax_bar_sync();
-    const bool have_o = ok && nv > 0 && warp_wait(rf_smem_u32(&sm.bar_final), 0, abort);
+    const bool have_o = nv > 0 && !*abort && warp_wait(rf_smem_u32(&sm.bar_final), 0, abort) && !*abort;
     const float m0 = sm.row_m[0][row], m1 = sm.row_m[1][row];
     const float l0 = sm.row_l[0][row], l1 = sm.row_l[1][row];
     const float m = fmaxf(m0, m1);
@@ -682,8 +739,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
     for (int c0 = wg * (D / 2); c0 < (wg + 1) * (D / 2); c0 += 32) {
       uint32_t o0[32], o1[32];
-      if (use0) tmem_ld32(lane_base + 256 + c0, o0);
-      if (use1) tmem_ld32(lane_base + 384 + c0, o1);
+      if (use0) tmem_ld32(lane_base + kOCol + c0, o0);
+      if (use1) tmem_ld32(lane_base + kOCol + 128 + c0, o1);
       if (use0 || use1) tmem_wait_ld();
       uint32_t w[16];
 #pragma unroll

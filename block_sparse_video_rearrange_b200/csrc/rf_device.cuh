@@ -179,6 +179,19 @@ __device__ __forceinline__ bool mbar_try_wait_poll(uint32_t bar, uint32_t parity
   return ok != 0;
 }
 
+// One non-blocking test of phase `parity` (mbarrier.test_wait).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for phase `parity` of barrier `bar` to complete, for at most
 // RF_WAIT_LIMIT_NS; gives up early once *abort is set.  Returns false when it
 // gave up (the caller records it and unwinds).  kPoll: poll without the
@@ -186,7 +199,11 @@ __device__ __forceinline__ bool mbar_try_wait_poll(uint32_t bar, uint32_t parity
 #define RF_WAIT_LIMIT_NS 1000000000ull
 template <bool kPoll = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+#ifdef RF_POLL_TEST_WAIT
+  auto test = [&]() { return kPoll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity); };
+#else
   auto test = [&]() { return kPoll ? mbar_try_wait_poll(bar, parity) : mbar_try_wait(bar, parity); };
+#endif
   if (test()) return true;
   const uint64_t t0 = rf_globaltimer();
 #pragma unroll 1
@@ -397,6 +414,37 @@ __device__ __forceinline__ float rf_max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// 2^x of two values at once, with the range reduction and polynomial of
+// rf_exp2_poly run as paired fp32 instructions (one f32x2 instruction per step
+// for both values): x = j + r with j = round(x) from the 1.5 * 2^23 shifter,
+// 2^r from the same degree-3 polynomial, 2^j added to the exponent field.
+// With t = x + 1.5 * 2^23 rounded to an integer, the bits of t are
+// 0x4B400000 + j, and (bits << 23) is j << 23 modulo 2^32 because the low nine
+// bits of 0x4B400000 are zero: one shift and one add reassemble the result.
+// Inputs are clamped at -125.5 as in rf_exp2_poly.
+__device__ __forceinline__ void rf_exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShifter = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kC1 = 0.6933164596557617f, kC2 = 0.24192412197589874f,
+                  kC3 = 0.054602622985839844f;
+  x0 = fmaxf(x0, -125.5f);
+  x1 = fmaxf(x1, -125.5f);
+  const uint64_t x = rf_f2(__float_as_uint(x0), __float_as_uint(x1));
+  const uint64_t sh = rf_f2(__float_as_uint(kShifter), __float_as_uint(kShifter));
+  const uint64_t nsh = rf_f2(__float_as_uint(-kShifter), __float_as_uint(-kShifter));
+  const uint64_t m1 = rf_f2(__float_as_uint(-1.0f), __float_as_uint(-1.0f));
+  const uint64_t t = rf_add2(x, sh);                 // j in the low mantissa bits
+  const uint64_t r = rf_fma2(rf_add2(t, nsh), m1, x);  // x - j, exact
+  uint64_t p = rf_fma2(rf_f2(__float_as_uint(kC3), __float_as_uint(kC3)), r,
+                       rf_f2(__float_as_uint(kC2), __float_as_uint(kC2)));
+  p = rf_fma2(p, r, rf_f2(__float_as_uint(kC1), __float_as_uint(kC1)));
+  p = rf_fma2(p, r, rf_f2(__float_as_uint(1.0f), __float_as_uint(1.0f)));
+  uint32_t t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+  y0 = __uint_as_float(p0 + (t0 << 23));
+  y1 = __uint_as_float(p1 + (t1 << 23));
 }
 
 // Two floats to packed 16-bit (lo = a, hi = b), round to nearest even.
