@@ -63,9 +63,9 @@ def parse():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--workload", default="aligned", choices=sorted(WORKLOAD_DESC))
     ap.add_argument("--sparsity", type=float, default=None)
-    ap.add_argument("--precision", default="native", choices=["native", "mix", "mxfp4"],
+    ap.add_argument("--precision", default="native", choices=["native", "mix", "fp8", "mxfp4"],
                     help="kernel precision (mix: E4M3 Q K^T with per-block scales, 16-bit P V; "
-                         "mxfp4: MXFP4 operands with UOS scaling and PNQ)")
+                         "fp8: E4M3 for P V as well; mxfp4: MXFP4 operands with UOS scaling and PNQ)")
     ap.add_argument("--order", default="tile", choices=["tile", "frame_pair"],
                     help="token order of the aligned video (frame_pair: frames paired into 2x8x8 blocks)")
     ap.add_argument("--mode", default="auto", choices=["auto", "plain", "ulysses", "independent"],
@@ -226,7 +226,10 @@ def algorithmic_bytes(plan, elem=2):
     sel = 4 * t * n * m + 4 * t * n
     inv = 2 * rows * plan.n1 * plan.d * elem
     # precision "mix": the rearrange also writes one-byte copies of Q' and K' and their scales
-    quant = rows * (plan.n1 + plan.n2) * plan.d + 4 * t * (plan.n1 + plan.n2) if plan.precision == "mix" else 0
+    quant = rows * (plan.n1 + plan.n2) * plan.d + 4 * t * (plan.n1 + plan.n2) if plan.precision in ("mix", "fp8") else 0
+    # precision "fp8": and the transposed one-byte copy of V' (whole blocks) with its exponents
+    if plan.precision == "fp8":
+        quant += plan.n2 * t * 128 * plan.d + 4 * t * plan.n2
     # precision "mxfp4": 16-bit MXFP4-rounded copies of Q', K' and V'
     if plan.precision == "mxfp4":
         quant = rows * (plan.n1 + 2 * plan.n2) * plan.d * 2
@@ -644,6 +647,15 @@ def main():
                 alt = 1.0 / (0.5 / f8 + 0.5 / bf)
                 extra_roof = {"fp8_gemm_tflops_measured_here": round(f8, 1),
                               "peak_with_measured_fp8": round(alt, 1), "frac_with_measured_fp8": round(achieved / alt, 4)}
+        if args.precision == "fp8":
+            # both products at the fp8 rate: 2x the measured 16-bit rate (nominal 4.5 / 2.25)
+            bf = peak
+            peak = round(bf * 2.0, 1)
+            peak_note += "; fp8: QK^T and PV at 2x (fp8, nominal ratio x measured bf16)"
+            f8 = measure_fp8_gemm_tflops(dev)
+            if f8:
+                extra_roof = {"fp8_gemm_tflops_measured_here": round(f8, 1), "peak_with_measured_fp8": round(f8, 1),
+                              "frac_with_measured_fp8": round(achieved / f8, 4)}
         if args.precision == "mxfp4":
             peak_note += "; mxfp4: both products run on the 16-bit tensor cores -> 1x"
         front_bytes, inv_bytes = algorithmic_bytes(plan)
@@ -663,12 +675,15 @@ def main():
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": {"mix": "e4m3+", "mxfp4": "mxfp4 on "}.get(args.precision, "") + ("bf16" if w.dtype == "bf16" else "fp16"),
+            "dtype": {"mix": "e4m3+", "fp8": "e4m3 (from ", "mxfp4": "mxfp4 on "}.get(args.precision, "")
+                     + ("bf16" if w.dtype == "bf16" else "fp16") + (")" if args.precision == "fp8" else ""),
             "data": "synthetic (seeded smooth-field + noise per 8x8 cell; no real activations available)",
             "config": {"workload": WORKLOAD_DESC[w.name.split("@")[0]] + (f" [reduced to {w.n1} heads]" if args.heads else ""),
                        "sparsity": w.sparsity,
                        **({"token_order": args.order} if args.order != "tile" else {}),
                        **({"precision": "mix (E4M3 QK^T, 16-bit PV)"} if args.precision == "mix" else {}),
+                       **({"precision": "fp8 (E4M3 QK^T and PV; V on power-of-two block scales)"}
+                          if args.precision == "fp8" else {}),
                        **({"block_shape": "128 x 64 (attention on the 64-row halves of the step's 128-row "
                                           "selection, expanded once after warm-up)"} if args.block_kv == 64 else {}),
                        **({"precision": "mxfp4 (UOS Qmax 7.25, PNQ)"} if args.precision == "mxfp4" else {}),

@@ -93,14 +93,16 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy rescale while growth <= 256x
 
-// kQk8: Q and K tiles hold E4M3 codes (precision "mix"), one byte per element.
-template <int D, bool kQk8>
+// kQk8: Q and K tiles hold E4M3 codes (precisions "mix" and "fp8"), one byte
+// per element.  kPv8: V tiles hold E4M3 codes stored transposed (D rows of 128
+// keys, precision "fp8").
+template <int D, bool kQk8, bool kPv8 = false>
 struct __align__(1024) AttnSmem {
   static constexpr int kQkTileBytes = RF_BLOCK * D * (kQk8 ? 1 : 2);
-  static constexpr int kVTileBytes = RF_BLOCK * D * 2;   // 128 rows x D x 16-bit
+  static constexpr int kVTileBytes = RF_BLOCK * D * (kPv8 ? 1 : 2);
   // V ring: V_{j+kStagesV} is requested as soon as O += P_j V_j is done.  The
   // one-byte Q and K tiles leave room for a third V stage.
-  static constexpr int kStagesV = kQk8 ? 3 : 2;
+  static constexpr int kStagesV = kPv8 ? 4 : (kQk8 ? 3 : 2);
   uint8_t q[kQkTileBytes];
   uint8_t k[kStagesK][kQkTileBytes];
   uint8_t v[kStagesV][kVTileBytes];
@@ -123,6 +125,8 @@ struct __align__(1024) AttnSmem {
   // 128-key tile each (b = -1: none), hence two spare entries
   int list[RF_MAX_KV_LIST + 2];
   float kscale[kQk8 ? RF_MAX_KV_LIST : 1];  // dequantization scale of K block list[j]
+  int vexp[kPv8 ? RF_MAX_KV_LIST : 1];      // power-of-two exponent of V block list[j]
+  int vexp_max;                             // the largest of them
 };
 
 struct AttnArgs {
@@ -131,8 +135,9 @@ struct AttnArgs {
   const int32_t* sel_num;
   uint16_t* o_r;
   uint32_t* status;
-  const float* q_scale;  // precision "mix": E4M3 scales [n1][t_qblk] and [n2][t_qblk]
+  const float* q_scale;  // precisions "mix" and "fp8": E4M3 scales [n1][t_qblk] and [n2][t_qblk]
   const float* k_scale;
+  const int32_t* v_exp;  // precision "fp8": V exponents [n2][t_qblk]
   float sl2;  // scale * log2(e)
 };
 
@@ -207,6 +212,51 @@ __device__ __forceinline__ void quarter_row_exp(const uint32_t* sr, int c0, int 
     pk[c >> 1] = rf_pack2<kBf16>(p0, p1);
   }
   tmem_st16(p_addr, pk);
+}
+
+// Precision "fp8": p = 2^(s * sl2 - m) for the 32 scores c0 .. c0 + 31 of a row
+// (the first vr valid; pairs selected by kEmuPairMask from the FMA-pipe
+// polynomial).  The fp32 values go to the row sum (acc, as in
+// quarter_row_exp); p * down, down = 2^-shift the power-of-two step from this
+// V block's exponent to the row's largest, is rounded to E4M3 (nearest even,
+// saturating) and stored four codes per column, the lowest key in the lowest
+// byte, to the 8 TMEM columns at p_addr.
+template <bool kFull>
+__device__ __forceinline__ void quarter_row_exp_f8(const uint32_t* sr, int c0, int vr, float sl2, float neg_m,
+                                                   float down, uint32_t p_addr, uint64_t* acc) {
+  const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
+  const uint64_t negm2 = rf_f2(__float_as_uint(neg_m), __float_as_uint(neg_m));
+  const uint64_t down2 = rf_f2(__float_as_uint(down), __float_as_uint(down));
+  uint32_t pk[8];
+#pragma unroll
+  for (int c = 0; c < 32; c += 4) {
+    uint32_t half[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cc = c + 2 * h;
+      float x0, x1, p0, p1;
+      rf_f2_split(rf_fma2(rf_f2(sr[c0 + cc], sr[c0 + cc + 1]), sl2x2, negm2), x0, x1);
+      if ((kEmuPairMask >> ((cc >> 1) & 15)) & 1u) {
+        rf_exp2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = rf_ex2(x0);
+        p1 = rf_ex2(x1);
+      }
+      if (!kFull) {
+        p0 = c0 + cc < vr ? p0 : 0.f;
+        p1 = c0 + cc + 1 < vr ? p1 : 0.f;
+      }
+      const uint64_t pp = rf_f2(__float_as_uint(p0), __float_as_uint(p1));
+      acc[(cc >> 1) & 3] = rf_add2(acc[(cc >> 1) & 3], pp);
+      float y0, y1;
+      rf_f2_split(rf_mul2(pp, down2), y0, y1);
+      unsigned short two;
+      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(y1), "f"(y0));
+      half[h] = two;
+    }
+    pk[c >> 2] = half[0] | (half[1] << 16);
+  }
+  tmem_st8(p_addr, pk);
 }
 
 // Maxima of the four 32-column groups of a row of raw scores (the first vr
@@ -284,17 +334,17 @@ __device__ __forceinline__ float acc_sum(const uint64_t* acc) {
   return s;
 }
 
-template <int D, bool kBf16, bool kQk8, bool kMx>
+template <int D, bool kBf16, bool kQk8, bool kMx, bool kPv8>
 __global__ void __launch_bounds__(kThreads, 1)
     rf_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs a) {
-  using Smem = AttnSmem<D, kQk8>;
+  using Smem = AttnSmem<D, kQk8, kPv8>;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   // Tiles are read as 128-byte-wide swizzle boxes of 128 rows.
   constexpr int kQkBoxes = D * (kQk8 ? 1 : 2) / 128;  // boxes per Q or K tile
-  constexpr int kVBoxes = D * 2 / 128;                // boxes per V tile
+  constexpr int kVBoxes = kPv8 ? 1 : D * 2 / 128;     // boxes per V tile
   constexpr uint32_t kQkTileBytes = Smem::kQkTileBytes;
   constexpr uint32_t kVTileBytes = Smem::kVTileBytes;
   constexpr int kStagesV = Smem::kStagesV;
@@ -366,6 +416,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.list[c] = v;
     if constexpr (kQk8)
       if (v >= 0 && v < nkv) sm.kscale[c] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
+    if constexpr (kPv8)
+      if (v >= 0 && v < nkv) sm.vexp[c] = a.v_exp[(size_t)gk * g.t_qblk + s.qblk_off + v];
   }
   __syncthreads();
   if (warp == 0) {
@@ -374,20 +426,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     // below its own read position, and every lane reads before the ballot.
     int bad = (lane == 0 && num != num_raw) ? 1 : 0;
     int cnt = 0;
+    int vmax = -127;  // precision "fp8": the largest V exponent of the row
     const uint32_t lt = (1u << lane) - 1u;
     for (int c0 = 0; c0 < num; c0 += 32) {
       const int c = c0 + lane;
       const int v = c < num ? sm.list[c] : -1;
       float ks = 0.f;
       if constexpr (kQk8) ks = c < num ? sm.kscale[c] : 0.f;
+      int ve = -127;
+      if constexpr (kPv8) ve = c < num ? sm.vexp[c] : -127;
       const bool ok = c < num && v >= 0 && v < nkv;
       if (c < num && v != -1 && !ok) ++bad;
       const uint32_t ball = __ballot_sync(0xffffffffu, ok);
       if (ok) {
         sm.list[cnt + __popc(ball & lt)] = v;
         if constexpr (kQk8) sm.kscale[cnt + __popc(ball & lt)] = ks;
+        if constexpr (kPv8) {
+          sm.vexp[cnt + __popc(ball & lt)] = ve;
+          vmax = max(vmax, ve);
+        }
       }
       cnt += __popc(ball);
+    }
+    if constexpr (kPv8) {
+      vmax = __reduce_max_sync(0xffffffffu, vmax);
+      if (lane == 0) sm.vexp_max = vmax;
     }
     bad = __reduce_add_sync(0xffffffffu, bad);
     int units = cnt;  // tiles of 128 keys
@@ -466,7 +529,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t bar = rf_smem_u32(&full[st]);
       mbar_arrive_expect_tx(bar, tile_bytes);
-      if (!kv64) {
+      if (kPv8 && !is_k) {
+        // transposed E4M3 V block: D rows of 128 keys, one 128-byte box
+        tma_load_3d(rf_smem_u32(tiles + st * tile_bytes), map, bar, 0, 0,
+                    gk * g.t_qblk + s.qblk_off + sm.list[j]);
+      } else if (!kv64) {
         int r0, nr;
         rf_block_span(s, sm.list[j], r0, nr);
         coords(g.n2, gk, r0, c1, c2);
@@ -543,9 +610,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
     } else {
-      // precision "mxfp4": P and V are f16 whatever the input type
-      const uint32_t idesc_pv = umma_idesc_f16(kMx ? 0u : fmt, 128, D, 1);
-      const uint64_t dv0 = umma_desc_sw128(rf_smem_u32(sm.v[0]), kBoxBytes, 1024);
+      // precision "mxfp4": P and V are f16 whatever the input type; precision
+      // "fp8": both E4M3 (format 0 of kind::f8f6f4), V transposed, so K-major
+      const uint32_t idesc_pv = umma_idesc_f16(kMx || kPv8 ? 0u : fmt, 128, D, kPv8 ? 0u : 1u);
+      const uint64_t dv0 = kPv8 ? umma_desc_sw128(rf_smem_u32(sm.v[0]), 16, 1024)
+                                : umma_desc_sw128(rf_smem_u32(sm.v[0]), kBoxBytes, 1024);
       for (int j = 0; ok && j < nv; ++j) {
         const int b = j & 1, st = j % kStagesV;
         const uint32_t ph = (j >> 1) & 1;
@@ -559,18 +628,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!warp_wait<true>(rf_smem_u32(&sm.bar_v_full[st]), (j / kStagesV) & 1, abort)) { ok = false; break; }
         tc_fence_after();
         if (elect_one()) {
+          if constexpr (kPv8) {
+            // 32 keys per MMA: 8 TMEM columns of P', 32 bytes of each V row
 #pragma unroll
-          for (int kk = 0; kk < RF_BLOCK / 32; ++kk)
-            mma_ts(d_o, a_p + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), idesc_pv,
-                   (j >= 2 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ts_f8(d_o, a_p + kk * 8, dv + (uint32_t)(kk * 2), idesc_pv, (j >= 2 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < RF_BLOCK / 32; ++kk)
+              mma_ts(d_o, a_p + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), idesc_pv,
+                     (j >= 2 || kk > 0) ? 1u : 0u);
+          }
         }
         __syncwarp();
         if (!warp_wait<true>(rf_smem_u32(&sm.bar_p_full[b]), ph, abort)) { ok = false; break; }
         tc_fence_after();
         if (elect_one()) {
+          if constexpr (kPv8) {
 #pragma unroll
-          for (int kk = RF_BLOCK / 32; kk < RF_BLOCK / 16; ++kk)
-            mma_ts(d_o, a_p + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), idesc_pv, 1u);
+            for (int kk = 2; kk < 4; ++kk) mma_ts_f8(d_o, a_p + kk * 8, dv + (uint32_t)(kk * 2), idesc_pv, 1u);
+          } else {
+#pragma unroll
+            for (int kk = RF_BLOCK / 32; kk < RF_BLOCK / 16; ++kk)
+              mma_ts(d_o, a_p + kk * 8, dv + (uint32_t)(kk * (2048 >> 4)), idesc_pv, 1u);
+          }
           tc_commit(rf_smem_u32(&sm.bar_v_empty[st]));
           tc_commit(rf_smem_u32(&sm.bar_pv_done[b]));
         }
@@ -604,6 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // precision "mix": S_j carries the E4M3 scales of the Q block and of K block j
     const float sl2_q = kQk8 ? a.sl2 * a.q_scale[(size_t)n * g.t_qblk + tb] : a.sl2;
     const int my_blocks = (nv + 1 - wg) >> 1;  // blocks j < nv with j % 2 == wg
+    const int vexp_max = kPv8 ? sm.vexp_max : 0;
     const uint32_t scol = lane_base;                          // S_j (both groups in turn)
     const uint32_t pcol = lane_base + kPCol + (uint32_t)(wg * 64);
     const uint32_t ocol = lane_base + kOCol + (uint32_t)(wg * 128);
@@ -623,6 +705,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;
       }
       const float sl2 = kQk8 ? sl2_q * sm.kscale[j] : sl2_q;
+      // precision "fp8": P' = P * 2^-(exp_max - exp_j) for the P V product
+      float down = 1.f;
+      if constexpr (kPv8) {
+        const int shift = vexp_max - sm.vexp[j];
+        down = shift <= 126 ? rf_pow2(-shift) : 0.f;
+      }
       uint32_t sr[128];
       tmem_ld32(scol, sr);
       tmem_ld32(scol + 32, sr + 32);
@@ -682,6 +770,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           group_exp_mx<false>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
           group_exp_mx<false>(sr, 32, vr, sl2, m_run, gm[1], pcol + 16, lsum);
         }
+      } else if constexpr (kPv8) {
+        if (vr == RF_BLOCK) {
+          quarter_row_exp_f8<true>(sr, 0, vr, sl2, -m_run, down, pcol, acc);
+          quarter_row_exp_f8<true>(sr, 32, vr, sl2, -m_run, down, pcol + 8, acc);
+        } else {
+          quarter_row_exp_f8<false>(sr, 0, vr, sl2, -m_run, down, pcol, acc);
+          quarter_row_exp_f8<false>(sr, 32, vr, sl2, -m_run, down, pcol + 8, acc);
+        }
       } else {
         if (vr == RF_BLOCK) {
           quarter_row_exp<kBf16, true>(sr, 0, vr, sl2, -m_run, pcol, acc);
@@ -703,6 +799,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           group_exp_mx<false>(sr, 96, vr, sl2, m_run, gm[3], pcol + 48, lsum);
         }
         l_run += lsum;
+      } else if constexpr (kPv8) {
+        if (vr == RF_BLOCK) {
+          quarter_row_exp_f8<true>(sr, 64, vr, sl2, -m_run, down, pcol + 16, acc);
+          quarter_row_exp_f8<true>(sr, 96, vr, sl2, -m_run, down, pcol + 24, acc);
+        } else {
+          quarter_row_exp_f8<false>(sr, 64, vr, sl2, -m_run, down, pcol + 16, acc);
+          quarter_row_exp_f8<false>(sr, 96, vr, sl2, -m_run, down, pcol + 24, acc);
+        }
+        l_run += acc_sum(acc);
       } else {
         if (vr == RF_BLOCK) {
           quarter_row_exp<kBf16, true>(sr, 64, vr, sl2, -m_run, pcol + 32, acc);
@@ -731,7 +836,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float a0 = l0 > 0.f ? rf_ex2(m0 - m) : 0.f;
     const float a1 = l1 > 0.f ? rf_ex2(m1 - m) : 0.f;
     const float l = a0 * l0 + a1 * l1;
-    const float inv = l > 0.f ? 1.0f / l : 0.f;
+    // precision "fp8": P V ran on P * 2^-exp_max times the V codes
+    const float vsc = kPv8 ? (vexp_max >= -126 ? rf_pow2(vexp_max) : 0.f) : 1.f;
+    const float inv = l > 0.f ? vsc / l : 0.f;
     const float s0 = a0 * inv, s1 = a1 * inv;
     const bool use0 = have_o && nv > 0, use1 = have_o && nv > 1;
     uint16_t* dst = a.o_r + rf_row_offset(g, s, g.n1, n, q_r0 + min(row, q_rows - 1));
@@ -843,14 +950,32 @@ rf_status_t make_map(CUtensorMap* m, const rf_plan* p, const void* base, int hea
   return RF_OK;
 }
 
-template <int D, bool kBf16, bool kQk8, bool kMx = false>
+// Tensor map over precision "fp8"'s transposed E4M3 V codes, uint8
+// [n2 * t_qblk][D][128]: one 128 x 128-byte box (128-byte swizzle) per block.
+rf_status_t make_map_v8(CUtensorMap* m, const rf_plan* p, const void* base) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return rf_fail(RF_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const RfGeomDev& g = p->g;
+  const cuuint64_t d = (cuuint64_t)g.d;
+  cuuint64_t dims[3] = {(cuuint64_t)RF_BLOCK, d, (cuuint64_t)g.n2 * (cuuint64_t)g.t_qblk};
+  cuuint64_t strides[2] = {(cuuint64_t)RF_BLOCK, (cuuint64_t)RF_BLOCK * d};
+  cuuint32_t box[3] = {(cuuint32_t)RF_BLOCK, (cuuint32_t)g.d, 1}, estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return rf_fail(RF_ERR_CUDA, "cuTensorMapEncodeTiled (fp8 V) failed: " + std::to_string((int)r));
+  return RF_OK;
+}
+
+template <int D, bool kBf16, bool kQk8, bool kMx = false, bool kPv8 = false>
 rf_status_t launch_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const AttnArgs& args, unsigned grid, cudaStream_t st) {
-  size_t smem = sizeof(AttnSmem<D, kQk8>) + 1024;
+  size_t smem = sizeof(AttnSmem<D, kQk8, kPv8>) + 1024;
   // D = 64 tiles are small: ask for enough shared memory that one CTA holds
   // an SM, since each CTA takes all 512 TMEM columns.
   if (smem < 120 * 1024) smem = 120 * 1024;
-  auto kern = rf_attn_kernel<D, kBf16, kQk8, kMx>;
+  auto kern = rf_attn_kernel<D, kBf16, kQk8, kMx, kPv8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return rf_check_launch("cudaFuncSetAttribute(rf_attn_kernel)");
@@ -881,7 +1006,8 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   rf_status_t s;
   // precision "mix": Q K^T reads the E4M3 copies rf_rearrange wrote into ws;
   // precision "mxfp4": every operand reads the MXFP4 copies in ws (V as f16).
-  const bool mix = p->precision == RF_PRECISION_MIX;
+  const bool fp8 = p->precision == RF_PRECISION_FP8;
+  const bool mix = p->precision == RF_PRECISION_MIX || fp8;   // E4M3 Q and K
   const bool mx = p->precision == RF_PRECISION_MXFP4;
   char* w = static_cast<char*>(ws);
   const void* qsrc = mix ? static_cast<const void*>(w + p->off_q8) : mx ? static_cast<const void*>(w + p->off_qx) : q_r;
@@ -891,7 +1017,11 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   if ((s = make_map(&mq, p, qsrc, g.n1, qk_elem)) != RF_OK) return s;
   const int kv_box = g.block_kv == 64 ? 64 : RF_BLOCK;
   if ((s = make_map(&mk, p, ksrc, g.n2, qk_elem, kv_box)) != RF_OK) return s;
-  if ((s = make_map(&mv, p, vsrc, g.n2, mx ? kElemF16 : kElemPlan, kv_box)) != RF_OK) return s;
+  if (fp8) {
+    if ((s = make_map_v8(&mv, p, w + p->off_v8)) != RF_OK) return s;
+  } else if ((s = make_map(&mv, p, vsrc, g.n2, mx ? kElemF16 : kElemPlan, kv_box)) != RF_OK) {
+    return s;
+  }
   AttnArgs args;
   args.g = g;
   args.sel_idx = sel_idx;
@@ -900,9 +1030,13 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   args.status = reinterpret_cast<uint32_t*>(w + p->off_status);
   args.q_scale = mix ? reinterpret_cast<const float*>(w + p->off_qs) : nullptr;
   args.k_scale = mix ? reinterpret_cast<const float*>(w + p->off_ks) : nullptr;
+  args.v_exp = fp8 ? reinterpret_cast<const int32_t*>(w + p->off_vexp) : nullptr;
   args.sl2 = scale * kLog2e;
   const bool bf = p->dtype == RF_BF16;
   if (g.d == 128) {
+    if (fp8)
+      return bf ? launch_t<128, true, true, false, true>(mq, mk, mv, args, (unsigned)grid, st)
+                : launch_t<128, false, true, false, true>(mq, mk, mv, args, (unsigned)grid, st);
     if (mix)
       return bf ? launch_t<128, true, true>(mq, mk, mv, args, (unsigned)grid, st)
                 : launch_t<128, false, true>(mq, mk, mv, args, (unsigned)grid, st);

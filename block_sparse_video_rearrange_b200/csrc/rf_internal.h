@@ -58,6 +58,7 @@ struct rf_plan {
   rf_token_order_t token_order;
   int64_t off_q8, off_k8, off_qs, off_ks;  // RF_PRECISION_MIX workspace regions, else -1
   int64_t off_qx, off_kx, off_vx;          // RF_PRECISION_MXFP4 workspace regions, else -1
+  int64_t off_v8, off_vexp;                // RF_PRECISION_FP8: transposed E4M3 V' and its exponents
   int64_t off_quant;                       // first precision-specific region (ws_bytes if none)
   int64_t kept_flops_upper;
 };

@@ -130,10 +130,8 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   if (opt.precision != RF_PRECISION_NATIVE && opt.precision != RF_PRECISION_MIX &&
       opt.precision != RF_PRECISION_FP8 && opt.precision != RF_PRECISION_MXFP4)
     return rf_fail(RF_ERR_INVALID_ARG, "unknown precision");
-  if (opt.precision == RF_PRECISION_FP8)
-    return rf_fail(RF_ERR_UNSUPPORTED, "precision fp8 (FP8 P V) is not built; use mix");
-  if (opt.precision == RF_PRECISION_MIX && d != 128)
-    return rf_fail(RF_ERR_UNSUPPORTED, "precision mix is built for head dim 128 only");
+  if ((opt.precision == RF_PRECISION_MIX || opt.precision == RF_PRECISION_FP8) && d != 128)
+    return rf_fail(RF_ERR_UNSUPPORTED, "precisions mix and fp8 are built for head dim 128 only");
   const rf_token_order_t order = (rf_token_order_t)opt.token_order;
   if (layout != RF_LAYOUT_BNSD && layout != RF_LAYOUT_TND)
     return rf_fail(RF_ERR_INVALID_ARG, "layout must be BNSD or TND");
@@ -254,8 +252,9 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   p->token_order = order;
   p->off_q8 = p->off_k8 = p->off_qs = p->off_ks = -1;
   p->off_qx = p->off_kx = p->off_vx = -1;
+  p->off_v8 = p->off_vexp = -1;
   p->off_quant = off;
-  if (p->precision == RF_PRECISION_MIX) {
+  if (p->precision == RF_PRECISION_MIX || p->precision == RF_PRECISION_FP8) {
     p->off_q8 = off;
     off = align_up(off + p->rows_total * n1 * d, 256);
     p->off_k8 = off;
@@ -263,6 +262,16 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
     p->off_qs = off;
     off = align_up(off + (int64_t)n1 * qblk * 4, 256);
     p->off_ks = off;
+    off = align_up(off + (int64_t)n2 * qblk * 4, 256);
+  }
+  // RF_PRECISION_FP8 also: E4M3 codes of V' stored transposed per block
+  // ([n2][t_qblk][d][128]: the 128 keys of one column contiguous, the layout a
+  // K-major B operand of P V needs) and their power-of-two exponents (int32
+  // [n2][t_qblk]).
+  if (p->precision == RF_PRECISION_FP8) {
+    p->off_v8 = off;
+    off = align_up(off + (int64_t)n2 * qblk * RF_BLOCK * d, 256);
+    p->off_vexp = off;
     off = align_up(off + (int64_t)n2 * qblk * 4, 256);
   }
   // RF_PRECISION_MXFP4: MXFP4-rounded 16-bit copies of Q', K', V' (layouts of
@@ -303,6 +312,8 @@ rf_status_t rf_plan_info(const rf_plan_t* p, rf_plan_info_t* out) {
   out->ws_q_mx = p->off_qx;
   out->ws_k_mx = p->off_kx;
   out->ws_v_mx = p->off_vx;
+  out->ws_v8 = p->off_v8;
+  out->ws_v_exp = p->off_vexp;
   return RF_OK;
 }
 
@@ -378,6 +389,21 @@ rf_status_t rf_quantize_mx(const rf_plan_t* p, const void* q_r, const void* k_r,
   if (st != RF_OK) return st;
   if ((st = rf_require_device()) != RF_OK) return st;
   return rf_launch_quantize(p, q_r, k_r, v_r, ws, (cudaStream_t)stream);
+}
+
+rf_status_t rf_quantize(const rf_plan_t* p, const void* q_r, const void* k_r, const void* v_r,
+                        void* ws, size_t ws_bytes, rf_stream_t stream) {
+  g_last_error.clear();
+  if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
+  if (p->precision == RF_PRECISION_NATIVE)
+    return rf_fail(RF_ERR_INVALID_ARG, "a native-precision plan has no quantized copies");
+  const bool need_v = p->precision != RF_PRECISION_MIX;
+  if (!q_r || !k_r || !aligned16(q_r) || !aligned16(k_r) || (need_v && (!v_r || !aligned16(v_r))))
+    return rf_fail(RF_ERR_INVALID_ARG, "inputs must be non-null and 16-byte aligned");
+  rf_status_t st = check_ws(p, ws, ws_bytes);
+  if (st != RF_OK) return st;
+  if ((st = rf_require_device()) != RF_OK) return st;
+  return rf_launch_quantize(p, q_r, k_r, need_v ? v_r : nullptr, ws, (cudaStream_t)stream);
 }
 
 rf_status_t rf_pool_select(const rf_plan_t* p, const void* q_r, const void* k_r,

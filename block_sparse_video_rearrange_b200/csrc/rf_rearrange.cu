@@ -11,7 +11,9 @@
 // token of each 128-token block.
 //
 // With precision "mix" the rearrange also writes an E4M3 copy of each Q and K
-// block with its fp32 scale (amax / 448) while the block is in registers.
+// block with its fp32 scale (amax / 448) while the block is in registers;
+// with precision "fp8" also an E4M3 copy of each V block on a power-of-two
+// scale, transposed through shared memory (the layout P V's B operand needs).
 // With precision "mxfp4" it writes MXFP4-rounded copies instead: Q and K rows
 // in groups of 32 columns, V columns in groups of 32 rows of each block, each
 // group on its UOS power-of-two scale, stored as the exact 16-bit values.
@@ -28,12 +30,14 @@
 namespace {
 
 enum Mode { kRearrange = 0, kInverse = 1, kPoolOnly = 2, kQuantOnly = 3 };
-enum Quant { kQuantNone = 0, kQuantE4M3 = 1, kQuantMx = 2 };
+enum Quant { kQuantNone = 0, kQuantE4M3 = 1, kQuantMx = 2, kQuantFp8 = 3 };
 
 // Outputs of the fused quantization.  Precision "mix": one-byte E4M3 copies of
 // Q' and K' in their layouts and one fp32 scale per (head, global block).
 // Precision "mxfp4": MXFP4-rounded copies of Q' and K' (input dtype) and of V'
 // (always f16, the type of the P V product), in the layouts of q_r, k_r, v_r.
+// Precision "fp8": the "mix" outputs, and E4M3 codes of V' transposed per block
+// ([n2][t_qblk][D][128] bytes) with one power-of-two exponent per (head, block).
 struct QuantOut {
   uint8_t* q8;
   uint8_t* k8;
@@ -42,6 +46,8 @@ struct QuantOut {
   uint4* qx;
   uint4* kx;
   uint4* vx;
+  uint8_t* v8;
+  int32_t* v_exp;
 };
 
 // Eight 16-bit values (one 16-byte chunk) rounded to MXFP4, element i on
@@ -222,7 +228,7 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
   }
-  if constexpr (kQuant == kQuantE4M3 && (MODE == kRearrange || MODE == kQuantOnly)) {
+  if constexpr ((kQuant == kQuantE4M3 || kQuant == kQuantFp8) && (MODE == kRearrange || MODE == kQuantOnly)) {
     if (tensor < 2) {  // uniform over the CTA: Q and K blocks get an E4M3 copy
       // amax over the block's valid rows (rows past nrows hold zeros).  For
       // finite bf16 and fp16 alike |x| orders as the 15-bit magnitude field,
@@ -265,6 +271,49 @@ __global__ void __launch_bounds__(kThreads)
         float* sc = tensor == 0 ? qo.q_scale : qo.k_scale;
         sc[(size_t)head * g.t_qblk + tb] = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
       }
+    } else if constexpr (kQuant == kQuantFp8) {
+      // V (precision "fp8"): E4M3 codes of v * 2^-e, e the smallest integer
+      // with amax <= 448 * 2^e (amax / 448 is a correctly rounded division and
+      // amax a 16-bit value, so a boundary amax = 448 * 2^k gives exactly 2^k),
+      // written transposed: column c of the block holds its 128 keys together.
+      constexpr int kTileStride = RF_BLOCK + 4;   // bytes per tile row (33 words)
+      __shared__ __align__(16) uint8_t tile[D * kTileStride];
+      uint32_t mb = 0u;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        mb = __vmaxu2(mb, val[i].x & 0x7FFF7FFFu);
+        mb = __vmaxu2(mb, val[i].y & 0x7FFF7FFFu);
+        mb = __vmaxu2(mb, val[i].z & 0x7FFF7FFFu);
+        mb = __vmaxu2(mb, val[i].w & 0x7FFF7FFFu);
+      }
+      mb = __reduce_max_sync(0xffffffffu, max(mb & 0xFFFFu, mb >> 16));
+      if ((threadIdx.x & 31) == 0) amax_w[threadIdx.x >> 5] = mb;
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < kThreads / 32; ++i) mb = max(mb, amax_w[i]);
+      const float amax = Dec::lo(mb);
+      // an all-zero block takes the smallest exponent: it never sets a row's largest
+      const int e = amax > 0.f ? rf_ceil_log2(__fdiv_rn(amax, 448.0f)) : -127;
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int rr = rl + i * kRowLanes;       // rows past nrows hold zeros: code 0
+        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          unsigned short two;
+          asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
+              : "=h"(two) : "f"(rf_scale_pow2(Dec::hi(w[c]), -e)), "f"(rf_scale_pow2(Dec::lo(w[c]), -e)));
+          tile[(ch * 8 + 2 * c) * kTileStride + rr] = (uint8_t)(two & 0xFFu);
+          tile[(ch * 8 + 2 * c + 1) * kTileStride + rr] = (uint8_t)(two >> 8);
+        }
+      }
+      __syncthreads();
+      uint32_t* out = reinterpret_cast<uint32_t*>(qo.v8 + ((size_t)head * g.t_qblk + tb) * (size_t)(RF_BLOCK * D));
+      for (int wd = threadIdx.x; wd < D * RF_BLOCK / 4; wd += kThreads) {
+        const int d = wd / (RF_BLOCK / 4), c4 = wd % (RF_BLOCK / 4);
+        out[wd] = *reinterpret_cast<const uint32_t*>(&tile[d * kTileStride + 4 * c4]);
+      }
+      if (threadIdx.x == 0) qo.v_exp[(size_t)head * g.t_qblk + tb] = e;
     }
   }
   if constexpr (MODE == kInverse || MODE == kQuantOnly) {
@@ -312,9 +361,14 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
   float* pq = ws ? reinterpret_cast<float*>(w + p->off_pq) : nullptr;
   float* pk = ws ? reinterpret_cast<float*>(w + p->off_pk) : nullptr;
   const bool quant_stage = MODE == kRearrange || MODE == kQuantOnly;
-  const bool quant = quant_stage && p->precision == RF_PRECISION_MIX;
+  const bool fp8 = quant_stage && p->precision == RF_PRECISION_FP8;
+  const bool quant = quant_stage && (p->precision == RF_PRECISION_MIX || fp8);
   const bool mx = quant_stage && p->precision == RF_PRECISION_MXFP4;
-  QuantOut qout{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  QuantOut qout{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  if (fp8) {
+    qout.v8 = reinterpret_cast<uint8_t*>(w + p->off_v8);
+    qout.v_exp = reinterpret_cast<int32_t*>(w + p->off_vexp);
+  }
   if (quant) {
     qout.q8 = reinterpret_cast<uint8_t*>(w + p->off_q8);
     qout.k8 = reinterpret_cast<uint8_t*>(w + p->off_k8);
@@ -335,7 +389,10 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
   const bool bf = p->dtype == RF_BF16;
   dim3 grd((unsigned)grid), blk(kThreads);
   if (g.d == 128) {
-    if (quant) {
+    if (fp8) {
+      if (bf) rf_permute_kernel<128, MODE, DecodeBf16, kQuantFp8><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+      else    rf_permute_kernel<128, MODE, DecodeF16, kQuantFp8><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
+    } else if (quant) {
       // precision mix is built for D = 128 only (checked when the plan is made)
       if (bf) rf_permute_kernel<128, MODE, DecodeBf16, kQuantE4M3><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
       else    rf_permute_kernel<128, MODE, DecodeF16, kQuantE4M3><<<grd, blk, 0, st>>>(g, a, b, c, x, y, z, pq, pk, qout);
@@ -371,8 +428,8 @@ rf_status_t rf_launch_pool(const rf_plan* p, const void* q_r, const void* k_r, v
 
 rf_status_t rf_launch_quantize(const rf_plan* p, const void* q_r, const void* k_r, const void* v_r,
                                void* ws, cudaStream_t st) {
-  // mix quantizes Q and K; mxfp4 also V (the third tensor's heads)
-  const int heads = p->g.n1 + p->g.n2 + (p->precision == RF_PRECISION_MXFP4 ? p->g.n2 : 0);
+  // mix quantizes Q and K; fp8 and mxfp4 also V (the third tensor's heads)
+  const int heads = p->g.n1 + p->g.n2 + (p->precision == RF_PRECISION_MIX ? 0 : p->g.n2);
   return launch<kQuantOnly>(p, q_r, k_r, v_r, nullptr, nullptr, nullptr, ws, st, heads);
 }
 

@@ -36,7 +36,7 @@ EXPORTED = ("rf_plan_create", "rf_plan_info", "rf_plan_seq_info", "rf_rearrange"
             "rf_block_sparse_attn", "rf_inverse_rearrange", "rf_forward", "rf_check_device_status",
             "rf_plan_destroy", "rf_status_string", "rf_last_error", "rf_plan_permutation",
             "rf_selftest_exp2", "rf_pool_select_noalloc", "rf_plan_create_ex", "rf_quantize_qk",
-            "rf_selftest_expired_wait", "rf_quantize_mx")
+            "rf_selftest_expired_wait", "rf_quantize_mx", "rf_quantize")
 
 
 class RfError(RuntimeError):
@@ -59,7 +59,8 @@ class PlanInfo(ctypes.Structure):
                 ("d", ctypes.c_int32), ("precision", ctypes.c_int32), ("token_order", ctypes.c_int32),
                 ("ws_q8", ctypes.c_int64), ("ws_k8", ctypes.c_int64),
                 ("ws_q_scale", ctypes.c_int64), ("ws_k_scale", ctypes.c_int64),
-                ("ws_q_mx", ctypes.c_int64), ("ws_k_mx", ctypes.c_int64), ("ws_v_mx", ctypes.c_int64)]
+                ("ws_q_mx", ctypes.c_int64), ("ws_k_mx", ctypes.c_int64), ("ws_v_mx", ctypes.c_int64),
+                ("ws_v8", ctypes.c_int64), ("ws_v_exp", ctypes.c_int64)]
 
 
 class PlanOptions(ctypes.Structure):
@@ -86,6 +87,7 @@ def _load() -> ctypes.CDLL:
                               i32, i32, ctypes.POINTER(PlanOptions), ctypes.POINTER(vp)],
         "rf_quantize_qk": [vp, vp, vp, vp, sz, vp],
         "rf_quantize_mx": [vp, vp, vp, vp, vp, sz, vp],
+        "rf_quantize": [vp, vp, vp, vp, vp, sz, vp],
         "rf_selftest_expired_wait": [vp, vp, sz, vp],
         "rf_plan_info": [vp, ctypes.POINTER(PlanInfo)],
         "rf_plan_seq_info": [vp, i32, ctypes.POINTER(SeqInfo)],
@@ -296,6 +298,17 @@ def quantize_mx(plan: Plan, q_r, k_r, v_r, ws, stream=None) -> None:
     _expect(v_r, plan.tensor_shape(plan.n2), plan.torch_dtype, "v_r")
     _check(_lib.rf_quantize_mx(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(v_r), _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream)), "rf_quantize_mx")
+
+
+def quantize(plan: Plan, q_r, k_r, v_r, ws, stream=None) -> None:
+    """Every quantized copy the plan's precision needs ("mix", "fp8", "mxfp4"), from
+    rearranged q_r / k_r / v_r, into ws (v_r may be None for "mix")."""
+    _expect(q_r, plan.tensor_shape(plan.n1), plan.torch_dtype, "q_r")
+    _expect(k_r, plan.tensor_shape(plan.n2), plan.torch_dtype, "k_r")
+    if v_r is not None:
+        _expect(v_r, plan.tensor_shape(plan.n2), plan.torch_dtype, "v_r")
+    _check(_lib.rf_quantize(plan.handle, _ptr(q_r), _ptr(k_r), _ptr(v_r), _ptr(ws),
+                            ws.numel() * ws.element_size(), _stream(stream)), "rf_quantize")
 
 
 def inverse_rearrange(plan: Plan, o_r, o, stream=None) -> None:

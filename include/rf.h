@@ -137,6 +137,13 @@ typedef struct {
    * copies of Q', K' (the inputs' 16-bit type) and V' (always f16), each with
    * the layout and strides of q_r / k_r / v_r. */
   int64_t ws_q_mx, ws_k_mx, ws_v_mx;
+  /* RF_PRECISION_FP8 only (else -1): byte offsets in ws of the E4M3 codes of V'
+   * and of their exponents.  The codes are stored transposed per block, uint8
+   * [n2][t_qblk][d][128]: for head h and global block t, column c of the block
+   * holds its 128 keys contiguously (rows past a partial block's end are 0).
+   * The exponents are int32 [n2][t_qblk]: the codes of block t of head h
+   * represent code * 2^exp. ws_q8 .. ws_k_scale are as for RF_PRECISION_MIX. */
+  int64_t ws_v8, ws_v_exp;
 } rf_plan_info_t;
 
 /* Per-sequence geometry under suffix promotion ([UG] "Geometry handling"). */
@@ -192,9 +199,22 @@ RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int
  *                        all-zero block has inv = scale = 1), and
  *                        rf_block_sparse_attn multiplies each S tile by
  *                        scale_q * scale_k.  Head dim 128 only.
- *   RF_PRECISION_FP8     FP8 for P V as well: not built (RF_ERR_UNSUPPORTED).
+ *   RF_PRECISION_FP8     FP8 E4M3 for P V as well.  Q' and K' as in
+ *                        RF_PRECISION_MIX.  V' is quantized per (head, 128-row
+ *                        block) on a power-of-two scale: exp = the smallest
+ *                        integer with amax <= 448 * 2^exp (-127 for an all-zero
+ *                        block), codes = E4M3(v * 2^-exp) rounded to nearest
+ *                        even with saturation (the scaling is exact).  The
+ *                        softmax probabilities of key block j enter the P V
+ *                        product as E4M3 values of P * 2^(exp_j - exp_max),
+ *                        exp_max the largest V exponent among the row's selected
+ *                        blocks (so every code stays below 448); the row sum is
+ *                        taken from the unrounded probabilities, and the output
+ *                        is multiplied back by 2^exp_max.  Both products run on
+ *                        the FP8 tensor cores (kind::f8f6f4).  Head dim 128 only,
+ *                        blockShape 128 x 128.
  * The pages name the three modes and nothing more; the E4M3 format, the block
- * granularity and the scale rule above are this library's reading.
+ * granularity and the scale rules above are this library's reading.
  *   RF_PRECISION_MXFP4   MXFP4 attention with Universal Optimal Scaling and
  *                        Pre-Normalization Quantization ([MX] "MXAttention",
  *                        abstract).  Every operand of both products is MXFP4:
@@ -230,8 +250,8 @@ typedef struct {
 /* rf_plan_create with options (rf_plan_create is rf_plan_create_ex with
  * options == NULL, i.e. tile order and native precision).  Every other
  * argument and error as rf_plan_create; an unknown option value or a non-zero
- * reserved field is RF_ERR_INVALID_ARG; RF_PRECISION_FP8, or RF_PRECISION_MIX
- * with d != 128, is RF_ERR_UNSUPPORTED.  RF_PRECISION_MXFP4 takes d 64 or 128.  Every later call on the plan
+ * reserved field is RF_ERR_INVALID_ARG; RF_PRECISION_MIX or RF_PRECISION_FP8
+ * with d != 128 is RF_ERR_UNSUPPORTED.  RF_PRECISION_MXFP4 takes d 64 or 128.  Every later call on the plan
  * (rearrange, pooling, selection, attention, inverse, rf_plan_permutation)
  * follows the plan's options. */
 RF_API rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
@@ -275,6 +295,15 @@ RF_API rf_status_t rf_quantize_qk(const rf_plan_t* plan, const void* q_r, const 
  * precision. */
 RF_API rf_status_t rf_quantize_mx(const rf_plan_t* plan, const void* q_r, const void* k_r,
                                   const void* v_r, void* ws, size_t ws_bytes, rf_stream_t stream);
+/* Every quantized copy the plan's precision needs, written into ws from
+ * already-rearranged q_r, k_r, v_r exactly as rf_rearrange writes them in its
+ * own pass (see rf_precision_t): "mix" the E4M3 Q' and K' with their scales
+ * (v_r may be NULL); "fp8" those and the transposed E4M3 V' with its
+ * exponents; "mxfp4" the MXFP4-rounded Q', K', V'.  For callers that produce
+ * q_r / k_r / v_r themselves.  Inputs 16-byte aligned and non-null (v_r except
+ * for "mix").  RF_ERR_INVALID_ARG for a native plan. */
+RF_API rf_status_t rf_quantize(const rf_plan_t* plan, const void* q_r, const void* k_r,
+                               const void* v_r, void* ws, size_t ws_bytes, rf_stream_t stream);
 /* Steps 2-3 ([UG] opening paragraphs and "Configuration"; [API] selectIdx and
  * selectNum constraints).
  * q_r, k_r    : rearranged Q and K (read only when pool_mode == RF_POOL_RECOMPUTE;

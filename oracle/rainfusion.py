@@ -562,3 +562,109 @@ def dequantize_e4m3(p: Problem, codes: np.ndarray, scales: np.ndarray, heads: in
             v = e4m3_decode(p.head_rows(codes, s, n)[r.start:r.stop]) * np.float64(scales[n, t])
             p.head_rows(out, s, n)[r.start:r.stop] = v
     return out
+
+
+# --------------------------------------------------------------------------------------
+# "fp8" kernel precision ([UG] "Configuration": precision "fp8"; "Wan2.2 T2V quantization
+# on Ascend": FP8 block-sparse attention).  The pages give the name only; reading R24:
+# Q and K are quantized as in "mix"; V is quantized to E4M3 with one power-of-two scale
+# per (head, 128-row block), 2^e with e the smallest integer for which the block's
+# largest magnitude is at most 448 * 2^e (codes E4M3(v * 2^-e): an exact scaling, then
+# round to nearest even with saturation; an all-zero block takes the smallest exponent,
+# -127, so that it never raises a row's largest one); the softmax probabilities of each
+# key block enter the P V product as E4M3 values of P * 2^(e_j - e_max), e_max the
+# largest V exponent among the row's selected blocks, while the row sum uses the
+# unrounded probabilities.
+FP8_ZERO_EXP = -127
+# --------------------------------------------------------------------------------------
+
+def pow2_exponent(amax: float, top: float = E4M3_MAX) -> int:
+    """Smallest integer e with amax <= top * 2^e (0 for amax == 0).  Exact: the
+    comparisons are between float64 values that hold amax and top * 2^e exactly."""
+    amax = float(amax)
+    if amax == 0.0:
+        return 0
+    e = math.ceil(math.log2(amax / top))
+    while amax > top * 2.0 ** e:
+        e += 1
+    while amax <= top * 2.0 ** (e - 1):
+        e -= 1
+    return e
+
+
+def quantize_block_e4m3_pow2(x: np.ndarray) -> Tuple[np.ndarray, int]:
+    """One block (rows x D) of 16-bit values: E4M3 codes of x * 2^-e and the exponent e
+    (reading R24); an all-zero block has e = -127 and all codes zero."""
+    x = np.asarray(x, dtype=np.float64)
+    amax = float(np.max(np.abs(x))) if x.size else 0.0
+    if amax == 0.0:
+        return np.zeros(x.shape, dtype=np.uint8), FP8_ZERO_EXP
+    e = pow2_exponent(amax)
+    return e4m3_round(x * 2.0 ** (-e)), e
+
+
+def quantize_v_fp8(p: Problem, v_r: np.ndarray, heads: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Per (head, block) power-of-two E4M3 quantization of a rearranged V: uint8 codes
+    shaped like v_r and int32 exponents [heads, T_qblk] by global block number."""
+    codes = np.zeros(v_r.shape, dtype=np.uint8)
+    exps = np.zeros((heads, p.t_qblk), dtype=np.int32)
+    for t, (s, g, b) in enumerate(qblock_table(p)):
+        r = block_rows(g, b)
+        for n in range(heads):
+            c, e = quantize_block_e4m3_pow2(p.head_rows(v_r, s, n)[r.start:r.stop])
+            p.head_rows(codes, s, n)[r.start:r.stop] = c
+            exps[n, t] = e
+    return codes, exps
+
+
+def dequantize_v_fp8(p: Problem, codes: np.ndarray, exps: np.ndarray, heads: int) -> np.ndarray:
+    """float64 values code * 2^e of its (head, block), in the layout of codes."""
+    out = np.zeros(codes.shape, dtype=np.float64)
+    for t, (s, g, b) in enumerate(qblock_table(p)):
+        r = block_rows(g, b)
+        for n in range(heads):
+            p.head_rows(out, s, n)[r.start:r.stop] = (
+                e4m3_decode(p.head_rows(codes, s, n)[r.start:r.stop]) * 2.0 ** int(exps[n, t]))
+    return out
+
+
+def fp8_probability_error_bound(p: Problem, q_r: np.ndarray, k_r: np.ndarray, v_r: np.ndarray,
+                                idx: np.ndarray, num: np.ndarray, scale: float,
+                                items: Sequence[Tuple[int, int]],
+                                v_exps: np.ndarray | None = None) -> Dict[Tuple[int, int], np.ndarray]:
+    """Per output element of the listed (q-block, head) items: the largest change that
+    rounding every probability to E4M3 can make to softmax(scale q K^T) V when the row
+    sum stays exact.  P_i is taken relative to the row's largest logit (P_i <= 1).  In
+    the normal range P~_i = P_i (1 + d_i), |d_i| <= 2^-4 (half a step of a 3-bit
+    mantissa).  A probability of key block j enters as E4M3(P_i 2^u 2^(e_j - e_max)),
+    where 2^u in [1, 2^8] is the kernel's own normalisation; below the normal range
+    (2^-6) the rounding error is at most half a subnormal step, 2^-10, in those units,
+    so at most min(P_i, 2^-10 2^(e_max - e_j)) in units of P_i (and 0 when v_exps is
+    None).  The change is sum_i (P~_i - P_i) V_i / sum_i P_i, so
+    |change| <= sum_i (2^-4 P_i + min(P_i, 2^-10 2^(e_max - e_j))) |V_i| / sum_i P_i."""
+    G = p.n1 // p.n2
+    table = qblock_table(p)
+    out = {}
+    for (t, n) in items:
+        s, g, b = table[t]
+        qrows = block_rows(g, b)
+        krows: List[int] = []
+        for j in idx[t, n, :num[t, n]]:
+            if j >= 0:
+                krows.extend(block_rows(g, int(j)))
+        q = p.head_rows(q_r, s, n)[qrows.start:qrows.stop]
+        k = p.head_rows(k_r, s, n // G)[krows]
+        v = p.head_rows(v_r, s, n // G)[krows]
+        logits = scale * (q @ k.T)
+        logits -= logits.max(axis=1, keepdims=True)
+        w = np.exp(logits)
+        err = 2.0 ** -4 * w
+        if v_exps is not None:
+            t0 = t - b                                   # first global block of this sequence
+            blocks = [int(j) for j in idx[t, n, :num[t, n]] if j >= 0]
+            e = np.array([v_exps[n // G, t0 + j] for j in blocks], dtype=np.float64)
+            step = np.concatenate([np.full(len(block_rows(g, j)), 2.0 ** (-10 + e.max() - ej))
+                                   for j, ej in zip(blocks, e)])
+            err = err + np.minimum(w, step[None, :])
+        out[(t, n)] = (err @ np.abs(v)) / w.sum(axis=1, keepdims=True)
+    return out

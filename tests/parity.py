@@ -64,8 +64,10 @@ def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "fro
     out = dict(plan=plan, q_r=to_bits(b.q_r), k_r=to_bits(b.k_r), v_r=to_bits(b.v_r), o_r=to_bits(b.o_r),
                o=to_bits(b.o), idx=b.select_idx.cpu().numpy(), num=b.select_num.cpu().numpy(),
                pooled_q=pq, pooled_k=pk, scale=scale)
-    if precision == "mix":
+    if precision in ("mix", "fp8"):
         out.update(mix_buffers(plan, b.ws))
+    if precision == "fp8":
+        out.update(fp8_buffers(plan, b.ws, problem(w)))
     if precision == "mxfp4":
         out.update(mx_buffers(plan, b.ws))
     return out
@@ -114,6 +116,77 @@ def mix_buffers(plan: rf.Plan, ws: torch.Tensor) -> Dict[str, np.ndarray]:
     qs = region(info.ws_q_scale, plan.n1 * t * 4).view(np.float32).reshape(plan.n1, t)
     ks = region(info.ws_k_scale, plan.n2 * t * 4).view(np.float32).reshape(plan.n2, t)
     return dict(q8=q8, k8=k8, q_scale=qs, k_scale=ks)
+
+
+def fp8_buffers(plan: rf.Plan, ws: torch.Tensor, p: orc.Problem) -> Dict[str, np.ndarray]:
+    """Precision fp8: the transposed E4M3 V' codes put back into the layout of v_r (rows
+    past a partial block's end are dropped) and the int32 exponents [n2, t_qblk]."""
+    info = plan.info
+    ws8 = ws.view(torch.uint8)
+    t, d, n2 = int(info.t_qblk), plan.d, plan.n2
+    raw = ws8[int(info.ws_v8):int(info.ws_v8) + n2 * t * 128 * d].cpu().numpy().reshape(n2, t, d, 128)
+    exps = ws8[int(info.ws_v_exp):int(info.ws_v_exp) + n2 * t * 4].cpu().numpy().view(np.int32).reshape(n2, t)
+    codes = np.zeros(plan.tensor_shape(n2), dtype=np.uint8)
+    for tb, (s, g, b) in enumerate(orc.qblock_table(p)):
+        r = orc.block_rows(g, b)
+        for n in range(n2):
+            p.head_rows(codes, s, n)[r.start:r.stop] = raw[n, tb, :, :len(r)].T
+    return dict(v8=codes, v_exp=exps, v8_raw=raw)
+
+
+def check_fp8_quantization(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu) -> None:
+    """Precision fp8: Q', K' as mix; V' codes and exponents bit-exact against the oracle,
+    and the rows past a partial block's end hold code 0."""
+    check_mix_quantization(p, w, rbits, gpu)
+    vf = synth.bits_to_float64(rbits[2], w.dtype)
+    codes, exps = orc.quantize_v_fp8(p, vf, w.n2)
+    assert np.array_equal(gpu["v_exp"], exps), "V exponents differ"
+    diff = gpu["v8"] != codes
+    assert not diff.any(), f"V E4M3 codes differ at {int(diff.sum())} elements"
+    for tb, (s, g, b) in enumerate(orc.qblock_table(p)):
+        n_valid = len(orc.block_rows(g, b))
+        assert not gpu["v8_raw"][:, tb, :, n_valid:].any(), tb
+
+
+def fp8_reference_inputs(p: orc.Problem, w: synth.Workload, gpu, rbits: Sequence[np.ndarray]):
+    """float64 Q', K', V' as precision fp8 sees them (codes x scales)."""
+    qf = orc.dequantize_e4m3(p, gpu["q8"], gpu["q_scale"], w.n1)
+    kf = orc.dequantize_e4m3(p, gpu["k8"], gpu["k_scale"], w.n2)
+    vf = orc.dequantize_v_fp8(p, gpu["v8"], gpu["v_exp"], w.n2)
+    return qf, kf, vf
+
+
+def check_fp8_attention(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu,
+                        items: Sequence[Tuple[int, int]] | None = None) -> Dict[str, float]:
+    """Precision fp8 output against the oracle run on the dequantized Q', K', V' with
+    exact probabilities: every element within the oracle's bound on rounding the
+    probabilities to E4M3 (fp8_probability_error_bound) plus the output's own 16-bit
+    rounding (half an ulp, 2^-8 relative for bf16) and 1e-3 for the fp32 arithmetic;
+    relative L2 within the native bar."""
+    qf, kf, vf = fp8_reference_inputs(p, w, gpu, rbits)
+    if items is None:
+        items = [(t, n) for t in range(p.t_qblk) for n in range(w.n1)]
+    ref = orc.attention(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items)
+    bound = orc.fp8_probability_error_bound(p, qf, kf, vf, gpu["idx"], gpu["num"], gpu["scale"], items,
+                                            v_exps=gpu["v_exp"])
+    o_r = synth.bits_to_float64(gpu["o_r"], w.dtype)
+    table = orc.qblock_table(p)
+    num = den = 0.0
+    mx = worst = 0.0
+    for (t, n), rows in ref.items():
+        s, g, b = table[t]
+        r = orc.block_rows(g, b)
+        got = p.head_rows(o_r, s, n)[r.start:r.stop]
+        d = np.abs(got - rows)
+        lim = bound[(t, n)] + 2.0 ** -8 * np.abs(rows) + 1e-3
+        assert np.all(d <= lim), (t, n, float(np.max(d - lim)))
+        mx = max(mx, float(np.max(d)))
+        worst = max(worst, float(np.max(d / lim)))
+        num += float(np.sum(d * d))
+        den += float(np.sum(rows * rows))
+    rel = math.sqrt(num / max(den, 1e-300))
+    assert rel <= REL_L2, f"rel L2 err {rel}"
+    return dict(max_abs=mx, rel_l2=rel, items=len(ref), worst_fraction_of_bound=worst)
 
 
 def check_mix_quantization(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], gpu) -> None:

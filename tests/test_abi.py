@@ -175,7 +175,8 @@ def test_plan_options_are_validated():
     bad = rf.PlanOptions(0, 0)
     bad.reserved[3] = 1
     assert _create_ex(bad) == (1, False)                          # reserved fields must be zero
-    assert _create_ex(rf.PlanOptions(0, 2), d=128) == (6, False)  # fp8 P V: not built
+    assert _create_ex(rf.PlanOptions(0, 2), d=128) == (0, True)   # fp8 (FP8 P V as well)
+    assert _create_ex(rf.PlanOptions(0, 2), d=64) == (6, False)   # fp8: head dim 128 only
     assert _create_ex(rf.PlanOptions(0, 1), d=64) == (6, False)   # mix: head dim 128 only
     assert _create_ex(rf.PlanOptions(1, 1), d=128) == (0, True)
     with pytest.raises(ValueError):
@@ -202,6 +203,36 @@ def test_mix_precision_workspace_layout(layout, seqs, n1, n2):
     assert b.workspace_bytes >= b.ws_k_scale + n2 * t * 4
     for f in ("rows_total", "t_qblk", "max_kv_blocks", "pooled_blocks", "ws_pooled_q", "ws_pooled_k"):
         assert getattr(a, f) == getattr(b, f), f
+
+
+@pytest.mark.parametrize("layout,seqs,n1,n2", [("BNSD", [(512, 21, 30, 52)], 40, 40),
+                                               ("TND", [(256, 13, 32, 48), (384, 21, 24, 40)], 32, 8)])
+def test_fp8_precision_workspace_layout(layout, seqs, n1, n2):
+    """Precision fp8: the mix regions, then the transposed E4M3 V' (one byte per
+    element, [n2][t_qblk][128][128]) and its int32 exponents [n2][t_qblk]."""
+    mix = rf.Plan(seqs, n1, n2, 128, layout, "bf16", 0.8, precision="mix")
+    f8 = rf.Plan(seqs, n1, n2, 128, layout, "bf16", 0.8, precision="fp8")
+    a, b = mix.info, f8.info
+    assert b.precision == 2
+    assert a.ws_v8 == a.ws_v_exp == -1
+    for f in ("ws_q8", "ws_k8", "ws_q_scale", "ws_k_scale"):
+        assert getattr(a, f) == getattr(b, f), f
+    t = int(b.t_qblk)
+    assert b.ws_v8 >= a.workspace_bytes and b.ws_v8 % 256 == 0
+    assert b.ws_v_exp >= b.ws_v8 + n2 * t * 128 * 128 and b.ws_v_exp % 256 == 0
+    assert b.workspace_bytes >= b.ws_v_exp + n2 * t * 4
+    with pytest.raises(rf.RfError) as e:
+        rf.Plan(seqs, n1, n2, 128, layout, "bf16", 0.8, precision="fp8", block_kv=64)
+    assert e.value.status == 6
+
+
+def test_generic_quantize_entry_point_validates_on_the_host():
+    fake = ctypes.c_void_p(1 << 20)
+    native = rf.Plan([(128, 9, 16, 32)], 2, 2, 128)
+    assert rf.lib().rf_quantize(native.handle, fake, fake, fake, fake, native.workspace_bytes, None) == 1
+    f8 = rf.Plan([(128, 9, 16, 32)], 2, 2, 128, precision="fp8")
+    assert rf.lib().rf_quantize(f8.handle, fake, fake, None, fake, f8.workspace_bytes, None) == 1   # needs V
+    assert rf.lib().rf_quantize(f8.handle, fake, fake, fake, fake, 16, None) == 3   # workspace too small
 
 
 def test_quantize_needs_a_mix_plan():

@@ -511,3 +511,59 @@ def test_kv64_random_selection_against_the_oracle(name):
     rbits = [orc.rearrange(p, x) for x in bits]
     got = dict(idx=clean, num=clean_num, scale=gpu["scale"], o_r=o64)
     parity.check_attention(p, w, rbits, got, block_kv=64)
+
+
+# ------------------------------------------------------------------------------------------
+# Precision "fp8" (user guide "Configuration": precision "fp8"; reading R24): E4M3 Q K^T as
+# in mix, E4M3 V' on power-of-two scales, probabilities rounded to E4M3 for P V.  Codes and
+# exponents bit-exact; output within the oracle's bound on the probability rounding.
+# ------------------------------------------------------------------------------------------
+
+FP8_SMALL = ["ragged_d128", "tnd_gqa_small", "dense", "s_one", "all_promoted"]
+
+
+@pytest.mark.parametrize("name", FP8_SMALL)
+def test_fp8_small_parity(name):
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision="fp8")
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    parity.check_fp8_quantization(p, w, rbits, gpu)
+    qbars, kbars = parity.oracle_pooled(p, w, rbits)
+    parity.check_pooled(p, qbars, kbars, gpu)             # pooling still reads the 16-bit values
+    parity.check_selection(p, qbars, kbars, gpu)
+    err = parity.check_fp8_attention(p, w, rbits, gpu)
+    print(f"fp8 {name}: {err}")
+
+
+@pytest.mark.parametrize("name,s", [("wan", None), ("tnd_gqa", None), ("aligned", 0.8)])
+def test_fp8_full_size_parity(name, s):
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, precision="fp8")
+    rbits = [orc.rearrange(p, x) for x in bits]
+    parity.check_fp8_quantization(p, w, rbits, gpu)
+    items = parity.sample_items(p, np.random.default_rng(11), per_kind=3)
+    err = parity.check_fp8_attention(p, w, rbits, gpu, items)
+    print(f"fp8 {name}: {err}")
+    # the quantization error itself, against the unquantized oracle: reported, bounded loosely
+    err = parity.check_attention(p, w, rbits, gpu, items, check=False)
+    assert err["rel_l2"] <= 0.1, err
+
+
+def test_fp8_quantize_entry_point_equals_fused_quantization():
+    w = SMALL["tnd_gqa_small"]
+    bits = synth.generate_qkv(w)
+    fused = parity.run_gpu(w, bits, precision="fp8")
+    plan = fused["plan"]
+    b = rf.Buffers(plan)
+    q_r, k_r, v_r = (parity.to_device(fused[n], w.dtype) for n in ("q_r", "k_r", "v_r"))
+    rf.quantize(plan, q_r, k_r, v_r, b.ws)
+    torch.cuda.synchronize()
+    alone = parity.mix_buffers(plan, b.ws)
+    alone.update(parity.fp8_buffers(plan, b.ws, parity.problem(w)))
+    for key in ("q8", "k8", "q_scale", "k_scale", "v8_raw", "v_exp"):
+        assert np.array_equal(alone[key], fused[key]), key

@@ -89,3 +89,111 @@ def test_problem_quantization_covers_partial_prefix_block():
     assert scales[1, 0] == np.float32(np.max(np.abs(x[0, 1, :100])) / np.float32(448))
     deq = rf.dequantize_e4m3(p, codes, scales, 2)
     assert np.max(np.abs(deq - x)) <= np.max(np.abs(x)) * 2.0 ** -4
+
+
+# ---------------- precision "fp8" (reading R24): V on power-of-two scales ----------------
+
+def test_pow2_exponent_is_the_smallest_fitting_integer():
+    rng = np.random.default_rng(6)
+    vals = list(rng.lognormal(0.0, 4.0, 500)) + [448.0 * 2.0 ** k for k in range(-20, 20)]
+    vals += [float(np.nextafter(448.0 * 2.0 ** k, np.inf)) for k in range(-10, 10)]
+    vals += [float(np.nextafter(448.0 * 2.0 ** k, 0.0)) for k in range(-10, 10)]
+    for a in vals:
+        brute = next(e for e in range(-200, 200) if a <= 448.0 * 2.0 ** e)   # scan from below
+        assert rf.pow2_exponent(a) == brute, a
+    assert rf.pow2_exponent(0.0) == 0
+
+
+def test_pow2_block_quantization_matches_an_independent_conversion():
+    rng = np.random.default_rng(7)
+    for scale in (3.0, 0.01, 500.0):
+        x = (rng.standard_normal((128, 128)) * scale).astype(np.float32)
+        codes, e = rf.quantize_block_e4m3_pow2(x)
+        amax = float(np.max(np.abs(x)))
+        assert amax <= 448.0 * 2.0 ** e and amax > 448.0 * 2.0 ** (e - 1)
+        # the scaling by 2^-e is exact, so a library cast of the scaled values must agree
+        ref = torch.from_numpy((x.astype(np.float64) * 2.0 ** -e).astype(np.float32)) \
+            .to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        assert np.array_equal(codes, ref)
+        top = rf.e4m3_decode(codes[np.unravel_index(np.argmax(np.abs(x)), x.shape)])
+        assert 224.0 <= abs(top) <= 448.0                   # the largest value lands in the top binade
+        deq = rf.e4m3_decode(codes) * 2.0 ** e
+        err = np.abs(deq - x)
+        normal = np.abs(x) * 2.0 ** -e >= 2.0 ** -6
+        assert np.all(err[normal] <= np.abs(x[normal]) * 2.0 ** -4)
+        assert np.all(err[~normal] <= 2.0 ** -10 * 2.0 ** e)
+    zeros, e0 = rf.quantize_block_e4m3_pow2(np.zeros((4, 8), dtype=np.float32))
+    assert e0 == -127 and not zeros.any()              # never the row's largest exponent
+
+
+def test_fp8_v_quantization_covers_partial_prefix_block():
+    p = rf.make_problem("TND", 1, [(100, 8, 16, 32), (0, 8, 16, 16)], 4, 2, 128, 0.8)
+    rng = np.random.default_rng(8)
+    t_rows = sum(g.length for g in p.geoms)
+    x = rng.standard_normal((t_rows, 2, 128)).astype(np.float32)
+    codes, exps = rf.quantize_v_fp8(p, x, 2)
+    assert exps.shape == (2, p.t_qblk) and exps.dtype == np.int32
+    # the partial prefix block (Lp = 100) takes its exponent from its 100 valid rows
+    assert exps[1, 0] == rf.pow2_exponent(float(np.max(np.abs(x[:100, 1]))))
+    deq = rf.dequantize_v_fp8(p, codes, exps, 2)
+    assert np.max(np.abs(deq - x)) <= np.max(np.abs(x)) * 2.0 ** -4
+
+
+def test_fp8_probability_bound_holds_for_explicitly_rounded_probabilities():
+    """Round every probability to E4M3 by hand (on a power-of-two scale that keeps them in
+    the normal range) and check the output change against the oracle's bound."""
+    w = dict(layout="BNSD", batch=1, seqs=[(64, 8, 16, 32)], n1=2, n2=2, d=64, sparsity=0.8)
+    p = rf.make_problem(w["layout"], 1, w["seqs"], 2, 2, 64, 0.8)
+    rng = np.random.default_rng(9)
+    L = p.geoms[0].length
+    q, k, v = (rng.standard_normal((1, 2, L, 64)) * 0.8 for _ in range(3))
+    qb, kb = rf.pooled_means(p, q, 2), rf.pooled_means(p, k, 2)
+    idx, num = rf.select(p, qb, kb)
+    items = [(t, n) for t in (0, 3, 10, 20) for n in (0, 1)]
+    exact = rf.attention(p, q, k, v, idx, num, 0.125, items)
+    bound = rf.fp8_probability_error_bound(p, q, k, v, idx, num, 0.125, items)
+    table = rf.qblock_table(p)
+    for (t, n) in items:
+        s, g, b = table[t]
+        rows = rf.block_rows(g, b)
+        keys = [r for j in idx[t, n, :num[t, n]] for r in rf.block_rows(g, int(j))]
+        lg = 0.125 * (q[0, n, rows.start:rows.stop] @ k[0, n, keys].T)
+        lg -= lg.max(axis=1, keepdims=True)
+        pr = np.exp(lg)
+        # on 2^6 the largest probability (1) sits at 64: values down to 2^-12 stay normal
+        keep = pr >= 2.0 ** -12
+        pq = np.where(keep, rf.e4m3_decode(rf.e4m3_round(pr * 64.0)) / 64.0, pr)
+        o_round = (pq @ v[0, n, keys]) / pr.sum(axis=1, keepdims=True)
+        assert np.all(np.abs(o_round - exact[(t, n)]) <= bound[(t, n)] + 1e-12)
+
+
+@pytest.mark.parametrize("u", [0, 3, 8])
+def test_fp8_probability_bound_covers_block_shifts_and_subnormals(u):
+    """Round P * 2^u * 2^(e_j - e_max) to E4M3 exactly as the reading states, with V
+    exponents that differ between blocks (so small probabilities of low-exponent blocks
+    fall below the normal range), and check the change against the bound."""
+    p = rf.make_problem("BNSD", 1, [(64, 8, 16, 32)], 2, 2, 64, 0.8)
+    rng = np.random.default_rng(10 + u)
+    L = p.geoms[0].length
+    q, k = (rng.standard_normal((1, 2, L, 64)) * 1.5 for _ in range(2))
+    v = rng.standard_normal((1, 2, L, 64))
+    qb, kb = rf.pooled_means(p, q, 2), rf.pooled_means(p, k, 2)
+    idx, num = rf.select(p, qb, kb)
+    vexp = rng.integers(-9, -2, size=(2, p.t_qblk)).astype(np.int32)
+    items = [(t, n) for t in (0, 2, 9, 25) for n in (0, 1)]
+    exact = rf.attention(p, q, k, v, idx, num, 0.125, items)
+    bound = rf.fp8_probability_error_bound(p, q, k, v, idx, num, 0.125, items, v_exps=vexp)
+    table = rf.qblock_table(p)
+    for (t, n) in items:
+        s, g, b = table[t]
+        rows = rf.block_rows(g, b)
+        blocks = [int(j) for j in idx[t, n, :num[t, n]]]
+        keys = [r for j in blocks for r in rf.block_rows(g, j)]
+        e = np.concatenate([np.full(len(rf.block_rows(g, j)), vexp[n, t - b + j]) for j in blocks])
+        lg = 0.125 * (q[0, n, rows.start:rows.stop] @ k[0, n, keys].T)
+        lg -= lg.max(axis=1, keepdims=True)
+        pr = np.exp(lg)
+        f = 2.0 ** (u + e - e.max())[None, :]
+        pq = rf.e4m3_decode(rf.e4m3_round(pr * f)) / f
+        o_round = (pq @ v[0, n, keys]) / pr.sum(axis=1, keepdims=True)
+        assert np.all(np.abs(o_round - exact[(t, n)]) <= bound[(t, n)] + 1e-12)
