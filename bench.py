@@ -230,9 +230,11 @@ def algorithmic_bytes(plan, elem=2):
     # precision "fp8": and the transposed one-byte copy of V' (whole blocks) with its exponents
     if plan.precision == "fp8":
         quant += plan.n2 * t * 128 * plan.d + 4 * t * plan.n2
-    # precision "mxfp4": 16-bit MXFP4-rounded copies of Q', K' and V'
+    # precision "mxfp4": the MXFP4-rounded copies of Q', K' and V' (head dim 128: one-byte
+    # E4M3 carriers, V' as whole transposed blocks; head dim 64: 16-bit copies)
     if plan.precision == "mxfp4":
-        quant = rows * (plan.n1 + 2 * plan.n2) * plan.d * 2
+        quant = (rows * (plan.n1 + plan.n2) * plan.d + plan.n2 * t * 128 * plan.d if plan.d == 128
+                 else rows * (plan.n1 + 2 * plan.n2) * plan.d * 2)
     return 2 * qkv + sel + quant, inv
 
 
@@ -656,8 +658,12 @@ def main():
             if f8:
                 extra_roof = {"fp8_gemm_tflops_measured_here": round(f8, 1), "peak_with_measured_fp8": round(f8, 1),
                               "frac_with_measured_fp8": round(achieved / f8, 4)}
-        if args.precision == "mxfp4":
-            peak_note += "; mxfp4: both products run on the 16-bit tensor cores -> 1x"
+        if args.precision == "mxfp4" and w.d == 128:
+            # both products on the FP8 tensor cores (MXFP4 values carried exactly in E4M3)
+            peak = round(peak * 2.0, 1)
+            peak_note += "; mxfp4 at head dim 128: both products on E4M3 carriers at 2x (fp8, nominal ratio)"
+        elif args.precision == "mxfp4":
+            peak_note += "; mxfp4 at head dim 64: both products run on the 16-bit tensor cores -> 1x"
         front_bytes, inv_bytes = algorithmic_bytes(plan)
         front_ms = float(np.mean(per[:, 0] + per[:, 1]))
         inv_ms = float(np.mean(per[:, 3]))
@@ -686,7 +692,8 @@ def main():
                           if args.precision == "fp8" else {}),
                        **({"block_shape": "128 x 64 (attention on the 64-row halves of the step's 128-row "
                                           "selection, expanded once after warm-up)"} if args.block_kv == 64 else {}),
-                       **({"precision": "mxfp4 (UOS Qmax 7.25, PNQ)"} if args.precision == "mxfp4" else {}),
+                       **({"precision": "mxfp4 (UOS Qmax 7.25, PNQ; values carried in E4M3 at head dim 128)"}
+                          if args.precision == "mxfp4" else {}),
                        "global_batch": w.batch * world, "seq_len": int(plan.info.rows_total),
                        "parallelism": f"independent layer per GPU x{world}",
                        "l2": "inputs larger than L2 (Q+K+V %.2f GB vs 126 MB)" % (

@@ -92,6 +92,11 @@ constexpr uint32_t kOCol = 256;  // O_w, the accumulator of softmax group w, at 
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: lazy rescale while growth <= 256x
+// Precision mxfp4 with E4M3 carriers (head dim 128): the running max is kept
+// exact (threshold 0, so P <= 1) and the E4M3 P values are stored times 2^8
+// (at most 256 < 448), which keeps every MXFP4 value of P with 2^e >= 2^-16
+// exact in E4M3; the output is multiplied back by 2^-8.
+constexpr int kMxP8Up = 8;
 
 // kQk8: Q and K tiles hold E4M3 codes (precisions "mix" and "fp8"), one byte
 // per element.  kPv8: V tiles hold E4M3 codes stored transposed (D rows of 128
@@ -287,21 +292,26 @@ __device__ __forceinline__ void group_max4(const uint32_t* sr, int vr, float* gm
 // exponentials are taken as 2^(s * sl2 - (m + e)), rounded to E2M1 (the
 // hardware conversion saturates at 6), summed exactly in f16 (at most 32
 // values of at most 6 on a 0.5 grid) and scaled by 2^e.
-template <bool kFull>
+template <bool kFull, bool kOut8 = false>
 __device__ __forceinline__ void group_exp_mx(const uint32_t* sr, int cb, int vr, float sl2, float m,
                                              float gmax, uint32_t p_addr, float& lsum) {
+  constexpr int kUp = kOut8 ? kMxP8Up : 0;   // E4M3 P is stored times 2^kUp
   const uint64_t sl2x2 = rf_f2(__float_as_uint(sl2), __float_as_uint(sl2));
   const bool live = kFull || cb < vr;
   const int e = live ? (int)ceilf(fmaf(gmax, sl2, -m) - kMxLog2Qmax) : 0;
   const float neg_me = -(m + (float)e);
   const uint64_t negme2 = rf_f2(__float_as_uint(neg_me), __float_as_uint(neg_me));
-  // 2^e as f16 (normal from 2^-14, subnormal down to 2^-24; a group whose
-  // scale is below that rounds to zero in f16, as its P V terms would)
-  const unsigned short hb = e >= -14 ? (unsigned short)((15 + e) << 10)
-                                     : (e >= -24 ? (unsigned short)(1u << (e + 24)) : (unsigned short)0);
+  // 2^(e + kUp) as f16 (normal from 2^-14, subnormal down to 2^-24; a group
+  // whose scale is below that rounds to zero in f16, as its P V terms would)
+  const int eu = e + kUp;
+  const unsigned short hb = eu >= -14 ? (unsigned short)((15 + eu) << 10)
+                                      : (eu >= -24 ? (unsigned short)(1u << (eu + 24)) : (unsigned short)0);
   const __half2 up2 = __half2half2(__ushort_as_half(hb));
   __half2 acc0 = __float2half2_rn(0.f), acc1 = acc0;
-  uint32_t pk[16];
+  // kOut8: the rounded values times 2^(e + kUp), exact in f16, converted to
+  // E4M3 codes four per column (exact for -8 <= e + kUp <= 6); else the f16
+  // pairs themselves
+  uint32_t pk[kOut8 ? 8 : 16];
 #pragma unroll
   for (int c = 0; c < 32; c += 2) {
     float x0, x1;
@@ -316,11 +326,19 @@ __device__ __forceinline__ void group_exp_mx(const uint32_t* sr, int cb, int vr,
     if (c & 2) acc1 = __hadd2(acc1, rh);
     else       acc0 = __hadd2(acc0, rh);
     const __half2 ph = __hmul2(rh, up2);
-    pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
+    if constexpr (kOut8) {
+      unsigned short two;
+      asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(two) : "r"(*reinterpret_cast<const uint32_t*>(&ph)));
+      if (c & 2) pk[c >> 2] |= (uint32_t)two << 16;
+      else       pk[c >> 2] = two;
+    } else {
+      pk[c >> 1] = *reinterpret_cast<const uint32_t*>(&ph);
+    }
   }
   const float2 sum = __half22float2(__hadd2(acc0, acc1));
   if (live && e >= -126) lsum = fmaf(sum.x + sum.y, rf_pow2(e), lsum);
-  tmem_st16(p_addr, pk);
+  if constexpr (kOut8) tmem_st8(p_addr, pk);
+  else                 tmem_st16(p_addr, pk);
 }
 
 __device__ __forceinline__ float acc_sum(const uint64_t* acc) {
@@ -414,9 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   for (int c = threadIdx.x; c < num; c += kThreads) {
     const int v = row[c];
     sm.list[c] = v;
-    if constexpr (kQk8)
+    // precision mxfp4 carries its values in E4M3 with unit scales: nothing to load
+    if constexpr (kQk8 && !kMx)
       if (v >= 0 && v < nkv) sm.kscale[c] = a.k_scale[(size_t)gk * g.t_qblk + s.qblk_off + v];
-    if constexpr (kPv8)
+    if constexpr (kPv8 && !kMx)
       if (v >= 0 && v < nkv) sm.vexp[c] = a.v_exp[(size_t)gk * g.t_qblk + s.qblk_off + v];
   }
   __syncthreads();
@@ -426,15 +445,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // below its own read position, and every lane reads before the ballot.
     int bad = (lane == 0 && num != num_raw) ? 1 : 0;
     int cnt = 0;
-    int vmax = -127;  // precision "fp8": the largest V exponent of the row
+    int vmax = kMx ? 0 : -127;  // precision "fp8": the largest V exponent of the row
     const uint32_t lt = (1u << lane) - 1u;
     for (int c0 = 0; c0 < num; c0 += 32) {
       const int c = c0 + lane;
       const int v = c < num ? sm.list[c] : -1;
-      float ks = 0.f;
-      if constexpr (kQk8) ks = c < num ? sm.kscale[c] : 0.f;
-      int ve = -127;
-      if constexpr (kPv8) ve = c < num ? sm.vexp[c] : -127;
+      float ks = 1.f;
+      if constexpr (kQk8 && !kMx) ks = c < num ? sm.kscale[c] : 0.f;
+      int ve = kMx ? 0 : -127;
+      if constexpr (kPv8 && !kMx) ve = c < num ? sm.vexp[c] : -127;
       const bool ok = c < num && v >= 0 && v < nkv;
       if (c < num && v != -1 && !ok) ++bad;
       const uint32_t ball = __ballot_sync(0xffffffffu, ok);
@@ -683,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = (warp & 3) * 32 + lane;   // query row = TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     // precision "mix": S_j carries the E4M3 scales of the Q block and of K block j
-    const float sl2_q = kQk8 ? a.sl2 * a.q_scale[(size_t)n * g.t_qblk + tb] : a.sl2;
+    const float sl2_q = (kQk8 && !kMx) ? a.sl2 * a.q_scale[(size_t)n * g.t_qblk + tb] : a.sl2;
     const int my_blocks = (nv + 1 - wg) >> 1;  // blocks j < nv with j % 2 == wg
     const int vexp_max = kPv8 ? sm.vexp_max : 0;
     const uint32_t scol = lane_base;                          // S_j (both groups in turn)
@@ -704,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         vr = (sm.list[j] == s.n_pb - 1) ? vr_last : RF_BLOCK;
       }
-      const float sl2 = kQk8 ? sl2_q * sm.kscale[j] : sl2_q;
+      const float sl2 = (kQk8 && !kMx) ? sl2_q * sm.kscale[j] : sl2_q;
       // precision "fp8": P' = P * 2^-(exp_max - exp_j) for the P V product
       float down = 1.f;
       if constexpr (kPv8) {
@@ -735,7 +754,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!warp_wait(rf_smem_u32(&sm.bar_pv_done[wg]), (i - 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
       }
-      const bool rescale = __any_sync(0xffffffffu, mx_t > m_run + kRescaleThreshold);
+      constexpr float kThr = (kMx && kPv8) ? 0.f : kRescaleThreshold;
+      const bool rescale = __any_sync(0xffffffffu, mx_t > m_run + kThr);
       if (rescale) {
         // mxfp4: the running max stays an integer
         const float m_new = kMx ? ceilf(fmaxf(m_run, mx_t)) : fmaxf(m_run, mx_t);
@@ -762,13 +782,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // computed.
       uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
       float lsum = 0.f;
+      constexpr uint32_t kQCols = kPv8 ? 8 : 16;   // TMEM columns per 32 keys of P
       if constexpr (kMx) {
         if (vr == RF_BLOCK) {
-          group_exp_mx<true>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
-          group_exp_mx<true>(sr, 32, vr, sl2, m_run, gm[1], pcol + 16, lsum);
+          group_exp_mx<true, kPv8>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
+          group_exp_mx<true, kPv8>(sr, 32, vr, sl2, m_run, gm[1], pcol + kQCols, lsum);
         } else {
-          group_exp_mx<false>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
-          group_exp_mx<false>(sr, 32, vr, sl2, m_run, gm[1], pcol + 16, lsum);
+          group_exp_mx<false, kPv8>(sr, 0, vr, sl2, m_run, gm[0], pcol, lsum);
+          group_exp_mx<false, kPv8>(sr, 32, vr, sl2, m_run, gm[1], pcol + kQCols, lsum);
         }
       } else if constexpr (kPv8) {
         if (vr == RF_BLOCK) {
@@ -792,11 +813,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(rf_smem_u32(&sm.bar_p_half[wg]));
       if constexpr (kMx) {
         if (vr == RF_BLOCK) {
-          group_exp_mx<true>(sr, 64, vr, sl2, m_run, gm[2], pcol + 32, lsum);
-          group_exp_mx<true>(sr, 96, vr, sl2, m_run, gm[3], pcol + 48, lsum);
+          group_exp_mx<true, kPv8>(sr, 64, vr, sl2, m_run, gm[2], pcol + 2 * kQCols, lsum);
+          group_exp_mx<true, kPv8>(sr, 96, vr, sl2, m_run, gm[3], pcol + 3 * kQCols, lsum);
         } else {
-          group_exp_mx<false>(sr, 64, vr, sl2, m_run, gm[2], pcol + 32, lsum);
-          group_exp_mx<false>(sr, 96, vr, sl2, m_run, gm[3], pcol + 48, lsum);
+          group_exp_mx<false, kPv8>(sr, 64, vr, sl2, m_run, gm[2], pcol + 2 * kQCols, lsum);
+          group_exp_mx<false, kPv8>(sr, 96, vr, sl2, m_run, gm[3], pcol + 3 * kQCols, lsum);
         }
         l_run += lsum;
       } else if constexpr (kPv8) {
@@ -837,7 +858,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float a1 = l1 > 0.f ? rf_ex2(m1 - m) : 0.f;
     const float l = a0 * l0 + a1 * l1;
     // precision "fp8": P V ran on P * 2^-exp_max times the V codes
-    const float vsc = kPv8 ? (vexp_max >= -126 ? rf_pow2(vexp_max) : 0.f) : 1.f;
+    const float vsc = kMx ? (kPv8 ? rf_pow2(-kMxP8Up) : 1.f)
+                          : (kPv8 ? (vexp_max >= -126 ? rf_pow2(vexp_max) : 0.f) : 1.f);
     const float inv = l > 0.f ? vsc / l : 0.f;
     const float s0 = a0 * inv, s1 = a1 * inv;
     const bool use0 = have_o && nv > 0, use1 = have_o && nv > 1;
@@ -1007,8 +1029,9 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   // precision "mix": Q K^T reads the E4M3 copies rf_rearrange wrote into ws;
   // precision "mxfp4": every operand reads the MXFP4 copies in ws (V as f16).
   const bool fp8 = p->precision == RF_PRECISION_FP8;
-  const bool mix = p->precision == RF_PRECISION_MIX || fp8;   // E4M3 Q and K
   const bool mx = p->precision == RF_PRECISION_MXFP4;
+  const bool mx8 = mx && g.d == 128;                           // MXFP4 values in E4M3 carriers
+  const bool mix = p->precision == RF_PRECISION_MIX || fp8 || mx8;   // E4M3 Q and K
   char* w = static_cast<char*>(ws);
   const void* qsrc = mix ? static_cast<const void*>(w + p->off_q8) : mx ? static_cast<const void*>(w + p->off_qx) : q_r;
   const void* ksrc = mix ? static_cast<const void*>(w + p->off_k8) : mx ? static_cast<const void*>(w + p->off_kx) : k_r;
@@ -1017,7 +1040,7 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   if ((s = make_map(&mq, p, qsrc, g.n1, qk_elem)) != RF_OK) return s;
   const int kv_box = g.block_kv == 64 ? 64 : RF_BLOCK;
   if ((s = make_map(&mk, p, ksrc, g.n2, qk_elem, kv_box)) != RF_OK) return s;
-  if (fp8) {
+  if (fp8 || mx8) {
     if ((s = make_map_v8(&mv, p, w + p->off_v8)) != RF_OK) return s;
   } else if ((s = make_map(&mv, p, vsrc, g.n2, mx ? kElemF16 : kElemPlan, kv_box)) != RF_OK) {
     return s;
@@ -1028,12 +1051,15 @@ rf_status_t rf_launch_attn(const rf_plan* p, const void* q_r, const void* k_r, c
   args.sel_num = sel_num;
   args.o_r = static_cast<uint16_t*>(o_r);
   args.status = reinterpret_cast<uint32_t*>(w + p->off_status);
-  args.q_scale = mix ? reinterpret_cast<const float*>(w + p->off_qs) : nullptr;
-  args.k_scale = mix ? reinterpret_cast<const float*>(w + p->off_ks) : nullptr;
+  args.q_scale = (mix && !mx8) ? reinterpret_cast<const float*>(w + p->off_qs) : nullptr;
+  args.k_scale = (mix && !mx8) ? reinterpret_cast<const float*>(w + p->off_ks) : nullptr;
   args.v_exp = fp8 ? reinterpret_cast<const int32_t*>(w + p->off_vexp) : nullptr;
   args.sl2 = scale * kLog2e;
   const bool bf = p->dtype == RF_BF16;
   if (g.d == 128) {
+    if (mx8)
+      return bf ? launch_t<128, true, true, true, true>(mq, mk, mv, args, (unsigned)grid, st)
+                : launch_t<128, false, true, true, true>(mq, mk, mv, args, (unsigned)grid, st);
     if (fp8)
       return bf ? launch_t<128, true, true, false, true>(mq, mk, mv, args, (unsigned)grid, st)
                 : launch_t<128, false, true, false, true>(mq, mk, mv, args, (unsigned)grid, st);

@@ -276,7 +276,18 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   }
   // RF_PRECISION_MXFP4: MXFP4-rounded 16-bit copies of Q', K', V' (layouts of
   // q_r / k_r / v_r).
-  if (p->precision == RF_PRECISION_MXFP4) {
+  // D = 128 carries the MXFP4 values as E4M3 codes instead (every value c * 2^e
+  // with -8 <= e <= 6 is one): Q' and K' one byte per element in the layouts of
+  // q_r / k_r (the mix regions, no scales), V' transposed per block (the fp8
+  // region, no exponents); both products then run on the FP8 tensor cores.
+  if (p->precision == RF_PRECISION_MXFP4 && d == 128) {
+    p->off_q8 = off;
+    off = align_up(off + p->rows_total * n1 * d, 256);
+    p->off_k8 = off;
+    off = align_up(off + p->rows_total * n2 * d, 256);
+    p->off_v8 = off;
+    off = align_up(off + (int64_t)n2 * qblk * RF_BLOCK * d, 256);
+  } else if (p->precision == RF_PRECISION_MXFP4) {
     p->off_qx = off;
     off = align_up(off + p->rows_total * n1 * d * 2, 256);
     p->off_kx = off;

@@ -72,6 +72,20 @@ __device__ __forceinline__ uint4 rf_mx_round8(const uint4 v, const int* e) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// The same rounding, the eight values returned as floats (exact: E2M1 times a
+// power of two).
+template <class Dec>
+__device__ __forceinline__ void rf_mx_round8f(const uint4 v, const int* e, float* y) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int e0 = e[2 * c], e1 = e[2 * c + 1];
+    const uint32_t h = rf_e2m1x2_round(rf_scale_pow2(Dec::lo(w[c]), -e0), rf_scale_pow2(Dec::hi(w[c]), -e1));
+    y[2 * c] = rf_scale_pow2(__half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu))), e0);
+    y[2 * c + 1] = rf_scale_pow2(__half2float(__ushort_as_half((unsigned short)(h >> 16))), e1);
+  }
+}
+
 // Four floats to four E4M3 codes (round to nearest even, saturating at
 // +-448), the first in the lowest byte.
 __device__ __forceinline__ uint32_t rf_e4m3x4(float a, float b, float c, float d) {
@@ -161,6 +175,10 @@ __global__ void __launch_bounds__(kThreads)
   }
   if constexpr (kQuant == kQuantMx && (MODE == kRearrange || MODE == kQuantOnly)) {
     constexpr bool kInBf16 = Dec::kBf16;
+    // D = 128: the rounded values are stored as E4M3 codes (every MXFP4 value
+    // c * 2^e with -8 <= e <= 6 is one), Q' and K' one byte per element in
+    // their layouts, V' transposed per block like precision fp8's.
+    constexpr bool kMx8 = D == 128;
     if (tensor < 2) {
       // Q and K: every row in groups of 32 columns.  A group is four 16-byte
       // chunks, held by four consecutive lanes (kChunks is a multiple of 4).
@@ -175,7 +193,17 @@ __global__ void __launch_bounds__(kThreads)
         mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
         const int e1 = rf_uos_exponent(Dec::lo(mb));
         const int e[8] = {e1, e1, e1, e1, e1, e1, e1, e1};
-        if (rr < nrows) dstx[dst_off[rr] + ch] = rf_mx_round8<Dec, kInBf16>(val[i], e);
+        if constexpr (kMx8) {
+          if (rr < nrows) {
+            float y[8];
+            rf_mx_round8f<Dec>(val[i], e, y);
+            uint8_t* dst8 = tensor == 0 ? qo.q8 : qo.k8;
+            *reinterpret_cast<uint2*>(dst8 + dst_off[rr] * 8 + ch * 8) =
+                make_uint2(rf_e4m3x4(y[0], y[1], y[2], y[3]), rf_e4m3x4(y[4], y[5], y[6], y[7]));
+          }
+        } else {
+          if (rr < nrows) dstx[dst_off[rr] + ch] = rf_mx_round8<Dec, kInBf16>(val[i], e);
+        }
       }
     } else {
       // V: every column in groups of 32 rows counted from the block's first
@@ -187,6 +215,8 @@ __global__ void __launch_bounds__(kThreads)
       constexpr int kWords = D / 2;  // packed 16-bit pairs per row
       __shared__ uint32_t part[kGroups][kRowLanes][kWords];
       __shared__ uint32_t gmax[kGroups][kWords];
+      constexpr int kVTileStride = RF_BLOCK + 4;   // bytes per row of the transposed tile
+      __shared__ __align__(16) uint8_t vtile[kMx8 ? D * kVTileStride : 16];
 #pragma unroll
       for (int gi = 0; gi < kGroups; ++gi) {
         uint32_t m4[4] = {0u, 0u, 0u, 0u};
@@ -223,7 +253,28 @@ __global__ void __launch_bounds__(kThreads)
         for (int j = 0; j < kRowsPerGroup; ++j) {
           const int i = gi * kRowsPerGroup + j;
           const int rr = rl + i * kRowLanes;
-          if (rr < nrows) qo.vx[dst_off[rr] + ch] = rf_mx_round8<Dec, false>(val[i], e);
+          if constexpr (kMx8) {
+            // rows past nrows hold zeros: code 0
+            float y[8];
+            rf_mx_round8f<Dec>(val[i], e, y);
+#pragma unroll
+            for (int c = 0; c < 8; c += 2) {
+              unsigned short two;
+              asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(two) : "f"(y[c + 1]), "f"(y[c]));
+              vtile[(ch * 8 + c) * kVTileStride + rr] = (uint8_t)(two & 0xFFu);
+              vtile[(ch * 8 + c + 1) * kVTileStride + rr] = (uint8_t)(two >> 8);
+            }
+          } else {
+            if (rr < nrows) qo.vx[dst_off[rr] + ch] = rf_mx_round8<Dec, false>(val[i], e);
+          }
+        }
+      }
+      if constexpr (kMx8) {
+        __syncthreads();
+        uint32_t* out = reinterpret_cast<uint32_t*>(qo.v8 + ((size_t)head * g.t_qblk + tb) * (size_t)(RF_BLOCK * D));
+        for (int wd = threadIdx.x; wd < D * RF_BLOCK / 4; wd += kThreads) {
+          const int d = wd / (RF_BLOCK / 4), c4 = wd % (RF_BLOCK / 4);
+          out[wd] = *reinterpret_cast<const uint32_t*>(&vtile[d * kVTileStride + 4 * c4]);
         }
       }
     }
@@ -375,7 +426,11 @@ rf_status_t launch(const rf_plan* p, const void* q, const void* k, const void* v
     qout.q_scale = reinterpret_cast<float*>(w + p->off_qs);
     qout.k_scale = reinterpret_cast<float*>(w + p->off_ks);
   }
-  if (mx) {
+  if (mx && g.d == 128) {   // E4M3 carriers of the MXFP4 values
+    qout.q8 = reinterpret_cast<uint8_t*>(w + p->off_q8);
+    qout.k8 = reinterpret_cast<uint8_t*>(w + p->off_k8);
+    qout.v8 = reinterpret_cast<uint8_t*>(w + p->off_v8);
+  } else if (mx) {
     qout.qx = reinterpret_cast<uint4*>(w + p->off_qx);
     qout.kx = reinterpret_cast<uint4*>(w + p->off_kx);
     qout.vx = reinterpret_cast<uint4*>(w + p->off_vx);

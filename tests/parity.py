@@ -74,16 +74,38 @@ def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "fro
 
 
 def mx_buffers(plan: rf.Plan, ws: torch.Tensor) -> Dict[str, np.ndarray]:
-    """Host copies (16-bit patterns) of the MXFP4 copies of Q', K' (plan dtype) and V' (f16)."""
+    """float64 values of the MXFP4 copies of Q', K', V' in the layouts of q_r, k_r, v_r:
+    at head dim 128 decoded from their E4M3 carriers (Q', K' one byte per element, V'
+    transposed per block), else from the 16-bit copies (Q', K' plan dtype, V' f16)."""
     info = plan.info
     ws8 = ws.view(torch.uint8)
     rows, d = int(info.rows_total), plan.d
+    if d == 128:
+        def bytes_(off, n):
+            return ws8[int(off):int(off) + n].cpu().numpy()
+        qx = orc.e4m3_decode(bytes_(info.ws_q8, rows * plan.n1 * d).reshape(plan.tensor_shape(plan.n1)))
+        kx = orc.e4m3_decode(bytes_(info.ws_k8, rows * plan.n2 * d).reshape(plan.tensor_shape(plan.n2)))
+        t = int(info.t_qblk)
+        raw = bytes_(info.ws_v8, plan.n2 * t * 128 * d).reshape(plan.n2, t, d, 128)
+        p = problem_of_plan(plan)
+        vx = np.zeros(plan.tensor_shape(plan.n2), dtype=np.float64)
+        for tb, (s, g, b) in enumerate(orc.qblock_table(p)):
+            r = orc.block_rows(g, b)
+            for n in range(plan.n2):
+                p.head_rows(vx, s, n)[r.start:r.stop] = orc.e4m3_decode(raw[n, tb, :, :len(r)].T)
+        return dict(qx=qx, kx=kx, vx=vx)
 
-    def region(off, heads):
+    def region(off, heads, dt):
         n = rows * heads * d * 2
-        return ws8[int(off):int(off) + n].cpu().numpy().view(np.uint16).reshape(plan.tensor_shape(heads))
-    return dict(qx=region(info.ws_q_mx, plan.n1), kx=region(info.ws_k_mx, plan.n2),
-                vx=region(info.ws_v_mx, plan.n2))
+        bits = ws8[int(off):int(off) + n].cpu().numpy().view(np.uint16).reshape(plan.tensor_shape(heads))
+        return synth.bits_to_float64(bits, dt)
+    return dict(qx=region(info.ws_q_mx, plan.n1, plan.dtype), kx=region(info.ws_k_mx, plan.n2, plan.dtype),
+                vx=region(info.ws_v_mx, plan.n2, "fp16"))
+
+
+def problem_of_plan(plan: rf.Plan) -> orc.Problem:
+    return orc.make_problem(plan.layout, plan.batch, plan.seqs, plan.n1, plan.n2, plan.d, plan.sparsity,
+                            plan.order)
 
 
 def oracle_mx_inputs(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray]):
@@ -95,10 +117,11 @@ def oracle_mx_inputs(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarr
 
 
 def check_mx_quantization(p: orc.Problem, w: synth.Workload, ref, gpu) -> None:
-    """The MXFP4 copies equal the oracle's rounding value for value (Q', K' in the input
-    type, V' in f16; every MXFP4 value of these inputs is exact in either)."""
-    for name, x, dt in (("qx", ref[0], w.dtype), ("kx", ref[1], w.dtype), ("vx", ref[2], "fp16")):
-        got = synth.bits_to_float64(gpu[name], dt)
+    """The MXFP4 copies equal the oracle's rounding value for value (carried as E4M3 at
+    head dim 128, else Q', K' in the input type and V' in f16; every MXFP4 value of
+    these inputs is exact in each)."""
+    for name, x in (("qx", ref[0]), ("kx", ref[1]), ("vx", ref[2])):
+        got = gpu[name]
         diff = got != x
         assert not diff.any(), f"{name}: {int(diff.sum())} values differ, e.g. {got[diff][:4]} vs {x[diff][:4]}"
 

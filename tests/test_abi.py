@@ -246,15 +246,25 @@ def test_quantize_needs_a_mix_plan():
                                                  ("TND", [(256, 13, 32, 48), (384, 21, 24, 40)], 32, 8, 128),
                                                  ("BNSD", [(128, 9, 16, 32)], 2, 2, 64)])
 def test_mxfp4_precision_workspace_layout(layout, seqs, n1, n2, d):
-    """The MXFP4 copies of Q', K', V' sit after the native workspace, 256-byte aligned,
-    two bytes per element each; the other mix fields stay -1."""
+    """The MXFP4 copies of Q', K', V' sit after the native workspace, 256-byte aligned:
+    at head dim 128 as E4M3 carriers (one byte per element of Q' and K' in their layouts,
+    V' transposed per block; no scales), else two bytes per element each."""
     nat = rf.Plan(seqs, n1, n2, d, layout, "bf16", 0.8)
     mx = rf.Plan(seqs, n1, n2, d, layout, "bf16", 0.8, precision="mxfp4")
     a, b = nat.info, mx.info
     assert b.precision == 3
     assert a.ws_q_mx == a.ws_k_mx == a.ws_v_mx == -1
-    assert b.ws_q8 == b.ws_k8 == b.ws_q_scale == b.ws_k_scale == -1
+    assert b.ws_q_scale == b.ws_k_scale == b.ws_v_exp == -1
     rows = int(b.rows_total)
+    if d == 128:
+        t = int(b.t_qblk)
+        assert b.ws_q_mx == b.ws_k_mx == b.ws_v_mx == -1
+        assert b.ws_q8 >= a.workspace_bytes and b.ws_q8 % 256 == 0
+        assert b.ws_k8 >= b.ws_q8 + rows * n1 * d and b.ws_k8 % 256 == 0
+        assert b.ws_v8 >= b.ws_k8 + rows * n2 * d and b.ws_v8 % 256 == 0
+        assert b.workspace_bytes >= b.ws_v8 + n2 * t * 128 * d
+        return
+    assert b.ws_q8 == b.ws_k8 == b.ws_v8 == -1
     assert b.ws_q_mx >= a.workspace_bytes and b.ws_q_mx % 256 == 0
     assert b.ws_k_mx >= b.ws_q_mx + rows * n1 * d * 2 and b.ws_k_mx % 256 == 0
     assert b.ws_v_mx >= b.ws_k_mx + rows * n2 * d * 2 and b.ws_v_mx % 256 == 0

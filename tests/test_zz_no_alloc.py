@@ -85,7 +85,7 @@ def test_noalloc_accepts_a_quantized_plan_whose_selection_part_fits(precision):
     w = CASES["wan"]
     bits = synth.generate_qkv(w)
     plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, precision=precision)
-    first = plan.info.ws_q8 if precision == "mix" else plan.info.ws_q_mx
+    first = min(o for o in (plan.info.ws_q8, plan.info.ws_q_mx) if o >= 0)   # the first quantized region
     assert plan.workspace_bytes > 32 << 20 and first <= 32 << 20
     q, k, v = (parity.to_device(x, w.dtype) for x in bits)
     b = rf.Buffers(plan)
