@@ -15,15 +15,16 @@
 // first frame) come first.
 //
 // Warp roles (384 threads = three warpgroups):
-//   warps 0-3  softmax warpgroup 0: the even-numbered selected blocks
-//   warps 4-7  softmax warpgroup 1: the odd-numbered selected blocks
+//   warps 0-3  softmax group 0: the even-numbered selected blocks
+//   warps 4-7  softmax group 1: the odd-numbered selected blocks
 //              (thread = query row = TMEM lane in both groups)
 //   warp 8     TMA producer of Q (once) and K_j through a 3-stage ring
 //   warp 9     TMEM allocation and the tcgen05.mma issue of S_j = Q K_j^T
-//   warp 10    TMA producer of V_j through a 2-stage ring (K and V have
-//              separate producers so that a K load never queues behind a V
-//              load that waits for an earlier P V product)
-//   warp 11    the tcgen05.mma issue of O += P_j V_j
+//   warp 10    TMA producer of V_j through a 2-stage ring (3 stages with
+//              one-byte Q and K, 4 with one-byte V); K and V have separate
+//              producers so that a K load never queues behind a V load that
+//              waits for an earlier P V product
+//   warp 11    the tcgen05.mma issue of O_w += P_j V_j
 // One elected thread per issuing warp issues that warp's MMAs.  A single
 // issuing thread cannot keep the tensor pipe busy at M = N = 128: every
 // barrier check costs it about as much as an MMA's worth of pipe time.
@@ -31,20 +32,21 @@
 // gives registers back (72 each) and the softmax groups take them (216 each),
 // so that a thread holds its whole 128-column score row: 2*128*216 + 128*72
 // = 384*168.
-// TMEM columns: S_w at [128 w, 128 w + 128) and O_w at [256 + 128 w, +D) for
-// softmax group w.  P_j is written back over its own score buffer as packed
-// 16-bit pairs and is the A operand (from TMEM) of O_w += P_j V_j.
-// S_j goes into buffer j % 2 once P_{j-2} V_{j-2} (which reads P_{j-2} from
-// it) is complete, so a group's chain is S_j -> softmax -> P_j V_j -> S_{j+2};
-// the two groups alternate, and one group's softmax overlaps the other
-// group's products.  P_j V_j goes in two halves of the key rows: the softmax
-// releases the first 64 columns of P_j before computing the rest.
+// TMEM columns: one score buffer S at [0, 128); P of group w at
+// [128 + 64 w, +64) (128 keys as packed 16-bit pairs, or 32 columns of four
+// E4M3 codes); O_w, the accumulator of group w, at [256 + 128 w, +D).
+// S_j goes into the score buffer as soon as the softmax has read S_{j-1} into
+// registers, so the next block's Q K^T runs while this block's softmax does.
+// P_j is the A operand (from TMEM) of O_w += P_j V_j, issued in two halves of
+// the key rows: the softmax releases the first 64 keys of P_j before it
+// computes the rest.  P buffer w and O_w take block j + 2 once
+// P_j V_j is complete.
 // Each group keeps its own running max, sum and accumulator over its half of
 // the blocks, so the groups never wait for each other; the epilogue merges
 // the two halves (a fixed split, so the result is deterministic).  O_w is
 // rescaled only when a row max grows by more than 2^8 (a warp-uniform
 // decision), right after the row max and before any of P_j is released (O_w
-// is at rest then: S_j was issued after the group's previous P V was complete).
+// is at rest then: the group waits for its previous P V product first).
 // The softmax works in the exp2 domain.  Column pairs selected by
 // RF_EMU_PAIR_MASK take their exponentials from a polynomial on the FMA pipe
 // (rf_exp2_poly2, two values per paired instruction) instead of the MUFU unit,
@@ -62,7 +64,16 @@
 // accumulates the row sum from the rounded values (PNQ) and hands P V the
 // rounded values times 2^e as f16.  Power-of-two scales make the rounded P
 // independent of which integer the running max is, so the result does not
-// depend on the order the blocks are visited in.
+// depend on the order the blocks are visited in.  At head dim 128 the MXFP4
+// values travel instead as E4M3 codes (an E2M1 value times a power of two in
+// range is exact in E4M3), so both products run on the FP8 tensor cores
+// (kind::f8f6f4) with unit scales.
+//
+// Precisions "mix" and "fp8" (user guide, "Configuration"): Q K^T on E4M3
+// copies of Q and K with one fp32 scale per (head, block), folded into the
+// exponent scale of S_j; "fp8" also runs P V on E4M3: V' per (head, block)
+// with a power-of-two scale 2^e_j, and P quantized per block as
+// P * 2^(e_j - e_max) so that one output scale 2^e_max serves every block.
 #include <cuda.h>
 #include <cuda_fp16.h>
 
