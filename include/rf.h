@@ -128,21 +128,25 @@ typedef struct {
   int32_t n1, n2, d;
   int32_t precision;       /* rf_precision_t of the plan */
   int32_t token_order;     /* rf_token_order_t of the plan */
-  /* RF_PRECISION_MIX only (else -1): byte offsets in ws of the E4M3 copies of
-   * Q' and K' (uint8, same layout and strides as q_r / k_r with one byte per
-   * element) and of their scales (fp32 [n1][t_qblk] and [n2][t_qblk], indexed
-   * by global query-block number). */
+  /* RF_PRECISION_MIX and RF_PRECISION_FP8 (else -1): byte offsets in ws of the
+   * E4M3 copies of Q' and K' (uint8, same layout and strides as q_r / k_r with
+   * one byte per element) and of their scales (fp32 [n1][t_qblk] and
+   * [n2][t_qblk], indexed by global query-block number).  RF_PRECISION_MXFP4 at
+   * head dim 128 uses ws_q8 and ws_k8 for its E4M3-carried MXFP4 values and has
+   * no scales (ws_q_scale = ws_k_scale = -1). */
   int64_t ws_q8, ws_k8, ws_q_scale, ws_k_scale;
-  /* RF_PRECISION_MXFP4 only (else -1): byte offsets in ws of the MXFP4-rounded
-   * copies of Q', K' (the inputs' 16-bit type) and V' (always f16), each with
-   * the layout and strides of q_r / k_r / v_r. */
+  /* RF_PRECISION_MXFP4 at head dim 64 only (else -1): byte offsets in ws of
+   * the MXFP4-rounded copies of Q', K' (the inputs' 16-bit type) and V' (always
+   * f16), each with the layout and strides of q_r / k_r / v_r. */
   int64_t ws_q_mx, ws_k_mx, ws_v_mx;
   /* RF_PRECISION_FP8 only (else -1): byte offsets in ws of the E4M3 codes of V'
    * and of their exponents.  The codes are stored transposed per block, uint8
    * [n2][t_qblk][d][128]: for head h and global block t, column c of the block
    * holds its 128 keys contiguously (rows past a partial block's end are 0).
    * The exponents are int32 [n2][t_qblk]: the codes of block t of head h
-   * represent code * 2^exp. ws_q8 .. ws_k_scale are as for RF_PRECISION_MIX. */
+   * represent code * 2^exp. ws_q8 .. ws_k_scale are as for RF_PRECISION_MIX.
+   * RF_PRECISION_MXFP4 at head dim 128 stores its E4M3-carried V' in ws_v8 in
+   * the same transposed layout, with no exponents (ws_v_exp = -1). */
   int64_t ws_v8, ws_v_exp;
 } rf_plan_info_t;
 
@@ -226,15 +230,23 @@ RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int
  *                        rows in groups of 32 columns; V columns and P rows in
  *                        groups of 32 keys counted from the first row of each
  *                        key block.  rf_rearrange (or rf_quantize_mx) writes the
- *                        rounded Q', K', V' into the workspace as exact 16-bit
- *                        values (V' as f16; values that would round past 65504
- *                        saturate there).  The softmax takes the exponentials
- *                        against an integer running maximum (log2 units), rounds
- *                        each group of 32 of them to MXFP4 the same way, and sums
- *                        the rounded values into the row sum, so the weights that
- *                        multiply V' sum to one exactly; P V runs in f16.  The
- *                        products use the 16-bit tensor cores, on which every
- *                        MXFP4 value is exact.  Head dim 64 or 128. */
+ *                        rounded Q', K', V' into the workspace.  The softmax
+ *                        takes the exponentials against an integer running
+ *                        maximum (log2 units), rounds each group of 32 of them to
+ *                        MXFP4 the same way, and sums the rounded values into the
+ *                        row sum, so the weights that multiply V' sum to one
+ *                        exactly.  Head dim 128: the rounded values are stored as
+ *                        E4M3 codes (an MXFP4 value c * 2^e is an E4M3 value for
+ *                        -8 <= e <= 6; outside that range it rounds to the
+ *                        nearest E4M3 value, saturating at 448), Q' and K' in
+ *                        their layouts, V' transposed per block as for
+ *                        RF_PRECISION_FP8; P enters
+ *                        P V as E4M3 of the rounded values times 2^8 and the
+ *                        output is multiplied by 2^-8; both products run on the
+ *                        FP8 tensor cores (kind::f8f6f4) with unit scales.  Head
+ *                        dim 64: exact 16-bit copies (V' as f16; values that
+ *                        would round past 65504 saturate there) on the 16-bit
+ *                        tensor cores, P V in f16. */
 typedef enum {
   RF_PRECISION_NATIVE = 0,
   RF_PRECISION_MIX = 1,
