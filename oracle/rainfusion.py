@@ -16,7 +16,7 @@ Sources (the web pages this path is described on):
         Block-wise Sparse Attention", abstract.
 
 Where the pages leave a step open, the reading taken is stated beside the code
-(R1..R14 below are the same readings listed in the design notes).
+(R1..R26 below are the same readings listed in the design notes).
 
 Pins (what ties this oracle to something other than itself) live in
 tests/test_oracle_*.py: the worked MiniMax geometry from [UG] "Geometry
@@ -60,6 +60,7 @@ class SeqGeometry:
     k: int            # ranked key blocks kept per sparse query block
     dense: bool       # the whole sequence runs dense (nb < 32)
     order: str = "tile"  # token order of the aligned video: "tile" or "frame_pair"
+    sparsity: float = 0.0  # the nominal dropped fraction the keep counts come from
 
     @property
     def n_blocks(self) -> int:
@@ -106,7 +107,7 @@ def geometry(prefix_len: int, t: int, h: int, w: int, sparsity: float,
     dense = nb < DENSE_MIN_BLOCKS
     k = nb if dense else keep_count(nb, sparsity)
     return SeqGeometry(prefix_len, t, h, w, h8, w8, aligned, sparse, promoted, lp,
-                       lp + sparse, n_pb, nb, ns, k, dense, order)
+                       lp + sparse, n_pb, nb, ns, k, dense, order, sparsity)
 
 
 # --------------------------------------------------------------------------------------
@@ -219,11 +220,40 @@ def kv_block_count(g: SeqGeometry, block_kv: int = BLOCK) -> int:
     return -(-g.lp // block_kv) + g.sparse // block_kv
 
 
-def block_means(x_r: np.ndarray, g: SeqGeometry) -> np.ndarray:
-    """[nb, D] float64 means of each sparse-region block of one head's rows x_r [L, D]."""
-    out = np.zeros((g.nb, x_r.shape[-1]), dtype=np.float64)
-    for i in range(g.nb):
-        rows = block_rows(g, g.n_pb + i)
+@dataclasses.dataclass(frozen=True)
+class KeyBlocks:
+    """Key-side block counts of one sequence when key blocks hold block_kv rows
+    (reading R26).  With block_kv = 128 they are the sequence's own n_pb, nb,
+    ns and k."""
+    block_kv: int
+    n_pb: int         # prefix key blocks, ceil(Lp / block_kv)
+    nb: int           # sparse-region key blocks, S / block_kv
+    ns: int           # first-frame sink key blocks, min(nb, ceil(h8 * w8 / block_kv))
+    k: int            # ranked key blocks kept per sparse query block (nb if dense)
+
+
+def key_blocks(g: SeqGeometry, block_kv: int = BLOCK) -> KeyBlocks:
+    """Reading R26 (blockShape 128 x block_kv, [API] "Formula"): key blocks of
+    block_kv rows tile the prefix and the sparse region like kv_block_rows; the
+    sinks are the key blocks holding first-frame tokens (the first frame leads
+    the sparse region, [UG] opening paragraphs); k keeps the same nominal
+    fraction of the key blocks (R4); a dense sequence (fewer than 32 query
+    blocks of 128 rows, [UG]) keeps every key block."""
+    n_pb = -(-g.lp // block_kv)
+    nb = g.sparse // block_kv
+    ns = min(nb, -(-(g.h8 * g.w8) // block_kv))
+    k = nb if g.dense else keep_count(nb, g.sparsity)
+    return KeyBlocks(block_kv, n_pb, nb, ns, k)
+
+
+def block_means(x_r: np.ndarray, g: SeqGeometry, block_kv: int = BLOCK) -> np.ndarray:
+    """[S / block_kv, D] float64 means of each sparse-region block of block_kv rows
+    of one head's rows x_r [L, D] (query blocks and, by default, key blocks hold
+    128 rows; reading R26 pools key blocks of 64 rows over their own rows)."""
+    kb = key_blocks(g, block_kv)
+    out = np.zeros((kb.nb, x_r.shape[-1]), dtype=np.float64)
+    for i in range(kb.nb):
+        rows = kv_block_rows(g, kb.n_pb + i, block_kv)
         out[i] = np.asarray(x_r[rows.start:rows.stop], dtype=np.float64).mean(axis=0)
     return out
 
@@ -244,10 +274,13 @@ def topk_blocks(scores: np.ndarray, k: int) -> List[int]:
     return order[:k].tolist()
 
 
-def select_sequence(qbar: np.ndarray, kbar: np.ndarray, g: SeqGeometry) -> Tuple[np.ndarray, np.ndarray]:
-    """selectIdx [n_blocks, N1, n_blocks] (-1 padded) and selectNum [n_blocks, N1] for one sequence.
+def select_sequence(qbar: np.ndarray, kbar: np.ndarray, g: SeqGeometry,
+                    block_kv: int = BLOCK) -> Tuple[np.ndarray, np.ndarray]:
+    """selectIdx [n_blocks, N1, key blocks] (-1 padded) and selectNum [n_blocks, N1] for one sequence.
 
-    qbar: [N1, nb, D], kbar: [N2, nb, D] float64 block means.
+    qbar: [N1, nb, D] float64 means of the 128-row query blocks; kbar: [N2,
+    S / block_kv, D] float64 means of the key blocks (block_kv rows, reading
+    R26; key-side counts from key_blocks).
     * Prefix query blocks and first-frame query blocks are dense ([UG]: prefix
       rows and first-frame blocks remain dense; reading R6).
     * Every other video query block i on head n ranks video key blocks j by
@@ -260,19 +293,21 @@ def select_sequence(qbar: np.ndarray, kbar: np.ndarray, g: SeqGeometry) -> Tuple
     """
     n1, n2 = qbar.shape[0], kbar.shape[0]
     G = n1 // n2
+    kb = key_blocks(g, block_kv)
     nblk = g.n_blocks
-    idx = np.full((nblk, n1, nblk), -1, dtype=np.int32)
+    nkv = kb.n_pb + kb.nb
+    idx = np.full((nblk, n1, nkv), -1, dtype=np.int32)
     num = np.zeros((nblk, n1), dtype=np.int32)
-    everything = list(range(nblk))
+    everything = list(range(nkv))
     for n in range(n1):
-        scores = qbar[n] @ kbar[n // G].T          # [nb, nb]: scores[i, j] = qbar_i . kbar_j
+        scores = qbar[n] @ kbar[n // G].T          # [nb, kb.nb]: scores[i, j] = qbar_i . kbar_j
         for qb in range(nblk):
             i = qb - g.n_pb
             if g.dense or qb < g.n_pb or i < g.ns:
                 row = everything
             else:
-                keep = set(topk_blocks(scores[i], g.k)) | set(range(g.ns))
-                row = list(range(g.n_pb)) + [g.n_pb + j for j in sorted(keep)]
+                keep = set(topk_blocks(scores[i], kb.k)) | set(range(kb.ns))
+                row = list(range(kb.n_pb)) + [kb.n_pb + j for j in sorted(keep)]
             idx[qb, n, :len(row)] = row
             num[qb, n] = len(row)
     return idx, num
@@ -386,24 +421,27 @@ def inverse_rearrange(p: Problem, y: np.ndarray) -> np.ndarray:
     return x
 
 
-def pooled_means(p: Problem, x_r: np.ndarray, heads: int) -> List[np.ndarray]:
-    """Per sequence, [heads, nb, D] float64 block means of the rearranged x_r."""
+def pooled_means(p: Problem, x_r: np.ndarray, heads: int, block_kv: int = BLOCK) -> List[np.ndarray]:
+    """Per sequence, [heads, S / block_kv, D] float64 block means of the rearranged x_r."""
     out = []
     for s, g in p.sequences():
-        out.append(np.stack([block_means(p.head_rows(x_r, s, n), g) for n in range(heads)])
-                   if g.nb else np.zeros((heads, 0, p.d)))
+        nbk = g.sparse // block_kv
+        out.append(np.stack([block_means(p.head_rows(x_r, s, n), g, block_kv) for n in range(heads)])
+                   if nbk else np.zeros((heads, 0, p.d)))
     return out
 
 
-def select(p: Problem, qbars: List[np.ndarray], kbars: List[np.ndarray]) -> Tuple[np.ndarray, np.ndarray]:
-    """selectIdx [T_qblk, N1, maxKv] and selectNum [T_qblk, N1] over all sequences ([API])."""
-    maxkv = p.max_kv_blocks
+def select(p: Problem, qbars: List[np.ndarray], kbars: List[np.ndarray],
+           block_kv: int = BLOCK) -> Tuple[np.ndarray, np.ndarray]:
+    """selectIdx [T_qblk, N1, maxKv] and selectNum [T_qblk, N1] over all sequences ([API]);
+    with block_kv = 64 the entries and maxKv count 64-row key blocks (reading R26)."""
+    maxkv = max(kv_block_count(g, block_kv) for g in p.geoms)
     idx = np.full((p.t_qblk, p.n1, maxkv), -1, dtype=np.int32)
     num = np.zeros((p.t_qblk, p.n1), dtype=np.int32)
     t0 = 0
     for (s, g), qb, kb in zip(p.sequences(), qbars, kbars):
-        i_s, n_s = select_sequence(qb, kb, g)
-        idx[t0:t0 + g.n_blocks, :, :g.n_blocks] = i_s
+        i_s, n_s = select_sequence(qb, kb, g, block_kv)
+        idx[t0:t0 + g.n_blocks, :, :i_s.shape[2]] = i_s
         num[t0:t0 + g.n_blocks] = n_s
         t0 += g.n_blocks
     return idx, num
@@ -450,24 +488,26 @@ def assemble_output(p: Problem, parts: Dict[Tuple[int, int], np.ndarray], like: 
     return o
 
 
-def run_path(p: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> Dict[str, object]:
-    """Whole path on float64 inputs in original order: permute, pool, select, attend, un-permute."""
+def run_path(p: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+             block_kv: int = BLOCK) -> Dict[str, object]:
+    """Whole path on float64 inputs in original order: permute, pool, select, attend, un-permute
+    (key blocks of block_kv rows, reading R26)."""
     q_r, k_r, v_r = rearrange(p, q), rearrange(p, k), rearrange(p, v)
-    qbars, kbars = pooled_means(p, q_r, p.n1), pooled_means(p, k_r, p.n2)
-    idx, num = select(p, qbars, kbars)
-    o_r = assemble_output(p, attention(p, q_r, k_r, v_r, idx, num, scale), q_r)
+    qbars, kbars = pooled_means(p, q_r, p.n1), pooled_means(p, k_r, p.n2, block_kv)
+    idx, num = select(p, qbars, kbars, block_kv)
+    o_r = assemble_output(p, attention(p, q_r, k_r, v_r, idx, num, scale, block_kv=block_kv), q_r)
     return dict(q_r=q_r, k_r=k_r, v_r=v_r, qbar=qbars, kbar=kbars, idx=idx, num=num,
                 o_r=o_r, o=inverse_rearrange(p, o_r))
 
 
-def kept_flops(p: Problem, idx: np.ndarray, num: np.ndarray) -> int:
+def kept_flops(p: Problem, idx: np.ndarray, num: np.ndarray, block_kv: int = BLOCK) -> int:
     """4 * D * (query rows) * (valid key rows) summed over selected (q-block, head, key block)."""
     table = qblock_table(p)
     total = 0
     for t, (s, g, b) in enumerate(table):
         mq = len(block_rows(g, b))
         for n in range(p.n1):
-            kv = sum(len(block_rows(g, int(j))) for j in idx[t, n, :num[t, n]])
+            kv = sum(len(kv_block_rows(g, int(j), block_kv)) for j in idx[t, n, :num[t, n]])
             total += 4 * p.d * mq * kv
     return total
 

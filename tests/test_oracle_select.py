@@ -124,3 +124,128 @@ def test_multi_sequence_select_pads_to_max():
     tail = idx[p.geoms[0].n_blocks:]
     assert np.all(tail[:, :, g1.n_blocks:] == -1)
     assert np.all(num[p.geoms[0].n_blocks:] == g1.n_blocks)
+
+
+# ---- key blocks of 64 rows (blockShape 128 x 64; reading R26) ----
+
+@pytest.mark.parametrize("geom", [(100, 9, 16, 32, 0.8), (64, 9, 16, 32, 0.9), (0, 21, 48, 80, 0.5),
+                                  (10, 2, 16, 16, 0.9), (7, 13, 27, 45, 0.8)])
+def test_key_blocks_of_128_rows_are_the_sequence_counts(geom):
+    g = rf.geometry(*geom)
+    kb = rf.key_blocks(g, 128)
+    assert (kb.n_pb, kb.nb, kb.ns, kb.k) == (g.n_pb, g.nb, g.ns, g.k)
+
+
+def test_key_blocks_of_64_rows_closed_forms():
+    # P = 100, (9, 16, 32): Lp = 100, S = 36 * 128 = 4608, first frame 16 * 32 = 512 tokens
+    kb = rf.key_blocks(rf.geometry(100, 9, 16, 32, 0.8), 64)
+    assert (kb.n_pb, kb.nb, kb.ns, kb.k) == (2, 72, 8, 15)        # ceil(100/64), 4608/64, 512/64, ceil(14.4)
+    kb = rf.key_blocks(rf.geometry(64, 9, 16, 32, 0.9), 64)
+    assert (kb.n_pb, kb.nb, kb.ns, kb.k) == (1, 72, 8, 8)         # ceil(0.1 * 72) = ceil(7.2)
+    kb = rf.key_blocks(rf.geometry(0, 21, 48, 80, 0.8), 64)       # the Aligned grid, no text
+    assert (kb.n_pb, kb.nb, kb.ns, kb.k) == (0, 1260, 60, 252)
+    kb = rf.key_blocks(rf.geometry(10, 2, 16, 16, 0.9), 64)       # 4 blocks of 128: dense
+    assert (kb.n_pb, kb.nb, kb.ns, kb.k) == (1, 8, 4, 8)
+
+
+def test_block_means_of_64_rows_brute_force():
+    g = rf.geometry(100, 8, 16, 32, 0.8)
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((g.length, 5))
+    m = rf.block_means(x, g, 64)
+    assert m.shape == (2 * g.nb, 5)
+    for i in range(2 * g.nb):
+        for c in range(5):
+            s = 0.0
+            for r in range(g.lp + 64 * i, g.lp + 64 * i + 64):
+                s += x[r, c]
+            assert abs(m[i, c] - s / 64) < 1e-12
+
+
+def _random_select64(p, t, h, w, s, n1=2, n2=2, d=8, seed=14):
+    g = rf.geometry(p, t, h, w, s)
+    kb = rf.key_blocks(g, 64)
+    rng = np.random.default_rng(seed)
+    qbar = rng.standard_normal((n1, g.nb, d))
+    kbar = rng.standard_normal((n2, kb.nb, d))
+    idx, num = rf.select_sequence(qbar, kbar, g, 64)
+    return g, kb, qbar, kbar, idx, num
+
+
+@pytest.mark.parametrize("s", [0.5, 0.8, 0.9])
+def test_kv64_selection_invariants(s):
+    g, kb, qbar, kbar, idx, num = _random_select64(100, 9, 16, 32, s)
+    nkv = kb.n_pb + kb.nb
+    assert idx.shape == (g.n_blocks, 2, nkv)
+    for qb in range(g.n_blocks):
+        for n in range(2):
+            row = idx[qb, n, :num[qb, n]].tolist()
+            assert np.all(idx[qb, n, num[qb, n]:] == -1)
+            assert row == sorted(row) and len(set(row)) == len(row)
+            assert row[:kb.n_pb] == list(range(kb.n_pb))            # prefix key blocks always kept
+            i = qb - g.n_pb
+            if qb < g.n_pb or i < g.ns:                             # dense query blocks (128-row units)
+                assert row == list(range(nkv))
+                continue
+            video = [b - kb.n_pb for b in row[kb.n_pb:]]
+            assert set(range(kb.ns)) <= set(video)                   # 64-row sinks kept
+            assert kb.n_pb + max(kb.k, kb.ns) <= num[qb, n] <= kb.n_pb + min(kb.k + kb.ns, kb.nb)
+            sc = qbar[n, i] @ kbar[n].T                              # 128-row query mean . 64-row key means
+            top = rf.topk_blocks(sc, kb.k)
+            assert set(top) <= set(video)
+            dropped = [j for j in range(kb.nb) if j not in video]
+            if dropped and top:
+                assert min(sc[top]) >= max(sc[dropped])
+
+
+@pytest.mark.parametrize("s", [0.5, 0.75])
+def test_kv64_selection_of_duplicated_halves_is_the_expanded_128_selection(s):
+    """Key rows whose two 64-row halves of every sparse 128-row block are equal give
+    equal 64-row means for both halves: the 64-row selection must then be the
+    128-row selection with every block replaced by the 64-row blocks that cover its
+    rows (here k64 = 2 k and ns64 = 2 ns, so nothing else can differ)."""
+    g = rf.geometry(100, 9, 16, 32, s)
+    kb = rf.key_blocks(g, 64)
+    assert kb.k == 2 * g.k and kb.ns == 2 * g.ns
+    rng = np.random.default_rng(15)
+    n1, n2, d = 4, 2, 8
+    k_r = rng.standard_normal((n2, g.length, d))
+    for j in range(g.nb):
+        r0 = g.lp + 128 * j
+        k_r[:, r0 + 64:r0 + 128] = k_r[:, r0:r0 + 64]
+    kbar64 = np.stack([rf.block_means(k_r[n], g, 64) for n in range(n2)])
+    assert np.array_equal(kbar64[:, 0::2], kbar64[:, 1::2])
+    qbar = rng.standard_normal((n1, g.nb, d))
+    idx64, num64 = rf.select_sequence(qbar, kbar64, g, 64)
+    idx128, num128 = rf.select_sequence(qbar, kbar64[:, 0::2], g)
+    cover = {}
+    for b in range(g.n_blocks):
+        rows = set(rf.block_rows(g, b))
+        cover[b] = [c for c in range(kb.n_pb + kb.nb) if rf.kv_block_rows(g, c, 64).start in rows]
+    for qb in range(g.n_blocks):
+        for n in range(n1):
+            want = [c for b in idx128[qb, n, :num128[qb, n]] for c in cover[int(b)]]
+            assert idx64[qb, n, :num64[qb, n]].tolist() == want
+
+
+def test_kv64_sparsity_zero_one_and_dense_sequence():
+    g, kb, _, _, idx, num = _random_select64(64, 9, 16, 32, 0.0)
+    assert np.all(num == kb.n_pb + kb.nb)
+    g, kb, _, _, idx, num = _random_select64(64, 9, 16, 32, 1.0)
+    for qb in range(g.n_pb + g.ns, g.n_blocks):
+        assert idx[qb, 0, :num[qb, 0]].tolist() == list(range(kb.n_pb + kb.ns))
+    g, kb, _, _, idx, num = _random_select64(10, 2, 16, 16, 0.9)
+    assert g.dense and np.all(num == kb.n_pb + kb.nb)
+
+
+def test_kv64_problem_select_pads_to_the_widest_sequence():
+    p = rf.make_problem("TND", 1, [(64, 9, 16, 32), (10, 2, 16, 16)], 2, 1, 8, 0.8)
+    rng = np.random.default_rng(16)
+    qb = [rng.standard_normal((2, g.nb, 8)) for g in p.geoms]
+    kb = [rng.standard_normal((1, 2 * g.nb, 8)) for g in p.geoms]
+    idx, num = rf.select(p, qb, kb, 64)
+    widths = [rf.kv_block_count(g, 64) for g in p.geoms]
+    assert idx.shape == (p.t_qblk, 2, max(widths))
+    tail = idx[p.geoms[0].n_blocks:]
+    assert np.all(tail[:, :, widths[1]:] == -1)
+    assert np.all(num[p.geoms[0].n_blocks:] == widths[1])
