@@ -164,57 +164,30 @@ def record_traffic(csv_path, key, scale, how):
 # ---------------------------------------------------------------------------------------
 
 def kept_flops_from_selection(plan, idx, num):
-    """4 * D * (query rows) * (valid key rows) over selected (q-block, head, key block)."""
+    """4 * D * (query rows) * (valid key rows) over selected (q-block, head, key block);
+    query blocks hold 128 rows, key blocks plan.block_kv (the last prefix block of
+    each kind possibly partial)."""
     total = 0
+    bk = plan.block_kv
     for si in plan.seq_info_all():
         nblk = si.n_pb + si.nb
-        lp, npb = int(si.lp), int(si.n_pb)
-        rows = np.full(nblk + 1, 128, dtype=np.int64)
-        rows[npb - 1] = lp - 128 * (npb - 1) if npb > 0 else 128
-        rows[nblk] = 0                                   # -1 entries map here
+        nkv = int(si.n_pb_kv) + int(si.nb_kv)
+        lp, npb, npk = int(si.lp), int(si.n_pb), int(si.n_pb_kv)
+        qrows = np.full(nblk, 128, dtype=np.int64)
+        if npb > 0:
+            qrows[npb - 1] = lp - 128 * (npb - 1)
+        krows = np.full(nkv + 1, bk, dtype=np.int64)
+        if npk > 0:
+            krows[npk - 1] = lp - bk * (npk - 1)
+        krows[nkv] = 0                                   # -1 entries map here
         t0 = int(si.qblk_offset)
         sel = idx[t0:t0 + nblk].astype(np.int64)
         n = num[t0:t0 + nblk]
         valid = np.arange(sel.shape[-1])[None, None, :] < n[:, :, None]
-        sel = np.where(valid & (sel >= 0), sel, nblk)
-        kv_rows = rows[sel].sum(axis=-1)                 # [nblk, N1]
-        q_rows = rows[:nblk][:, None]
-        total += int((4 * plan.d * q_rows * kv_rows).sum())
+        sel = np.where(valid & (sel >= 0), sel, nkv)
+        kv_rows = krows[sel].sum(axis=-1)                # [nblk, N1]
+        total += int((4 * plan.d * qrows[:, None] * kv_rows).sum())
     return total
-
-
-def expand_selection_kv64(plan, idx, num, width):
-    """The 128-row key-block selection rewritten over 64-row key blocks (every
-    selected block becomes the one or two 64-row blocks inside it, in order)."""
-    infos = plan.seq_info_all()
-    T, N, _ = idx.shape
-    out = np.full((T, N, width), -1, dtype=np.int32)
-    cnt = np.zeros((T, N), dtype=np.int32)
-    owner = []                                  # sequence of every global query block
-    for si in infos:
-        owner += [si] * (int(si.n_pb) + int(si.nb))
-    if plan.layout == "BNSD":
-        owner *= plan.batch                     # one geometry for every batch element
-    for t in range(T):
-        si = owner[t]
-        lp, n_pb = int(si.lp), int(si.n_pb)
-        n_pb64 = -(-lp // 64)
-        for n in range(N):
-            row = []
-            for bb in idx[t, n, :num[t, n]]:
-                bb = int(bb)
-                if bb < 0:
-                    continue
-                if bb < n_pb:
-                    row.append(2 * bb)
-                    if 128 * bb + 64 < lp:
-                        row.append(2 * bb + 1)
-                else:
-                    i = bb - n_pb
-                    row += [n_pb64 + 2 * i, n_pb64 + 2 * i + 1]
-            out[t, n, :len(row)] = row
-            cnt[t, n] = len(row)
-    return out, cnt
 
 
 def algorithmic_bytes(plan, elem=2):
@@ -518,16 +491,16 @@ def main():
     wr = synth.Workload(w.name, w.layout, w.dtype, w.batch, w.seqs, w.n1, w.n2, w.d, w.sparsity, w.seed + 7919 * rank)
     bits = synth.generate_qkv(wr)
     seqs = [(s.prefix_len, s.t, s.h, s.w) for s in w.seqs]
+    if args.block_kv == 64 and args.precision != "native":
+        raise SystemExit("--block-kv 64 runs native precision only")
     plan = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=args.order,
-                   precision=args.precision)
+                   precision=args.precision, block_kv=args.block_kv)
     tdt = plan.torch_dtype
     host = [torch.from_numpy(x.view(np.int16)).view(tdt).pin_memory() for x in bits]
     q, k, v = (h.to(dev) for h in host)
     b = rf.Buffers(plan, dev)
     scale = 1.0 / math.sqrt(w.d)
     stream = torch.cuda.current_stream(dev)
-
-    kv64 = None   # --block-kv 64: (plan, selectIdx, selectNum, workspace) over 64-row key blocks
 
     def step(ev=None):
         if ev is not None:
@@ -538,10 +511,7 @@ def main():
         rf.pool_select(plan, None, None, b.select_idx, b.select_num, b.ws)
         if ev is not None:
             ev[2].record(stream)
-        if kv64 is None:
-            rf.block_sparse_attn(plan, b.q_r, b.k_r, b.v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
-        else:
-            rf.block_sparse_attn(kv64[0], b.q_r, b.k_r, b.v_r, kv64[1], kv64[2], scale, b.o_r, kv64[3])
+        rf.block_sparse_attn(plan, b.q_r, b.k_r, b.v_r, b.select_idx, b.select_num, scale, b.o_r, b.ws)
         if ev is not None:
             ev[3].record(stream)
         rf.inverse_rearrange(plan, b.o_r, b.o)
@@ -551,18 +521,6 @@ def main():
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize(dev)
-    if args.block_kv == 64:
-        if args.precision != "native":
-            raise SystemExit("--block-kv 64 runs native precision only")
-        p64 = rf.Plan(seqs, w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=args.order,
-                      block_kv=64)
-        i64, n64 = expand_selection_kv64(plan, b.select_idx.cpu().numpy(), b.select_num.cpu().numpy(),
-                                         int(p64.info.max_kv_blocks))
-        kv64 = (p64, torch.from_numpy(i64).to(dev), torch.from_numpy(n64).to(dev),
-                torch.zeros(p64.workspace_bytes, dtype=torch.uint8, device=dev))
-        for _ in range(max(3, args.warmup)):
-            step()
-        torch.cuda.synchronize(dev)
     rf.raise_on_device_fault(plan, b.ws, "warm-up")
     flops = kept_flops_from_selection(plan, b.select_idx.cpu().numpy(), b.select_num.cpu().numpy())
     launches_per_step = 5 if any(not si.dense for si in plan.seq_info_all()) else 4
@@ -588,21 +546,19 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     per = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in evs])  # [steps, 4]
     rf.raise_on_device_fault(plan, b.ws, "timed steps")
-    if kv64 is not None:
-        rf.raise_on_device_fault(kv64[0], kv64[3], "timed steps (128 x 64)")
 
     # e2e: pinned host buffers through the public API (rf.rainfusion_attention, which
     # runs head chunks whose copies overlap the compute, then reads the status words);
     # copies inside the timed region, the result back on the host at the end of every step.
     e2e = None
-    # the public call has no 128 x 64 selection, so --block-kv 64 times the kernels only
-    if args.e2e_steps > 0 and kv64 is None:
+    if args.e2e_steps > 0:
         out_host = None
 
         def e2e_step():
             nonlocal out_host
             out_host = rf.rainfusion_attention(host[0], host[1], host[2], seqs, w.sparsity, w.layout, scale,
-                                               order=args.order, precision=args.precision, chunks=args.chunks)
+                                               order=args.order, precision=args.precision, chunks=args.chunks,
+                                               block_kv=args.block_kv)
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(dev)
@@ -690,8 +646,8 @@ def main():
                        **({"precision": "mix (E4M3 QK^T, 16-bit PV)"} if args.precision == "mix" else {}),
                        **({"precision": "fp8 (E4M3 QK^T and PV; V on power-of-two block scales)"}
                           if args.precision == "fp8" else {}),
-                       **({"block_shape": "128 x 64 (attention on the 64-row halves of the step's 128-row "
-                                          "selection, expanded once after warm-up)"} if args.block_kv == 64 else {}),
+                       **({"block_shape": "128 x 64 (64-row key blocks ranked against 128-row query "
+                                          "blocks)"} if args.block_kv == 64 else {}),
                        **({"precision": "mxfp4 (UOS Qmax 7.25, PNQ; values carried in E4M3 at head dim 128)"}
                           if args.precision == "mxfp4" else {}),
                        "global_batch": w.batch * world, "seq_len": int(plan.info.rows_total),

@@ -28,7 +28,13 @@ struct RfSeqDev {
   int n_pb, nb, ns, k, dense;
   int order;            // rf_token_order_t of the aligned video tokens
   int qblk_off;         // first global query block
-  int pool_off;         // first pooled block (sum of nb of earlier instances)
+  int pool_off;         // first pooled query block (sum of nb of earlier instances)
+  // Key side of the selection (block_kv rows per key block): prefix key
+  // blocks, sparse key blocks, first-frame sink key blocks, ranked blocks
+  // kept, and the first pooled key block.  With 128-row key blocks they are
+  // n_pb, nb, ns, k and pool_off.
+  int npk, nbk, nsk, kk;
+  int poolk_off;
 };
 
 struct RfGeomDev {
@@ -38,8 +44,10 @@ struct RfGeomDev {
   int t_qblk;
   int max_kv;
   int block_kv;         // key/value block rows: 128, or 64 ([API] blockShape 128 x 64)
-  int pooled_total;     // sum of nb over instances
+  int pooled_total;     // sum of nb over instances (query block means per head)
+  int pooled_k_total;   // sum of nbk over instances (key block means per head)
   int max_nb;
+  int max_nbk;
   RfSeqDev seq[RF_MAX_SEQS];
 };
 

@@ -66,8 +66,6 @@ extern "C" rf_status_t rf_pool_select_noalloc(const rf_plan_t* p, const void* q_
   if (!p) return rf_fail(RF_ERR_INVALID_ARG, "null plan");
   if (!q_r || !k_r || !select_idx || !select_num)
     return rf_fail(RF_ERR_INVALID_ARG, "null tensor");
-  if (p->g.block_kv != RF_BLOCK)
-    return rf_fail(RF_ERR_UNSUPPORTED, "selection ranks 128-row key blocks only");
   if ((reinterpret_cast<uintptr_t>(q_r) & 15) || (reinterpret_cast<uintptr_t>(k_r) & 15))
     return rf_fail(RF_ERR_INVALID_ARG, "q_r and k_r must be 16-byte aligned");
   // The selection part of the workspace layout (mix and mxfp4 plans put their

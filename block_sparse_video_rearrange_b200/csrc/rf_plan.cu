@@ -50,7 +50,23 @@ RfSeqDev seq_geometry(const rf_seq_geom_t& s, double sparsity, rf_token_order_t 
   if (d.ns > d.nb) d.ns = d.nb;
   d.dense = d.nb < RF_DENSE_MIN_BLOCKS ? 1 : 0;
   d.k = d.dense ? d.nb : keep_count(d.nb, sparsity);
+  d.npk = d.n_pb;
+  d.nbk = d.nb;
+  d.nsk = d.ns;
+  d.kk = d.k;
   return d;
+}
+
+// Key side of the selection with 64-row key blocks ([API] "Formula": blocks of
+// blockShapeX x blockShapeY): the prefix tiled from row 0 by ceil(Lp / 64)
+// key blocks, the sparse region by 2 nb; the sinks are the key blocks holding
+// first-frame tokens; k keeps the nominal fraction of the 64-row key blocks.
+void key_side_64(RfSeqDev& d, double sparsity) {
+  d.npk = rf_n_pb64(d);
+  d.nbk = 2 * d.nb;
+  d.nsk = (d.h8 * d.w8 + 63) / 64;
+  if (d.nsk > d.nbk) d.nsk = d.nbk;
+  d.kk = d.dense ? d.nbk : keep_count(d.nbk, sparsity);
 }
 
 }  // namespace
@@ -182,8 +198,8 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   g.d = d;
   g.n_seqs = layout == RF_LAYOUT_BNSD ? batch : n_seqs;
 
-  int64_t rows = 0, qblk = 0, pooled = 0, scores = 0, flops = 0;
-  int max_kv = 0, max_nb = 0;
+  int64_t rows = 0, qblk = 0, pooled = 0, pooled_k = 0, scores = 0, flops = 0;
+  int max_kv = 0, max_nb = 0, max_nbk = 0;
   for (int i = 0; i < g.n_seqs; ++i) {
     const rf_seq_geom_t& src = seqs[layout == RF_LAYOUT_BNSD ? 0 : i];
     RfSeqDev s = seq_geometry(src, sparsity, order);
@@ -192,16 +208,20 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
     s.qblk_off = (int)qblk;
     s.pool_off = (int)pooled;
     s.score_off = scores;
+    if (block_kv != RF_BLOCK) key_side_64(s, sparsity);
+    s.poolk_off = (int)pooled_k;
     g.seq[i] = s;
     int nblk = s.n_pb + s.nb;
     // selectIdx rows count key/value blocks of block_kv rows
-    const int nkv = block_kv == RF_BLOCK ? nblk : rf_n_pb64(s) + 2 * s.nb;
+    const int nkv = s.npk + s.nbk;
     if (nkv > max_kv) max_kv = nkv;
     if (s.nb > max_nb) max_nb = s.nb;
+    if (s.nbk > max_nbk) max_nbk = s.nbk;
     rows += s.L;
     qblk += nblk;
     pooled += s.nb;
-    if (!s.dense) scores += (int64_t)n1 * s.nb * s.nb;
+    pooled_k += s.nbk;
+    if (!s.dense) scores += (int64_t)n1 * s.nb * s.nbk;
     flops += 4ll * d * (int64_t)s.L * s.L * n1;
     if (layout == RF_LAYOUT_TND || i == 0) {
       rf_seq_info_t inf;
@@ -216,10 +236,14 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
       inf.k = s.k;
       inf.qblk_offset = s.qblk_off;
       inf.dense = s.dense;
+      inf.n_pb_kv = s.npk;
+      inf.nb_kv = s.nbk;
+      inf.ns_kv = s.nsk;
+      inf.k_kv = s.kk;
       p->info.push_back(inf);
     }
   }
-  if (max_kv > RF_MAX_KV_LIST || max_nb > RF_MAX_NB) {
+  if (max_kv > RF_MAX_KV_LIST || max_nb > RF_MAX_NB || max_nbk > RF_MAX_NB) {
     delete p;
     return rf_fail(RF_ERR_UNSUPPORTED, "a sequence has more than 2048 blocks (query or key/value)");
   }
@@ -231,19 +255,22 @@ rf_status_t rf_plan_create_ex(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t
   g.max_kv = max_kv;
   g.block_kv = block_kv;
   g.pooled_total = (int)pooled;
+  g.pooled_k_total = (int)pooled_k;
   g.max_nb = max_nb;
+  g.max_nbk = max_nbk;
   p->rows_total = layout == RF_LAYOUT_BNSD ? (int64_t)batch * g.seq[0].L : rows;
   p->kept_flops_upper = flops;
 
   // Workspace: [status words | pooled Q fp32 [N1][pooled][D] | pooled K fp32
-  // [N2][pooled][D] | block scores fp32, per non-dense sequence [N1][nb][nb]].
+  // [N2][pooled_k][D] | block scores fp32, per non-dense sequence [N1][nb][nbk]]
+  // (nbk = nb, or 2 nb with 64-row key blocks).
   int64_t off = 0;
   p->off_status = off;
   off += 256;
   p->off_pq = off;
   off = align_up(off + (int64_t)n1 * pooled * d * 4, 256);
   p->off_pk = off;
-  off = align_up(off + (int64_t)n2 * pooled * d * 4, 256);
+  off = align_up(off + (int64_t)n2 * pooled_k * d * 4, 256);
   p->off_scores = off;
   off = align_up(off + scores * 4, 256);
   // RF_PRECISION_MIX: E4M3 copies of Q' and K' (one byte per element, the
@@ -325,6 +352,7 @@ rf_status_t rf_plan_info(const rf_plan_t* p, rf_plan_info_t* out) {
   out->ws_v_mx = p->off_vx;
   out->ws_v8 = p->off_v8;
   out->ws_v_exp = p->off_vexp;
+  out->pooled_k_blocks = p->g.pooled_k_total;
   return RF_OK;
 }
 
@@ -425,9 +453,6 @@ rf_status_t rf_pool_select(const rf_plan_t* p, const void* q_r, const void* k_r,
   if (!select_idx || !select_num) return rf_fail(RF_ERR_INVALID_ARG, "null selectIdx/selectNum");
   if (pool_mode != RF_POOL_FROM_WS && pool_mode != RF_POOL_RECOMPUTE)
     return rf_fail(RF_ERR_INVALID_ARG, "bad pool mode");
-  if (p->g.block_kv != RF_BLOCK)
-    return rf_fail(RF_ERR_UNSUPPORTED, "selection ranks 128-row key blocks only; with blockShape 128 x 64 "
-                                       "the caller supplies selectIdx");
   if (pool_mode == RF_POOL_RECOMPUTE &&
       (!q_r || !k_r || !aligned16(q_r) || !aligned16(k_r)))
     return rf_fail(RF_ERR_INVALID_ARG, "recompute needs 16-byte aligned q_r and k_r");
@@ -480,9 +505,6 @@ rf_status_t rf_inverse_rearrange(const rf_plan_t* p, const void* o_r, void* o, r
 rf_status_t rf_forward(const rf_plan_t* p, const void* q, const void* k, const void* v, void* q_r,
                        void* k_r, void* v_r, int32_t* select_idx, int32_t* select_num, float scale,
                        void* o_r, void* o, void* ws, size_t ws_bytes, rf_stream_t stream) {
-  // Refuse before enqueuing anything when a later step would refuse.
-  if (p && p->g.block_kv != RF_BLOCK)
-    return rf_fail(RF_ERR_UNSUPPORTED, "rf_forward needs 128 x 128 blocks (selection ranks 128-row key blocks)");
   rf_status_t st = rf_rearrange(p, q, k, v, q_r, k_r, v_r, ws, ws_bytes, stream);
   if (st != RF_OK) return st;
   st = rf_pool_select(p, nullptr, nullptr, select_idx, select_num, ws, ws_bytes, RF_POOL_FROM_WS,

@@ -373,30 +373,44 @@ __global__ void __launch_bounds__(kThreads)
     if (!pool) return;  // uniform over the CTA
 
     // Column sums of the block in fp32 and a fixed order (a lane's rows in
-    // order, then the lanes in order), then the mean.
-    float acc[8];
+    // order, then the lanes in order), then the mean.  Q is pooled over the
+    // block's 128 rows.  K is pooled over its key blocks: the same 128 rows,
+    // or with 64-row key blocks each half on its own (row lane rl holds rows
+    // rl + i * kRowLanes, and kRowLanes divides 64, so rows 0-63 are the first
+    // half of every lane's rows).
+    const int parts = (tensor == 1 && g.block_kv == 64) ? 2 : 1;  // uniform over the CTA
+    constexpr int kHalf = kRowsPerThread / 2;
+    static_assert(64 % kRowLanes == 0 && kRowsPerThread % 2 == 0, "64-row halves must split the row lanes");
+    for (int part = 0; part < parts; ++part) {
+      float acc[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
 #pragma unroll
-    for (int i = 0; i < kRowsPerThread; ++i) {
-      const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        if (parts == 2 && (i < kHalf) != (part == 0)) continue;
+        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        acc[2 * c] += Dec::lo(w[c]);
-        acc[2 * c + 1] += Dec::hi(w[c]);
+        for (int c = 0; c < 4; ++c) {
+          acc[2 * c] += Dec::lo(w[c]);
+          acc[2 * c + 1] += Dec::hi(w[c]);
+        }
       }
-    }
+      if (part > 0) __syncthreads();  // the previous part's sums have been read
 #pragma unroll
-    for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
-    __syncthreads();
-    if (threadIdx.x < D) {
-      float sum = 0.f;
+      for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
+      __syncthreads();
+      if (threadIdx.x < D) {
+        float sum = 0.f;
 #pragma unroll 4
-      for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
-      float* out = tensor == 0 ? pooled_q : pooled_k;
-      const size_t idx =
-          ((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x;
-      out[idx] = sum * (1.0f / RF_BLOCK);
+        for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
+        size_t idx;
+        if (tensor == 0)
+          idx = ((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x;
+        else
+          idx = ((size_t)head * g.pooled_k_total + (size_t)(s.poolk_off + parts * (b - s.n_pb) + part)) * D +
+                threadIdx.x;
+        (tensor == 0 ? pooled_q : pooled_k)[idx] = sum * (parts == 2 ? 1.0f / 64 : 1.0f / RF_BLOCK);
+      }
     }
   }
 }

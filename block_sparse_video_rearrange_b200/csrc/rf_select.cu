@@ -12,9 +12,11 @@
 //
 // Two kernels:
 //  1. rf_scores_kernel: per sparse sequence and query head n, the fp32 matrix
-//     scores[i][j] = qbar[n][i] . kbar[n / G][j] (128 x 128 or 64 x 64
-//     tiles, 8 x 8 or 4 x 4 per thread, D chunks double-buffered through
-//     shared memory).
+//     scores[i][j] = qbar[n][i] . kbar[n / G][j] over the nb query blocks and
+//     the nbk key blocks (nbk = nb, or 2 nb with blockShape 128 x 64, whose
+//     key blocks of 64 rows are pooled over their own rows; [API] "Formula":
+//     blocks of blockShapeX x blockShapeY) (128 x 128 or 64 x 64 tiles, 8 x 8
+//     or 4 x 4 per thread, D chunks double-buffered through shared memory).
 //  2. rf_topk_kernel: one warp per selectIdx row.  Keys are the scores mapped
 //     to order-preserving 32-bit integers, held in registers (32 lanes x M).
 //     A bitwise radix select (over the bits below the keys' common prefix)
@@ -47,23 +49,23 @@ __global__ void __launch_bounds__(256, 2)
   // Decode blockIdx.x into (instance, head, tile row, tile col) over the
   // non-dense instances in order.
   int rem = blockIdx.x;
-  int si = -1, tiles = 0;
+  int si = -1, tiles_r = 0, tiles_c = 0;
   for (int i = 0; i < g.n_seqs; ++i) {
     const RfSeqDev& s = g.seq[i];
     if (s.dense) continue;
-    const int tn = (s.nb + kTile - 1) / kTile;
-    const int cnt = g.n1 * tn * tn;
-    if (rem < cnt) { si = i; tiles = tn; break; }
+    const int tr_n = (s.nb + kTile - 1) / kTile, tc_n = (s.nbk + kTile - 1) / kTile;
+    const int cnt = g.n1 * tr_n * tc_n;
+    if (rem < cnt) { si = i; tiles_r = tr_n; tiles_c = tc_n; break; }
     rem -= cnt;
   }
   if (si < 0) return;
   const RfSeqDev& s = g.seq[si];
-  const int n = rem / (tiles * tiles);
-  const int tr = (rem / tiles) % tiles;
-  const int tc = rem % tiles;
+  const int n = rem / (tiles_r * tiles_c);
+  const int tr = (rem / tiles_c) % tiles_r;
+  const int tc = rem % tiles_c;
   const int gk = n / (g.n1 / g.n2);
   const float* A = pq + ((size_t)n * g.pooled_total + s.pool_off) * g.d;
-  const float* B = pk + ((size_t)gk * g.pooled_total + s.pool_off) * g.d;
+  const float* B = pk + ((size_t)gk * g.pooled_k_total + s.poolk_off) * g.d;
   const int i0 = tr * kTile, j0 = tc * kTile;
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
 
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(256, 2)
       pa[rep] = make_float4(0.f, 0.f, 0.f, 0.f);
       pb[rep] = pa[rep];
       if (i0 + row < s.nb) pa[rep] = *reinterpret_cast<const float4*>(A + (size_t)(i0 + row) * g.d + k0 + 4 * c4);
-      if (j0 + row < s.nb) pb[rep] = *reinterpret_cast<const float4*>(B + (size_t)(j0 + row) * g.d + k0 + 4 * c4);
+      if (j0 + row < s.nbk) pb[rep] = *reinterpret_cast<const float4*>(B + (size_t)(j0 + row) * g.d + k0 + 4 * c4);
     }
   };
   auto stash = [&](int buf) {
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(256, 2)
     if (c + 1 < chunks) stash(buf ^ 1);
     __syncthreads();
   }
-  float* C = scores + s.score_off + (size_t)n * s.nb * s.nb;
+  float* C = scores + s.score_off + (size_t)n * s.nb * s.nbk;
 #pragma unroll
   for (int x = 0; x < TT; ++x) {
     const int i = i0 + (x >> 2) * 64 + ty * 4 + (x & 3);
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
     for (int y = 0; y < TT; ++y) {
       const int j = j0 + (y >> 2) * 64 + tx * 4 + (y & 3);
-      if (j < s.nb) C[(size_t)i * s.nb + j] = acc[x][y];
+      if (j < s.nbk) C[(size_t)i * s.nbk + j] = acc[x][y];
     }
   }
 }
@@ -142,7 +144,7 @@ __device__ __forceinline__ uint32_t rf_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <int M>  // keys per lane: nb <= 32 * M
+template <int M>  // keys per lane: nbk <= 32 * M
 __global__ void __launch_bounds__(256)
     rf_topk_kernel(const RfGeomDev g, const float* __restrict__ scores, int32_t* __restrict__ sel_idx,
                    int32_t* __restrict__ sel_num) {
@@ -153,25 +155,25 @@ __global__ void __launch_bounds__(256)
   const int tb = warp / g.n1, n = warp % g.n1;
   const RfSeqDev& s = g.seq[rf_seq_of_qblk(g, tb)];
   const int b = tb - s.qblk_off;
-  const int nblk = s.n_pb + s.nb;
+  const int nkv = s.npk + s.nbk;  // key blocks of the sequence
   int32_t* row = sel_idx + (size_t)warp * g.max_kv;
-  const int i = b - s.n_pb;
+  const int i = b - s.n_pb;       // query side: 128-row blocks
 
-  if (s.dense || b < s.n_pb || i < s.ns || s.k >= s.nb) {
-    for (int c = lane; c < g.max_kv; c += 32) row[c] = c < nblk ? c : -1;
-    if (lane == 0) sel_num[warp] = nblk;
+  if (s.dense || b < s.n_pb || i < s.ns || s.kk >= s.nbk) {
+    for (int c = lane; c < g.max_kv; c += 32) row[c] = c < nkv ? c : -1;
+    if (lane == 0) sel_num[warp] = nkv;
     return;
   }
 
   // Keys of this row; absent slots hold 0, below every real key.
-  const float* sc = scores + s.score_off + ((size_t)n * s.nb + i) * s.nb;
+  const float* sc = scores + s.score_off + ((size_t)n * s.nb + i) * s.nbk;
   uint32_t key[M];
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     const int j = lane + 32 * m;
-    key[m] = j < s.nb ? rf_key(sc[j]) : 0u;
+    key[m] = j < s.nbk ? rf_key(sc[j]) : 0u;
   }
-  const int k = s.k;
+  const int k = s.kk;
   unsigned long long sel = 0;  // bit m: block lane + 32m is kept
   if (k > 0) {
     // Largest T with #{key >= T} >= k, one bit at a time from the top.  All
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(256)
     uint32_t kmax = 0u, kmin = 0xFFFFFFFFu;
 #pragma unroll
     for (int m = 0; m < M; ++m)
-      if (lane + 32 * m < s.nb) {
+      if (lane + 32 * m < s.nbk) {
         kmax = max(kmax, key[m]);
         kmin = min(kmin, key[m]);
       }
@@ -217,16 +219,16 @@ __global__ void __launch_bounds__(256)
   // First-frame sinks.
 #pragma unroll
   for (int m = 0; m < M; ++m)
-    if (lane + 32 * m < s.ns) sel |= 1ull << m;
+    if (lane + 32 * m < s.nsk) sel |= 1ull << m;
 
-  for (int c = lane; c < s.n_pb; c += 32) row[c] = c;
-  int pos = s.n_pb;
+  for (int c = lane; c < s.npk; c += 32) row[c] = c;
+  int pos = s.npk;
   const uint32_t lt_mask = (1u << lane) - 1u;
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     const bool on = (sel >> m) & 1ull;
     const uint32_t ball = __ballot_sync(0xffffffffu, on);
-    if (on) row[pos + __popc(ball & lt_mask)] = s.n_pb + lane + 32 * m;
+    if (on) row[pos + __popc(ball & lt_mask)] = s.npk + lane + 32 * m;
     pos += __popc(ball);
   }
   for (int c = pos + lane; c < g.max_kv; c += 32) row[c] = -1;
@@ -245,10 +247,10 @@ rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_nu
   // per SM), else 64 x 64 tiles for more parallelism.
   long long tiles64 = 0, tiles128 = 0;
   for (int i = 0; i < g.n_seqs; ++i) {
-    if (g.seq[i].dense) continue;
-    const long long t64 = (g.seq[i].nb + 63) / 64, t128 = (g.seq[i].nb + 127) / 128;
-    tiles64 += (long long)g.n1 * t64 * t64;
-    tiles128 += (long long)g.n1 * t128 * t128;
+    const RfSeqDev& s = g.seq[i];
+    if (s.dense) continue;
+    tiles64 += (long long)g.n1 * ((s.nb + 63) / 64) * ((s.nbk + 63) / 64);
+    tiles128 += (long long)g.n1 * ((s.nb + 127) / 128) * ((s.nbk + 127) / 128);
   }
   if (tiles64 > 0) {
     int dev = 0, sms = 148;
@@ -263,10 +265,11 @@ rf_status_t rf_launch_select(const rf_plan* p, int32_t* sel_idx, int32_t* sel_nu
   const long long rows = (long long)g.t_qblk * g.n1;
   if (rows == 0) return RF_OK;
   const unsigned blocks = (unsigned)((rows * 32 + 255) / 256);
-  if (g.max_nb <= 256)       rf_topk_kernel<8><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
-  else if (g.max_nb <= 512)  rf_topk_kernel<16><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
-  else if (g.max_nb <= 640)  rf_topk_kernel<20><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
-  else if (g.max_nb <= 1024) rf_topk_kernel<32><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
-  else                       rf_topk_kernel<64><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  if (g.max_nbk <= 256)       rf_topk_kernel<8><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nbk <= 512)  rf_topk_kernel<16><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nbk <= 640)  rf_topk_kernel<20><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nbk <= 1024) rf_topk_kernel<32><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else if (g.max_nbk <= 1280) rf_topk_kernel<40><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
+  else                        rf_topk_kernel<64><<<blocks, 256, 0, st>>>(g, scores, sel_idx, sel_num);
   return rf_check_launch("rf_topk_kernel");
 }

@@ -62,7 +62,7 @@ class HostPipeline:
     def __init__(self, seqs: Sequence[Tuple[int, int, int, int]], n1: int, n2: int, d: int,
                  layout: str = "BNSD", dtype: str = "bf16", sparsity: float = 0.8, batch: int = 1,
                  chunks: Optional[int] = None, order: str = "tile", precision: str = "native",
-                 device=None):
+                 device=None, block_kv: int = 128):
         self.chunks = chunks if chunks is not None else default_chunks(n2)
         if n2 % self.chunks or n1 % self.chunks:
             raise ValueError(f"{self.chunks} chunks do not divide the heads ({n1}, {n2})")
@@ -71,7 +71,7 @@ class HostPipeline:
         self.layout, self.n1, self.n2, self.d = layout, n1, n2, d
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.plan = rf.Plan(seqs, n1 // self.chunks, n2 // self.chunks, d, layout, dtype, sparsity, batch=batch,
-                            order=order, precision=precision)
+                            order=order, precision=precision, block_kv=block_kv)
         p = self.plan
         self.sets = []
         for _ in range(2 if self.chunks > 1 else 1):

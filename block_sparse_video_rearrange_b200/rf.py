@@ -60,7 +60,8 @@ class PlanInfo(ctypes.Structure):
                 ("ws_q8", ctypes.c_int64), ("ws_k8", ctypes.c_int64),
                 ("ws_q_scale", ctypes.c_int64), ("ws_k_scale", ctypes.c_int64),
                 ("ws_q_mx", ctypes.c_int64), ("ws_k_mx", ctypes.c_int64), ("ws_v_mx", ctypes.c_int64),
-                ("ws_v8", ctypes.c_int64), ("ws_v_exp", ctypes.c_int64)]
+                ("ws_v8", ctypes.c_int64), ("ws_v_exp", ctypes.c_int64),
+                ("pooled_k_blocks", ctypes.c_int64)]
 
 
 class PlanOptions(ctypes.Structure):
@@ -72,7 +73,9 @@ class SeqInfo(ctypes.Structure):
     _fields_ = [("row_offset", ctypes.c_int64), ("length", ctypes.c_int64), ("lp", ctypes.c_int64),
                 ("sparse", ctypes.c_int64), ("promoted", ctypes.c_int64), ("n_pb", ctypes.c_int32),
                 ("nb", ctypes.c_int32), ("ns", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("qblk_offset", ctypes.c_int32), ("dense", ctypes.c_int32)]
+                ("qblk_offset", ctypes.c_int32), ("dense", ctypes.c_int32),
+                ("n_pb_kv", ctypes.c_int32), ("nb_kv", ctypes.c_int32), ("ns_kv", ctypes.c_int32),
+                ("k_kv", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -387,7 +390,8 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          layout: str = "BNSD", scale: Optional[float] = None,
                          plan: Optional[Plan] = None, bufs: Optional[Buffers] = None,
                          order: str = "tile", precision: str = "native",
-                         chunks: Optional[int] = None, check: bool = True) -> torch.Tensor:
+                         chunks: Optional[int] = None, check: bool = True,
+                         block_kv: int = 128) -> torch.Tensor:
     """User-level call: RainFusion v2 block-sparse attention of q, k, v (original token order).
 
     q, k, v may live on the host (pinned or not) or on the GPU; the result is
@@ -396,8 +400,11 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     (prefix_len, t, h, w) per sequence (BNSD: one for the whole batch).
     `order` is the token order of the aligned video ("tile", or "frame_pair"
     for 2x8x8 blocks over frame pairs) and `precision` the kernel precision
-    ("native", "mix" for E4M3 Q K^T, or "mxfp4" for MXFP4 attention with UOS
-    scaling and PNQ); both are ignored when `plan` is given.
+    ("native", "mix" for E4M3 Q K^T, "fp8" for E4M3 Q K^T and P V, or "mxfp4"
+    for MXFP4 attention with UOS scaling and PNQ), and `block_kv` the key block
+    length (128, or 64 for aclnnRainFusionAttention's blockShape 128 x 64, whose
+    selection ranks 64-row key blocks; native precision); all three are ignored
+    when `plan` is given.
 
     Host inputs run through `pipeline.HostPipeline` (made once per problem
     shape and kept): head chunks whose copies to and from the GPU overlap
@@ -421,10 +428,11 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
             n1, n2, d, batch = q.shape[1], k.shape[1], q.shape[2], 1
         dev = torch.device("cuda", torch.cuda.current_device())
         key = (tuple(map(tuple, seqs)), n1, n2, d, layout, dtype, float(sparsity), batch, order, precision,
-               chunks, dev.index)
+               chunks, dev.index, block_kv)
         pipe = _PIPELINES.pop(key, None)
         if pipe is None:
-            pipe = HostPipeline(seqs, n1, n2, d, layout, dtype, sparsity, batch, chunks, order, precision, dev)
+            pipe = HostPipeline(seqs, n1, n2, d, layout, dtype, sparsity, batch, chunks, order, precision, dev,
+                                block_kv)
             while len(_PIPELINES) >= _PIPELINES_KEPT:      # drop the least recently used shape
                 _PIPELINES.pop(next(iter(_PIPELINES)))
         _PIPELINES[key] = pipe                               # most recently used last
@@ -437,10 +445,10 @@ def rainfusion_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if plan is None:
         if layout == "BNSD":
             plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[3], "BNSD", dtype, sparsity, batch=q.shape[0],
-                        order=order, precision=precision)
+                        order=order, precision=precision, block_kv=block_kv)
         else:
             plan = Plan(seqs, q.shape[1], k.shape[1], q.shape[2], "TND", dtype, sparsity, order=order,
-                        precision=precision)
+                        precision=precision, block_kv=block_kv)
     host = not q.is_cuda
     dev = torch.device("cuda", torch.cuda.current_device()) if host else q.device
     if bufs is None:

@@ -123,7 +123,7 @@ typedef struct {
   int64_t pooled_blocks;   /* total sparse blocks over sequences (block means per head) */
   int64_t kept_flops_upper;/* 4*D*rows_q*rows_kv over the maximal selection (for reporting) */
   int64_t ws_pooled_q;     /* byte offset in ws of the Q block means, fp32 [n1][pooled_blocks][d] */
-  int64_t ws_pooled_k;     /* byte offset in ws of the K block means, fp32 [n2][pooled_blocks][d] */
+  int64_t ws_pooled_k;     /* byte offset in ws of the K block means, fp32 [n2][pooled_k_blocks][d] */
   int32_t n_seqs;          /* sequences (BNSD: batch elements) */
   int32_t n1, n2, d;
   int32_t precision;       /* rf_precision_t of the plan */
@@ -148,6 +148,9 @@ typedef struct {
    * RF_PRECISION_MXFP4 at head dim 128 stores its E4M3-carried V' in ws_v8 in
    * the same transposed layout, with no exponents (ws_v_exp = -1). */
   int64_t ws_v8, ws_v_exp;
+  /* key block means per key/value head: pooled_blocks, or 2 * pooled_blocks
+   * with blockShape 128 x 64 (the means of the 64-row key blocks) */
+  int64_t pooled_k_blocks;
 } rf_plan_info_t;
 
 /* Per-sequence geometry under suffix promotion ([UG] "Geometry handling"). */
@@ -163,6 +166,11 @@ typedef struct {
   int32_t k;           /* ranked key blocks kept per sparse query block */
   int32_t qblk_offset; /* first global query block of this sequence */
   int32_t dense;       /* 1: the sequence runs dense (nb < 32, [UG]) */
+  /* Key-side counts of the selection.  128-row key blocks: n_pb, nb, ns, k.
+   * 64-row key blocks (blockShape 128 x 64): ceil(lp / 64) prefix key blocks,
+   * 2 * nb sparse key blocks, min(nb_kv, ceil(h8 * w8 / 64)) first-frame sinks
+   * and k_kv = ceil((1 - sparsity) * nb_kv) ranked blocks kept (nb_kv if dense). */
+  int32_t n_pb_kv, nb_kv, ns_kv, k_kv;
 } rf_seq_info_t;
 
 typedef struct rf_plan rf_plan_t;
@@ -180,10 +188,8 @@ typedef struct rf_plan rf_plan_t;
  *                 rows: ceil(lp / 64) prefix key blocks from row 0, the last
  *                 possibly partial, then 2 * nb from row lp; native precision
  *                 only).  With 128 x 64, selectIdx entries and max_kv_blocks
- *                 count 64-row key blocks, the selection step (which ranks
- *                 128-row blocks) and rf_forward return RF_ERR_UNSUPPORTED, and
- *                 rf_block_sparse_attn takes a caller-made selectIdx.  Others:
- *                 RF_ERR_UNSUPPORTED.
+ *                 count 64-row key blocks, and the selection step ranks them
+ *                 (see rf_pool_select).  Others: RF_ERR_UNSUPPORTED.
  *   out         : receives the plan; free with rf_plan_destroy.
  * Errors: RF_ERR_INVALID_ARG for a broken constraint (out untouched). */
 RF_API rf_status_t rf_plan_create(const rf_seq_geom_t* seqs, int32_t n_seqs, int32_t batch,
@@ -328,7 +334,11 @@ RF_API rf_status_t rf_quantize(const rf_plan_t* plan, const void* q_r, const voi
  * video query blocks keep every prefix block, the first-frame sink blocks,
  * and the k key blocks with the highest block-mean dot product (ties: lower
  * block index), k = ceil((1 - sparsity) * nb).  Sequences with nb < 32 are
- * dense.  Deterministic (fp32 scores, no atomics). */
+ * dense.  With blockShape 128 x 64 the key blocks hold 64 rows ([API]
+ * "Formula": blocks of blockShapeX x blockShapeY): the 128-row query block
+ * means are ranked against 64-row key block means, and the prefix, sink and
+ * kept counts are rf_seq_info_t's n_pb_kv, ns_kv and k_kv.  Deterministic
+ * (fp32 scores, no atomics). */
 RF_API rf_status_t rf_pool_select(const rf_plan_t* plan, const void* q_r, const void* k_r,
                            int32_t* select_idx, int32_t* select_num, void* ws,
                            size_t ws_bytes, rf_pool_mode_t pool_mode, rf_stream_t stream);

@@ -42,10 +42,10 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
 
 
 def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "from_ws",
-            order: str = "tile", precision: str = "native") -> Dict[str, object]:
+            order: str = "tile", precision: str = "native", block_kv: int = 128) -> Dict[str, object]:
     """Whole path through the C ABI, one call per step; returns host copies of every result."""
     plan = rf.Plan(seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch, order=order,
-                   precision=precision)
+                   precision=precision, block_kv=block_kv)
     q, k, v = (to_device(b, w.dtype) for b in bits)
     b = rf.Buffers(plan)
     scale = 1.0 / math.sqrt(w.d)
@@ -57,10 +57,10 @@ def run_gpu(w: synth.Workload, bits: Sequence[np.ndarray], pool_mode: str = "fro
     assert st == 0, (st, flags)
     torch.cuda.synchronize()
     ws8 = b.ws.view(torch.uint8)
-    pooled = int(plan.info.pooled_blocks)
+    pooled, pooled_k = int(plan.info.pooled_blocks), int(plan.info.pooled_k_blocks)
     oq, ok_ = int(plan.info.ws_pooled_q), int(plan.info.ws_pooled_k)
     pq = ws8[oq:oq + w.n1 * pooled * w.d * 4].view(torch.float32).reshape(w.n1, pooled, w.d).cpu().numpy()
-    pk = ws8[ok_:ok_ + w.n2 * pooled * w.d * 4].view(torch.float32).reshape(w.n2, pooled, w.d).cpu().numpy()
+    pk = ws8[ok_:ok_ + w.n2 * pooled_k * w.d * 4].view(torch.float32).reshape(w.n2, pooled_k, w.d).cpu().numpy()
     out = dict(plan=plan, q_r=to_bits(b.q_r), k_r=to_bits(b.k_r), v_r=to_bits(b.v_r), o_r=to_bits(b.o_r),
                o=to_bits(b.o), idx=b.select_idx.cpu().numpy(), num=b.select_num.cpu().numpy(),
                pooled_q=pq, pooled_k=pk, scale=scale)
@@ -264,26 +264,30 @@ def check_permutation(p: orc.Problem, bits: Sequence[np.ndarray], gpu: Dict[str,
     assert np.array_equal(orc.inverse_rearrange(p, gpu["o_r"]), gpu["o"]), "inverse permutation differs"
 
 
-def oracle_pooled(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray]):
-    """Per sequence instance: [heads, nb, D] float64 means of the oracle-rearranged Q and K."""
+def oracle_pooled(p: orc.Problem, w: synth.Workload, rbits: Sequence[np.ndarray], block_kv: int = 128):
+    """Per sequence instance: float64 means of the oracle-rearranged Q ([heads, nb, D],
+    128-row query blocks) and K ([heads, S / block_kv, D], key blocks of block_kv rows)."""
     qf = synth.bits_to_float64(rbits[0], w.dtype)
     kf = synth.bits_to_float64(rbits[1], w.dtype)
-    return orc.pooled_means(p, qf, w.n1), orc.pooled_means(p, kf, w.n2)
+    return orc.pooled_means(p, qf, w.n1), orc.pooled_means(p, kf, w.n2, block_kv)
 
 
 def check_pooled(p: orc.Problem, qbars, kbars, gpu) -> None:
-    off = 0
+    offq = offk = 0
     for (s, g), qb, kb in zip(p.sequences(), qbars, kbars):
-        gq = gpu["pooled_q"][:, off:off + g.nb]
-        gk = gpu["pooled_k"][:, off:off + g.nb]
+        gq = gpu["pooled_q"][:, offq:offq + qb.shape[1]]
+        gk = gpu["pooled_k"][:, offk:offk + kb.shape[1]]
         for ref, got in ((qb, gq), (kb, gk)):
+            assert got.shape == ref.shape
             if ref.size:
                 err = np.max(np.abs(got - ref)) / max(1e-30, np.max(np.abs(ref)))
                 assert err < POOL_REL, f"pooled means rel err {err}"
-        off += g.nb
+        offq += qb.shape[1]
+        offk += kb.shape[1]
 
 
-def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int, int]] | None = None) -> Dict[str, int]:
+def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int, int]] | None = None,
+                    block_kv: int = 128) -> Dict[str, int]:
     """selectIdx / selectNum against the oracle's selection.  Returns counters.
 
     selectNum must equal the oracle's on every row (bit-exact).  A selectIdx row
@@ -291,7 +295,7 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
     non-sink video blocks, completed with the best-scoring sinks) must be a
     valid top-k of the oracle's float64 scores, in that every block in T scores
     at least as high as every video block outside T, up to TIE_REL relative."""
-    idx_o, num_o = orc.select(p, qbars, kbars)
+    idx_o, num_o = orc.select(p, qbars, kbars, block_kv)
     idx_g, num_g = gpu["idx"], gpu["num"]
     assert idx_g.shape == idx_o.shape and num_g.shape == num_o.shape
     table = orc.qblock_table(p)
@@ -311,18 +315,19 @@ def check_selection(p: orc.Problem, qbars, kbars, gpu, rows: Sequence[Tuple[int,
             stats["exact"] += 1
             continue
         s, g, qb = table[t]
+        kb = orc.key_blocks(g, block_kv)
         assert not g.dense and qb >= g.n_pb + g.ns, f"dense row (t={t}, n={n}) differs"
-        assert a[:g.n_pb] == list(range(g.n_pb)), (t, n, a[:g.n_pb])
+        assert a[:kb.n_pb] == list(range(kb.n_pb)), (t, n, a[:kb.n_pb])
         si = seq_pos[s]
         sc = qbars[si][n, qb - g.n_pb] @ kbars[si][n // G].T
-        video = [j - g.n_pb for j in a[g.n_pb:]]
-        sinks = set(range(g.ns))
+        video = [j - kb.n_pb for j in a[kb.n_pb:]]
+        sinks = set(range(kb.ns))
         assert sinks <= set(video), (t, n)
         chosen = [j for j in video if j not in sinks]
-        assert len(chosen) <= g.k, (t, n, len(chosen), g.k)
-        best_sinks = sorted(sinks, key=lambda j: (-sc[j], j))[:g.k - len(chosen)]
+        assert len(chosen) <= kb.k, (t, n, len(chosen), kb.k)
+        best_sinks = sorted(sinks, key=lambda j: (-sc[j], j))[:kb.k - len(chosen)]
         top = set(chosen) | set(best_sinks)
-        rest = [j for j in range(g.nb) if j not in top]
+        rest = [j for j in range(kb.nb) if j not in top]
         if top and rest:
             lo = min(top, key=lambda j: sc[j])
             hi = max(rest, key=lambda j: sc[j])

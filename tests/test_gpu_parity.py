@@ -513,6 +513,58 @@ def test_kv64_random_selection_against_the_oracle(name):
     parity.check_attention(p, w, rbits, got, block_kv=64)
 
 
+@pytest.mark.parametrize("name", KV64 + ["batch2_d64", "dense", "s_one"])
+def test_kv64_selection_small_full_parity(name):
+    """blockShape 128 x 64 end to end (reading R26): K pooled over 64-row key blocks,
+    those ranked against the 128-row query means, the attention on that selection."""
+    w = SMALL[name]
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, block_kv=64)
+    parity.check_permutation(p, bits, gpu)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits, 64)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu, block_kv=64)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 100)
+    parity.check_attention(p, w, rbits, gpu, block_kv=64)
+    if name == "dense":
+        assert np.all(gpu["num"] == orc.kv_block_count(p.geoms[0], 64))
+
+
+def test_kv64_recompute_forward_and_noalloc_equal_the_step_calls():
+    w = SMALL["tnd_gqa_small"]
+    bits = synth.generate_qkv(w)
+    a = parity.run_gpu(w, bits, block_kv=64)
+    b = parity.run_gpu(w, bits, pool_mode="recompute", block_kv=64)
+    assert np.array_equal(a["pooled_k"], b["pooled_k"])
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["num"], b["num"])
+    assert np.array_equal(a["o"], b["o"])
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, block_kv=64)
+    bufs = rf.Buffers(plan)
+    q, k, v = (parity.to_device(x, w.dtype) for x in bits)
+    out = rf.forward(plan, q, k, v, bufs)
+    torch.cuda.synchronize()
+    assert np.array_equal(parity.to_bits(out), a["o"])
+
+
+@pytest.mark.parametrize("name,s", [("wan", None), ("aligned", 0.8)])
+def test_kv64_full_size_parity(name, s):
+    """The 128 x 64 path at full size in the bench's launch configuration: 64-row K
+    means and the selection over every row, the attention on sampled items."""
+    w = synth.workload(name, s)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    gpu = parity.run_gpu(w, bits, block_kv=64)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qbars, kbars = parity.oracle_pooled(p, w, rbits, 64)
+    parity.check_pooled(p, qbars, kbars, gpu)
+    stats = parity.check_selection(p, qbars, kbars, gpu, block_kv=64)
+    assert stats["near_tie"] <= max(1, stats["rows"] // 1000), stats
+    items = parity.sample_items(p, np.random.default_rng(8), per_kind=3)
+    parity.check_attention(p, w, rbits, gpu, items, block_kv=64)
+
+
 # ------------------------------------------------------------------------------------------
 # Precision "fp8" (user guide "Configuration": precision "fp8"; reading R24): E4M3 Q K^T as
 # in mix, E4M3 V' on power-of-two scales, probabilities rounded to E4M3 for P V.  Codes and

@@ -81,3 +81,30 @@ def test_changed_select_num_fails():
     bad_idx[t, n, bad_num[t, n]] = -1
     with pytest.raises(AssertionError):
         parity.check_selection(p, qb, kb, dict(idx=bad_idx, num=bad_num))
+
+
+def test_kv64_checker_accepts_the_oracle_and_rejects_a_gap_swap():
+    """The same rule over 64-row key blocks (reading R26): the oracle's own selection
+    passes exactly; swapping the best kept key block for the worst dropped one fails."""
+    w = synth.Workload("chk64", "BNSD", "bf16", 1, (synth.SeqSpec(100, 9, 16, 32),), 2, 1, 64, 0.8, 42)
+    bits = synth.generate_qkv(w)
+    p = parity.problem(w)
+    rbits = [orc.rearrange(p, x) for x in bits]
+    qb, kb = parity.oracle_pooled(p, w, rbits, 64)
+    assert kb[0].shape[1] == 2 * p.geoms[0].nb
+    idx, num = orc.select(p, qb, kb, 64)
+    st = parity.check_selection(p, qb, kb, dict(idx=idx.copy(), num=num.copy()), block_kv=64)
+    assert st["exact"] == st["rows"]
+    g = p.geoms[0]
+    k64 = orc.key_blocks(g, 64)
+    t, n = g.n_pb + g.ns + 5, 1
+    sc = qb[0][n, t - g.n_pb] @ kb[0][0].T
+    row = idx[t, n, :num[t, n]].tolist()
+    video = [j - k64.n_pb for j in row[k64.n_pb:]]
+    kept = [j for j in video if j >= k64.ns]
+    dropped = [j for j in range(k64.nb) if j not in video]
+    lo, hi = max(kept, key=lambda j: sc[j]), min(dropped, key=lambda j: sc[j])
+    bad = idx.copy()
+    bad[t, n, :len(row)] = sorted(row[:k64.n_pb] + [k64.n_pb + j for j in (set(video) - {lo}) | {hi}])
+    with pytest.raises(AssertionError):
+        parity.check_selection(p, qb, kb, dict(idx=bad, num=num.copy()), block_kv=64)

@@ -34,11 +34,12 @@ def _cuda():
         pytest.skip("needs a GPU")
 
 
-@pytest.mark.parametrize("name", list(CASES))
-def test_noalloc_selection_equals_workspace_selection_twice(name):
+@pytest.mark.parametrize("name,block_kv", [(n, 128) for n in CASES] + [("tnd_gqa_small", 64), ("wan", 64)])
+def test_noalloc_selection_equals_workspace_selection_twice(name, block_kv):
     w = CASES[name]
     bits = synth.generate_qkv(w)
-    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch)
+    plan = rf.Plan(parity.seqs_of(w), w.n1, w.n2, w.d, w.layout, w.dtype, w.sparsity, batch=w.batch,
+                   block_kv=block_kv)
     assert plan.workspace_bytes <= 32 << 20
     q, k, v = (parity.to_device(x, w.dtype) for x in bits)
     b = rf.Buffers(plan)
