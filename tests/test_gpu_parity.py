@@ -548,6 +548,17 @@ def test_kv64_recompute_forward_and_noalloc_equal_the_step_calls():
     assert np.array_equal(parity.to_bits(out), a["o"])
 
 
+def test_kv64_user_call_with_host_tensors_equals_the_step_calls():
+    """rainfusion_attention(block_kv=64) on host tensors (the chunked host pipeline)
+    gives the step calls' output bit for bit."""
+    w = SMALL["batch2_d64"]
+    bits = synth.generate_qkv(w)
+    steps = parity.run_gpu(w, bits, block_kv=64)
+    q, k, v = (torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in bits)
+    out = rf.rainfusion_attention(q, k, v, parity.seqs_of(w), sparsity=w.sparsity, block_kv=64)
+    assert np.array_equal(out.view(torch.int16).numpy().view(np.uint16), steps["o"])
+
+
 @pytest.mark.parametrize("name,s", [("wan", None), ("aligned", 0.8)])
 def test_kv64_full_size_parity(name, s):
     """The 128 x 64 path at full size in the bench's launch configuration: 64-row K
