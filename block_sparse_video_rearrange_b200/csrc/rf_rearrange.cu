@@ -376,40 +376,55 @@ __global__ void __launch_bounds__(kThreads)
     // order, then the lanes in order), then the mean.  Q is pooled over the
     // block's 128 rows.  K is pooled over its key blocks: the same 128 rows,
     // or with 64-row key blocks each half on its own (row lane rl holds rows
-    // rl + i * kRowLanes, and kRowLanes divides 64, so rows 0-63 are the first
-    // half of every lane's rows).
-    const int parts = (tensor == 1 && g.block_kv == 64) ? 2 : 1;  // uniform over the CTA
-    constexpr int kHalf = kRowsPerThread / 2;
+    // rl + i * kRowLanes and kRowLanes divides 64, so the first half of every
+    // lane's rows is rows 0-63), summed into a second accumulator in the same
+    // pass so that no row value outlives its own addition.
+    const bool split = tensor == 1 && g.block_kv == 64;  // uniform over the CTA
     static_assert(64 % kRowLanes == 0 && kRowsPerThread % 2 == 0, "64-row halves must split the row lanes");
-    for (int part = 0; part < parts; ++part) {
-      float acc[8];
+    float acc[8], acc2[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+    for (int c = 0; c < 8; ++c) acc[c] = acc2[c] = 0.f;
 #pragma unroll
-      for (int i = 0; i < kRowsPerThread; ++i) {
-        if (parts == 2 && (i < kHalf) != (part == 0)) continue;
-        const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const uint32_t w[4] = {val[i].x, val[i].y, val[i].z, val[i].w};
+      const bool second = split && i >= kRowsPerThread / 2;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 4; ++c) {
+        if (second) {
+          acc2[2 * c] += Dec::lo(w[c]);
+          acc2[2 * c + 1] += Dec::hi(w[c]);
+        } else {
           acc[2 * c] += Dec::lo(w[c]);
           acc[2 * c + 1] += Dec::hi(w[c]);
         }
       }
-      if (part > 0) __syncthreads();  // the previous part's sums have been read
+    }
 #pragma unroll
-      for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
+    for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc[c];
+    __syncthreads();
+    const float inv_rows = split ? 1.0f / 64 : 1.0f / RF_BLOCK;
+    if (threadIdx.x < D) {
+      float sum = 0.f;
+#pragma unroll 4
+      for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
+      if (tensor == 0)
+        pooled_q[((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x] =
+            sum * inv_rows;
+      else
+        pooled_k[((size_t)head * g.pooled_k_total + (size_t)(s.poolk_off + (split ? 2 : 1) * (b - s.n_pb))) * D +
+                 threadIdx.x] = sum * inv_rows;
+    }
+    if (split) {
+      __syncthreads();  // the first half's sums have been read
+#pragma unroll
+      for (int c = 0; c < 8; ++c) red[rl][ch * 8 + c] = acc2[c];
       __syncthreads();
       if (threadIdx.x < D) {
         float sum = 0.f;
 #pragma unroll 4
         for (int l = 0; l < kRowLanes; ++l) sum += red[l][threadIdx.x];
-        size_t idx;
-        if (tensor == 0)
-          idx = ((size_t)head * g.pooled_total + (size_t)(s.pool_off + b - s.n_pb)) * D + threadIdx.x;
-        else
-          idx = ((size_t)head * g.pooled_k_total + (size_t)(s.poolk_off + parts * (b - s.n_pb) + part)) * D +
-                threadIdx.x;
-        (tensor == 0 ? pooled_q : pooled_k)[idx] = sum * (parts == 2 ? 1.0f / 64 : 1.0f / RF_BLOCK);
+        pooled_k[((size_t)head * g.pooled_k_total + (size_t)(s.poolk_off + 2 * (b - s.n_pb) + 1)) * D +
+                 threadIdx.x] = sum * inv_rows;
       }
     }
   }
