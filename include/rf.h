@@ -118,7 +118,8 @@ typedef struct {
 typedef struct {
   int64_t rows_total;      /* rows per head: BNSD B*L, TND T */
   int64_t t_qblk;          /* total query blocks over all sequences ([API] selectIdx dim 0) */
-  int64_t max_kv_blocks;   /* selectIdx dim 2 = max over sequences of n_pb + nb */
+  int64_t max_kv_blocks;   /* selectIdx dim 2 = max over sequences of n_pb_kv + nb_kv (n_pb + nb
+                            * with 128-row key blocks) */
   int64_t workspace_bytes; /* device workspace every call below needs */
   int64_t pooled_blocks;   /* total sparse blocks over sequences (block means per head) */
   int64_t kept_flops_upper;/* 4*D*rows_q*rows_kv over the maximal selection (for reporting) */
