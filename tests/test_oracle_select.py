@@ -249,3 +249,34 @@ def test_kv64_problem_select_pads_to_the_widest_sequence():
     tail = idx[p.geoms[0].n_blocks:]
     assert np.all(tail[:, :, widths[1]:] == -1)
     assert np.all(num[p.geoms[0].n_blocks:] == widths[1])
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(prefix=st.integers(0, 300), t=st.integers(1, 6), h=st.integers(8, 40), w=st.integers(8, 40),
+       s=st.sampled_from([0.0, 0.5, 0.8, 0.9, 1.0]), seed=st.integers(0, 1000))
+def test_kv64_selection_invariants_on_random_geometries(prefix, t, h, w, s, seed):
+    """Over random grids and sparsities: the key-side counts agree with kv_block_count,
+    dense rows list every key block, and every other row lists all prefix key blocks and
+    then exactly the sink key blocks together with the k best-scoring 64-row key blocks."""
+    g = rf.geometry(prefix, t, h, w, s)
+    kb = rf.key_blocks(g, 64)
+    assert kb.n_pb + kb.nb == rf.kv_block_count(g, 64)
+    if g.nb == 0:
+        return
+    rng = np.random.default_rng(seed)
+    qbar = rng.standard_normal((1, g.nb, 4))
+    kbar = rng.standard_normal((1, kb.nb, 4))
+    idx, num = rf.select_sequence(qbar, kbar, g, 64)
+    for qb in range(g.n_blocks):
+        row = idx[qb, 0, :num[qb, 0]].tolist()
+        i = qb - g.n_pb
+        if g.dense or qb < g.n_pb or i < g.ns:
+            assert row == list(range(kb.n_pb + kb.nb))
+            continue
+        assert row[:kb.n_pb] == list(range(kb.n_pb))
+        video = [b - kb.n_pb for b in row[kb.n_pb:]]
+        top = rf.topk_blocks(qbar[0, i] @ kbar[0].T, kb.k)
+        assert set(video) == set(top) | set(range(kb.ns))
