@@ -295,3 +295,28 @@ def test_keep_count_pins_reject_a_floor(monkeypatch):
     monkeypatch.setattr(rf.math, "ceil", _math.floor)
     wrong = [(p, t, h, w, s) for (p, t, h, w, s, nb, k) in PINNED_K if rf.geometry(p, t, h, w, s).k != k]
     assert len(wrong) >= 6, wrong
+
+
+# Key-side counts with 64-row key blocks (reading R26), worked out by hand for the same
+# configurations: n_pb64 = ceil(Lp / 64), nb64 = 2 nb, ns64 = min(nb64, ceil(h8 w8 / 64)),
+# k64 = ceil((1 - s) nb64 - 1e-6).
+PINNED_K64 = [
+    # (prefix, t, h, w, sparsity, n_pb64, nb64, ns64, k64)
+    (128, 9, 16, 32, 0.8, 2, 72, 8, 15),          # Tiny: Lp 128, first frame 512 tokens, 14.4 -> 15
+    (512, 21, 30, 52, 0.8, 142, 378, 18, 76),     # Wan2.2-shaped: Lp 9,080, 24 x 48 first frame, 75.6 -> 76
+    (256, 62, 24, 42, 0.5, 51, 930, 15, 465),     # MiniMax-H3-shaped: Lp 3,232, 24 x 40 first frame
+    (256, 62, 24, 42, 0.8, 51, 930, 15, 186),
+    (256, 62, 24, 42, 0.9, 51, 930, 15, 93),
+    (512, 21, 48, 80, 0.0, 8, 1260, 60, 1260),    # Aligned: Lp 512, 48 x 80 first frame
+    (512, 21, 48, 80, 0.5, 8, 1260, 60, 630),
+    (512, 21, 48, 80, 0.8, 8, 1260, 60, 252),
+    (512, 21, 48, 80, 0.9, 8, 1260, 60, 126),
+    (256, 13, 32, 48, 0.8, 4, 312, 24, 63),       # TND sequence 0: 62.4 -> 63
+    (384, 21, 24, 40, 0.8, 7, 314, 15, 63),       # TND sequence 1: Lp 448 (64 promoted), 62.8 -> 63
+]
+
+
+@pytest.mark.parametrize("p,t,h,w,s,npb,nb,ns,k", PINNED_K64)
+def test_key_blocks_of_64_rows_pinned_per_configuration(p, t, h, w, s, npb, nb, ns, k):
+    kb = rf.key_blocks(rf.geometry(p, t, h, w, s), 64)
+    assert (kb.n_pb, kb.nb, kb.ns, kb.k) == (npb, nb, ns, k)
